@@ -1,0 +1,167 @@
+/*
+ * sap.h -- C ABI of the B200 (sm_100a) packed causal attention library.
+ *
+ * The operation (HSAP / Sequence-Aware Parallelism paper page, abstract):
+ * causal attention over a *packed* sequence -- many documents laid end to end
+ * -- in which a token attends only to earlier (and its own) tokens of its own
+ * document, so that packing causes no cross-contamination.  The sequence is
+ * cut into P equal chunks as sequence parallelism would cut it; every
+ * (query-chunk, key/value-chunk) pair yields a partial output and its
+ * log-sum-exp ("partial attention computation", same abstract), and the
+ * partials are merged exactly, which by the equivalence stated in the
+ * sequence-parallelism explainer page (FAQ on equivalence with one device)
+ * gives the single-device result.  On one GPU the P chunks are simulated in
+ * place.
+ *
+ * Conventions used by every call
+ *   N      packed tokens;  cu_seqlens: int32[num_docs+1], cu[0] = 0,
+ *          non-decreasing, cu[num_docs] = N; document k is [cu[k], cu[k+1]).
+ *          Zero-length documents are allowed.
+ *   Q, O, dO, dQ : bf16, [N][hq][head_dim], contiguous (row = token).
+ *   K, V, dK, dV : bf16, [N][hkv][head_dim], contiguous.
+ *   LSE          : fp32, [hq][N], natural-log log-sum-exp of the scaled scores.
+ *   GQA          : query head h reads key/value head h / (hq / hkv).
+ *   Scores       : S_ij = softmax_scale * <q_i, k_j>, kept for doc(j) == doc(i)
+ *                  and j <= i (the diagonal is included).
+ *   Kernels support head_dim in {64, 128} and 128 x 128 tiles.
+ *
+ * Ownership: the caller owns every device buffer (inputs, outputs and the
+ * workspace).  The library owns only a plan: its host arrays and their device
+ * copy, released by sap_plan_destroy.  Device pointers must be 16-byte
+ * aligned.
+ *
+ * Streams: every device call is asynchronous on the given cudaStream_t
+ * (passed as void*, NULL = the legacy default stream).
+ *
+ * Errors: every int-returning call returns SAP_OK (0) or a negative SAP_ERR_*
+ * code; nothing is printed and no exception crosses the ABI.  A CUDA failure
+ * returns SAP_ERR_CUDA and the CUDA status is kept for sap_last_cuda_error().
+ * The kernels never trap: a pipeline wait that runs past its time limit sets a
+ * device error word, read (with a device synchronisation) by
+ * sap_device_status().
+ */
+#ifndef SAP_H_
+#define SAP_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+  SAP_OK = 0,
+  SAP_ERR_INVALID_ARG = -1,  /* null pointer, bad head counts, hq % hkv != 0, bad sizes        */
+  SAP_ERR_BAD_SEQLENS = -2,  /* cu[0] != 0, decreasing, or cu[num_docs] != N                   */
+  SAP_ERR_BAD_CHUNKS = -3,   /* P < 1, or P > 1 with N % P != 0 or (N/P) % block != 0          */
+  SAP_ERR_WORKSPACE = -4,    /* workspace missing or smaller than sap_workspace_size           */
+  SAP_ERR_CUDA = -5,         /* a CUDA runtime call failed (see sap_last_cuda_error)           */
+  SAP_ERR_DEVICE = -6,       /* the device error word is set (a kernel wait timed out)         */
+  SAP_ERR_UNSUPPORTED = -7,  /* head_dim not in {64,128}, or plan tiles other than 128 x 128   */
+  SAP_ERR_NOMEM = -8         /* host allocation failed                                         */
+};
+
+enum { SAP_TAG_FULL = 0, SAP_TAG_CAUSAL = 1, SAP_TAG_MASKED = 2 };
+enum { SAP_WS_FWD = 0, SAP_WS_BWD = 1 };
+
+typedef struct sap_plan_s* sap_plan_t;
+
+/* One non-empty (q-tile, kv-tile) pair of the packed causal mask.
+ *   tag FULL   : no pair of the block_m x block_n box is masked;
+ *   tag CAUSAL : the diagonal box (same token range) inside one document;
+ *   tag MASKED : anything else (document boundaries inside the box, or a
+ *                partial last tile).
+ * q_chunk = q_tile*block_m / C and kv_chunk = kv_tile*block_n / C, C = N / P. */
+typedef struct {
+  int32_t q_tile, kv_tile, q_chunk, kv_chunk, tag;
+} sap_item_t;
+
+/* Build a plan on the host (no device work).  Validates cu_seqlens and the
+ * chunking, lists the non-empty tiles in canonical order (q-tile ascending,
+ * then kv-tile ascending; bit-exact with the tile-list definition above), and
+ * derives the work schedule: forward units = (q-tile, kv-chunk) groups of
+ * items, partial slots for q-tiles that see more than one kv-chunk, the
+ * per-kv-tile lists for the backward pass, and heavy-first launch orders.
+ * P = num_chunks; with P = 1 any N >= 0 is accepted (a partial last tile is
+ * masked).  On success *out owns the plan. */
+int sap_plan(const int32_t* cu_seqlens_host, int32_t num_docs, int64_t total_tokens, int32_t num_chunks,
+             int32_t block_m, int32_t block_n, sap_plan_t* out);
+
+/* Canonical item list; host memory owned by the plan. */
+int sap_plan_items(sap_plan_t plan, const sap_item_t** items, int64_t* n_items);
+
+/* unmasked_pairs = sum over documents of L(L+1)/2 (per head);
+ * n_partial_slots = forward units that write a partial (q-tiles with > 1 unit);
+ * n_chunk_pairs = distinct (q_chunk, kv_chunk) pairs that hold an item. */
+int sap_plan_stats(sap_plan_t plan, int64_t* unmasked_pairs, int64_t* n_partial_slots, int32_t* n_chunk_pairs);
+
+/* Forward schedule, host memory owned by the plan:
+ *   units: int32[n_units][4] = (q_tile, item_begin, item_count, slot), slot = -1
+ *          when the unit writes O/LSE directly, else its partial slot;
+ *   order: int32[n_units], heavy-first (item_count descending, ties by index);
+ *   merges: int32[n_merges][3] = (q_tile, first_slot, n_slots). */
+int sap_plan_fwd_schedule(sap_plan_t plan, const int32_t** units, int64_t* n_units, const int32_t** order,
+                          const int32_t** merges, int64_t* n_merges);
+
+/* Backward schedule, host memory owned by the plan:
+ *   kv_units: int32[n_kv_units][3] = (kv_tile, first_entry, n_entries), heavy-first;
+ *   entries:  int32[n_items][2] = (q_tile, tag), grouped by kv tile, q-tile ascending. */
+int sap_plan_bwd_schedule(sap_plan_t plan, const int32_t** kv_units, int64_t* n_kv_units, const int32_t** entries);
+
+/* Copy the plan's device arrays to the current device on `stream`.  Called
+ * implicitly by the first device call that needs them; calling it first keeps
+ * the one host-to-device transfer out of later timed calls. */
+int sap_plan_upload(sap_plan_t plan, void* stream);
+
+void sap_plan_destroy(sap_plan_t plan);
+
+/* Workspace bytes for a call with these head counts (which = SAP_WS_FWD for
+ * sap_attn_fwd + sap_merge, SAP_WS_BWD for sap_attn_bwd).  The forward
+ * workspace holds the fp32 partial outputs and LSEs of the partial slots; the
+ * backward one holds the fp32 dQ accumulator and the per-row D and LSE*log2(e). */
+int sap_workspace_size(sap_plan_t plan, int32_t hq, int32_t hkv, int32_t head_dim, int32_t which, size_t* bytes);
+
+/* Forward: for every forward unit (q-tile, kv-chunk) and head, the partial
+ * attention of the q-tile's rows over that chunk's kv tiles (masked per tag),
+ * with online softmax in fp32 on tcgen05 tensor cores.  A q-tile with one unit
+ * writes bf16 O and fp32 LSE directly; the others leave fp32 partials (O, LSE)
+ * in the workspace for sap_merge.  Rows of a partial that see no key have
+ * LSE = -inf and O = 0. */
+int sap_attn_fwd(sap_plan_t plan, const void* q, const void* k, const void* v, int32_t hq, int32_t hkv,
+                 int32_t head_dim, float softmax_scale, void* o, float* lse, void* workspace, size_t ws_bytes,
+                 void* stream);
+
+/* Merge: for every q-tile with several partials, per (row, head)
+ *   LSE = M + log sum_b exp(LSE_b - M), M = max_b LSE_b;  O = sum_b exp(LSE_b - LSE) O_b,
+ * written as bf16 O and fp32 LSE.  Must follow sap_attn_fwd with the same
+ * workspace; a no-op when no q-tile has more than one partial. */
+int sap_merge(sap_plan_t plan, const void* workspace, size_t ws_bytes, int32_t hq, int32_t head_dim, void* o,
+              float* lse, void* stream);
+
+/* Backward with the merged O and LSE:  D_i = <dO_i, O_i>, P_ij = exp(S_ij - LSE_i),
+ * dV_j = sum P_ij dO_i, dS_ij = P_ij (<dO_i, V_j> - D_i), dQ_i = scale sum_j dS_ij K_j,
+ * dK_j = scale sum_i dS_ij Q_i, with dK/dV summed over the q heads of each kv
+ * head.  Chunk pairs need no merge here: the final LSE normalises every pair
+ * and their gradients add.  dQ is accumulated in fp32 in the workspace and
+ * converted to bf16 at the end. */
+int sap_attn_bwd(sap_plan_t plan, const void* q, const void* k, const void* v, const void* o, const float* lse,
+                 const void* dout, int32_t hq, int32_t hkv, int32_t head_dim, float softmax_scale, void* dq,
+                 void* dk, void* dv, void* workspace, size_t ws_bytes, void* stream);
+
+/* Synchronise the current device and return SAP_OK, or SAP_ERR_DEVICE if a
+ * kernel set the device error word (its code is stored in *code, then the word
+ * is cleared). */
+int sap_device_status(int32_t* code);
+
+/* Text for a status code. */
+const char* sap_error_string(int status);
+
+/* The last cudaError_t seen by a call that returned SAP_ERR_CUDA. */
+int sap_last_cuda_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SAP_H_ */

@@ -1,0 +1,422 @@
+// extern "C" entry points of libsap.so (declared in include/sap.h): argument
+// checks, plan upload, TMA tensor maps and kernel launches.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cstring>
+#include <mutex>
+#include <new>
+
+#include "kernels.cuh"
+#include "plan.hpp"
+#include "sap.h"
+
+namespace {
+
+thread_local int g_last_cuda_error = 0;
+
+// Device error word (bitwise OR of sap::kErr* codes), one per device.
+__device__ int g_device_err;
+
+int cuda_fail(cudaError_t e) {
+  g_last_cuda_error = (int)e;
+  return SAP_ERR_CUDA;
+}
+
+#define SAP_CUDA(call)                           \
+  do {                                           \
+    cudaError_t e_ = (call);                     \
+    if (e_ != cudaSuccess) return cuda_fail(e_); \
+  } while (0)
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool ready = false;
+  int sms = 0;
+  int* err = nullptr;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+int device_info(DeviceInfo** out) {
+  int dev = 0;
+  SAP_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) return SAP_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.ready) {
+    SAP_CUDA(cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev));
+    void* p = nullptr;
+    SAP_CUDA(cudaGetSymbolAddress(&p, g_device_err));
+    d.err = static_cast<int*>(p);
+    if (!g_encode) {
+      cudaDriverEntryPointQueryResult q;
+      void* fn = nullptr;
+      SAP_CUDA(cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q));
+      if (q != cudaDriverEntryPointSuccess || !fn) return cuda_fail(cudaErrorSymbolNotFound);
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    d.ready = true;
+  }
+  *out = &d;
+  return SAP_OK;
+}
+
+// [rows][heads][hd] bf16 -> 3-D map with 128-row x 64-column boxes, 128-byte swizzle.
+int make_map(CUtensorMap* map, const void* base, int64_t rows, int32_t heads, int32_t hd) {
+  cuuint64_t dims[3] = {(cuuint64_t)hd, (cuuint64_t)heads, (cuuint64_t)rows};
+  cuuint64_t strides[2] = {(cuuint64_t)hd * 2, (cuuint64_t)heads * hd * 2};
+  cuuint32_t box[3] = {64, 1, 128};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
+  return SAP_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
+
+int check_heads(int32_t hq, int32_t hkv, int32_t hd) {
+  if (hq <= 0 || hkv <= 0 || hq % hkv) return SAP_ERR_INVALID_ARG;
+  if (hd != 64 && hd != 128) return SAP_ERR_UNSUPPORTED;
+  return SAP_OK;
+}
+
+int check_kernel_plan(const sap_plan_s* p) {
+  if (!p) return SAP_ERR_INVALID_ARG;
+  if (p->block_m != 128 || p->block_n != 128) return SAP_ERR_UNSUPPORTED;
+  return SAP_OK;
+}
+
+// Workspace layouts (256-byte aligned pieces).
+struct FwdWs {
+  size_t o_part = 0, lse_part = 0, total = 0;
+};
+FwdWs fwd_ws(const sap_plan_s* p, int32_t hq, int32_t hd) {
+  FwdWs w;
+  const size_t slots = (size_t)p->n_slots;
+  w.o_part = 0;
+  w.lse_part = round_up((int64_t)(slots * hq * 128 * hd * 4), 256);
+  w.total = w.lse_part + round_up((int64_t)(slots * hq * 128 * 4), 256);
+  return w;
+}
+struct BwdWs {
+  size_t dq_acc = 0, dvec = 0, lse2 = 0, total = 0;
+  int64_t n_pad = 0;
+};
+BwdWs bwd_ws(const sap_plan_s* p, int32_t hq, int32_t hd) {
+  BwdWs w;
+  w.n_pad = round_up(p->n, 128);
+  w.dq_acc = 0;
+  w.dvec = round_up(w.n_pad * hq * hd * 4, 256);
+  w.lse2 = w.dvec + round_up(w.n_pad * hq * 4, 256);
+  w.total = w.lse2 + round_up(w.n_pad * hq * 4, 256);
+  return w;
+}
+
+}  // namespace
+
+extern "C" {
+
+int sap_plan(const int32_t* cu_seqlens_host, int32_t num_docs, int64_t total_tokens, int32_t num_chunks,
+             int32_t block_m, int32_t block_n, sap_plan_t* out) {
+  if (!out) return SAP_ERR_INVALID_ARG;
+  *out = nullptr;
+  sap_plan_s* p = new (std::nothrow) sap_plan_s();
+  if (!p) return SAP_ERR_NOMEM;
+  int rc;
+  try {
+    rc = sap_plan_build(cu_seqlens_host, num_docs, total_tokens, num_chunks, block_m, block_n, p);
+  } catch (const std::bad_alloc&) {
+    rc = SAP_ERR_NOMEM;
+  }
+  if (rc != SAP_OK) {
+    delete p;
+    return rc;
+  }
+  *out = p;
+  return SAP_OK;
+}
+
+int sap_plan_items(sap_plan_t plan, const sap_item_t** items, int64_t* n_items) {
+  if (!plan || !items || !n_items) return SAP_ERR_INVALID_ARG;
+  *items = plan->items.data();
+  *n_items = (int64_t)plan->items.size();
+  return SAP_OK;
+}
+
+int sap_plan_stats(sap_plan_t plan, int64_t* unmasked_pairs, int64_t* n_partial_slots, int32_t* n_chunk_pairs) {
+  if (!plan) return SAP_ERR_INVALID_ARG;
+  if (unmasked_pairs) *unmasked_pairs = plan->unmasked_pairs;
+  if (n_partial_slots) *n_partial_slots = plan->n_slots;
+  if (n_chunk_pairs) *n_chunk_pairs = plan->n_chunk_pairs;
+  return SAP_OK;
+}
+
+int sap_plan_fwd_schedule(sap_plan_t plan, const int32_t** units, int64_t* n_units, const int32_t** order,
+                          const int32_t** merges, int64_t* n_merges) {
+  if (!plan) return SAP_ERR_INVALID_ARG;
+  if (units) *units = plan->fwd_units.data();
+  if (n_units) *n_units = (int64_t)plan->fwd_units.size() / 4;
+  if (order) *order = plan->fwd_order.data();
+  if (merges) *merges = plan->merges.data();
+  if (n_merges) *n_merges = (int64_t)plan->merges.size() / 3;
+  return SAP_OK;
+}
+
+int sap_plan_bwd_schedule(sap_plan_t plan, const int32_t** kv_units, int64_t* n_kv_units, const int32_t** entries) {
+  if (!plan) return SAP_ERR_INVALID_ARG;
+  if (kv_units) *kv_units = plan->kv_units.data();
+  if (n_kv_units) *n_kv_units = (int64_t)plan->kv_units.size() / 3;
+  if (entries) *entries = plan->kv_entries.data();
+  return SAP_OK;
+}
+
+int sap_plan_upload(sap_plan_t p, void* stream) {
+  if (!p) return SAP_ERR_INVALID_ARG;
+  int dev = 0;
+  SAP_CUDA(cudaGetDevice(&dev));
+  if (p->dev && p->dev_id == dev) return SAP_OK;
+  if (p->dev) {
+    cudaFree(p->dev);
+    p->dev = nullptr;
+  }
+  // One int32 buffer; every piece starts on a 64-element (256-byte) boundary.
+  size_t off = 0;
+  auto place = [&](size_t words) {
+    size_t o = off;
+    off += (size_t)round_up((int64_t)words, 64);
+    return o;
+  };
+  p->off_items = place(p->items.size() * 5);
+  p->off_units = place(p->fwd_units.size());
+  p->off_order = place(p->fwd_order.size());
+  p->off_merges = place(p->merges.size());
+  p->off_kv_units = place(p->kv_units.size());
+  p->off_kv_entries = place(p->kv_entries.size());
+  p->off_tok_lo = place(p->tok_lo.size());
+  p->off_tok_hi = place(p->tok_hi.size());
+  p->dev_words = off > 0 ? off : 64;
+  void* d = nullptr;
+  SAP_CUDA(cudaMalloc(&d, p->dev_words * 4));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int32_t* base = static_cast<int32_t*>(d);
+  auto put = [&](size_t o, const void* src, size_t words) -> cudaError_t {
+    if (!words) return cudaSuccess;
+    return cudaMemcpyAsync(base + o, src, words * 4, cudaMemcpyHostToDevice, s);
+  };
+  cudaError_t e = cudaSuccess;
+  if (e == cudaSuccess) e = put(p->off_items, p->items.data(), p->items.size() * 5);
+  if (e == cudaSuccess) e = put(p->off_units, p->fwd_units.data(), p->fwd_units.size());
+  if (e == cudaSuccess) e = put(p->off_order, p->fwd_order.data(), p->fwd_order.size());
+  if (e == cudaSuccess) e = put(p->off_merges, p->merges.data(), p->merges.size());
+  if (e == cudaSuccess) e = put(p->off_kv_units, p->kv_units.data(), p->kv_units.size());
+  if (e == cudaSuccess) e = put(p->off_kv_entries, p->kv_entries.data(), p->kv_entries.size());
+  if (e == cudaSuccess) e = put(p->off_tok_lo, p->tok_lo.data(), p->tok_lo.size());
+  if (e == cudaSuccess) e = put(p->off_tok_hi, p->tok_hi.data(), p->tok_hi.size());
+  // The host arrays stay alive with the plan, but copies from pageable memory
+  // may still be staged: finish them before returning.
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) {
+    cudaFree(d);
+    return cuda_fail(e);
+  }
+  p->dev = d;
+  p->dev_id = dev;
+  return SAP_OK;
+}
+
+void sap_plan_destroy(sap_plan_t plan) {
+  if (!plan) return;
+  if (plan->dev) cudaFree(plan->dev);
+  delete plan;
+}
+
+int sap_workspace_size(sap_plan_t plan, int32_t hq, int32_t hkv, int32_t head_dim, int32_t which, size_t* bytes) {
+  if (!plan || !bytes) return SAP_ERR_INVALID_ARG;
+  int rc = check_heads(hq, hkv, head_dim);
+  if (rc) return rc;
+  if (which == SAP_WS_FWD)
+    *bytes = fwd_ws(plan, hq, head_dim).total;
+  else if (which == SAP_WS_BWD)
+    *bytes = bwd_ws(plan, hq, head_dim).total;
+  else
+    return SAP_ERR_INVALID_ARG;
+  return SAP_OK;
+}
+
+int sap_attn_fwd(sap_plan_t p, const void* q, const void* k, const void* v, int32_t hq, int32_t hkv,
+                 int32_t head_dim, float softmax_scale, void* o, float* lse, void* workspace, size_t ws_bytes,
+                 void* stream) {
+  int rc = check_kernel_plan(p);
+  if (rc) return rc;
+  if ((rc = check_heads(hq, hkv, head_dim))) return rc;
+  if (p->n == 0) return SAP_OK;
+  if (!q || !k || !v || !o || !lse) return SAP_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return SAP_ERR_INVALID_ARG;
+  const FwdWs ws = fwd_ws(p, hq, head_dim);
+  if (ws.total > 0 && p->n_slots > 0 && (!workspace || ws_bytes < ws.total)) return SAP_ERR_WORKSPACE;
+  DeviceInfo* di = nullptr;
+  if ((rc = device_info(&di))) return rc;
+  if ((rc = sap_plan_upload(p, stream))) return rc;
+  CUtensorMap tq, tk, tv;
+  if ((rc = make_map(&tq, q, p->n, hq, head_dim))) return rc;
+  if ((rc = make_map(&tk, k, p->n, hkv, head_dim))) return rc;
+  if ((rc = make_map(&tv, v, p->n, hkv, head_dim))) return rc;
+  const int32_t* base = static_cast<const int32_t*>(p->dev);
+  sap::FwdParams fp;
+  fp.items = base + p->off_items;
+  fp.units = base + p->off_units;
+  fp.order = base + p->off_order;
+  fp.tok_lo = base + p->off_tok_lo;
+  fp.n_units = (int32_t)(p->fwd_units.size() / 4);
+  fp.hq = hq;
+  fp.group = hq / hkv;
+  fp.n = p->n;
+  fp.scale_log2 = softmax_scale * 1.4426950408889634f;
+  fp.o = static_cast<__nv_bfloat16*>(o);
+  fp.lse = lse;
+  uint8_t* wsb = static_cast<uint8_t*>(workspace);
+  fp.o_part = p->n_slots ? reinterpret_cast<float*>(wsb + ws.o_part) : nullptr;
+  fp.lse_part = p->n_slots ? reinterpret_cast<float*>(wsb + ws.lse_part) : nullptr;
+  fp.err = di->err;
+  const int64_t work = (int64_t)fp.n_units * hq;
+  if (work == 0) return SAP_OK;
+  if (work > INT32_MAX) return SAP_ERR_INVALID_ARG;
+  const int grid = (int)(work < di->sms ? work : di->sms);
+  cudaError_t e = head_dim == 64 ? sap::launch_fwd<64>(tq, tk, tv, fp, grid, static_cast<cudaStream_t>(stream))
+                                 : sap::launch_fwd<128>(tq, tk, tv, fp, grid, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
+  return SAP_OK;
+}
+
+int sap_merge(sap_plan_t p, const void* workspace, size_t ws_bytes, int32_t hq, int32_t head_dim, void* o,
+              float* lse, void* stream) {
+  int rc = check_kernel_plan(p);
+  if (rc) return rc;
+  if (hq <= 0) return SAP_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return SAP_ERR_UNSUPPORTED;
+  const int64_t n_merges = (int64_t)p->merges.size() / 3;
+  if (p->n == 0 || n_merges == 0) return SAP_OK;
+  if (!o || !lse || !aligned16(o)) return SAP_ERR_INVALID_ARG;
+  const FwdWs ws = fwd_ws(p, hq, head_dim);
+  if (!workspace || ws_bytes < ws.total) return SAP_ERR_WORKSPACE;
+  if ((rc = sap_plan_upload(p, stream))) return rc;
+  const int32_t* base = static_cast<const int32_t*>(p->dev);
+  const uint8_t* wsb = static_cast<const uint8_t*>(workspace);
+  const float* op = reinterpret_cast<const float*>(wsb + ws.o_part);
+  const float* lp = reinterpret_cast<const float*>(wsb + ws.lse_part);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e =
+      head_dim == 64
+          ? sap::launch_merge<64>(base + p->off_merges, n_merges, hq, p->n, op, lp, static_cast<__nv_bfloat16*>(o),
+                                  lse, s)
+          : sap::launch_merge<128>(base + p->off_merges, n_merges, hq, p->n, op, lp,
+                                   static_cast<__nv_bfloat16*>(o), lse, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return SAP_OK;
+}
+
+int sap_attn_bwd(sap_plan_t p, const void* q, const void* k, const void* v, const void* o, const float* lse,
+                 const void* dout, int32_t hq, int32_t hkv, int32_t head_dim, float softmax_scale, void* dq,
+                 void* dk, void* dv, void* workspace, size_t ws_bytes, void* stream) {
+  int rc = check_kernel_plan(p);
+  if (rc) return rc;
+  if ((rc = check_heads(hq, hkv, head_dim))) return rc;
+  if (p->n == 0) return SAP_OK;
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return SAP_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, o, lse, dout, dq, dk, dv};
+  for (const void* ptr : ptrs)
+    if (!aligned16(ptr)) return SAP_ERR_INVALID_ARG;
+  const BwdWs ws = bwd_ws(p, hq, head_dim);
+  if (!workspace || ws_bytes < ws.total || !aligned16(workspace)) return SAP_ERR_WORKSPACE;
+  DeviceInfo* di = nullptr;
+  if ((rc = device_info(&di))) return rc;
+  if ((rc = sap_plan_upload(p, stream))) return rc;
+  CUtensorMap tq, tk, tv, tdo;
+  if ((rc = make_map(&tq, q, p->n, hq, head_dim))) return rc;
+  if ((rc = make_map(&tk, k, p->n, hkv, head_dim))) return rc;
+  if ((rc = make_map(&tv, v, p->n, hkv, head_dim))) return rc;
+  if ((rc = make_map(&tdo, dout, p->n, hq, head_dim))) return rc;
+  uint8_t* wsb = static_cast<uint8_t*>(workspace);
+  float* dq_acc = reinterpret_cast<float*>(wsb + ws.dq_acc);
+  float* dvec = reinterpret_cast<float*>(wsb + ws.dvec);
+  float* lse2 = reinterpret_cast<float*>(wsb + ws.lse2);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const __nv_bfloat16* ob = static_cast<const __nv_bfloat16*>(o);
+  const __nv_bfloat16* dob = static_cast<const __nv_bfloat16*>(dout);
+  cudaError_t e = head_dim == 64 ? sap::launch_bwd_pre<64>(ob, dob, lse, p->n, ws.n_pad, hq, dvec, lse2, dq_acc, s)
+                                 : sap::launch_bwd_pre<128>(ob, dob, lse, p->n, ws.n_pad, hq, dvec, lse2, dq_acc, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  const int32_t* base = static_cast<const int32_t*>(p->dev);
+  sap::BwdParams bp;
+  bp.kv_units = base + p->off_kv_units;
+  bp.entries = base + p->off_kv_entries;
+  bp.tok_hi = base + p->off_tok_hi;
+  bp.n_kv_units = (int32_t)(p->kv_units.size() / 3);
+  bp.hq = hq;
+  bp.hkv = hkv;
+  bp.group = hq / hkv;
+  bp.n = p->n;
+  bp.n_pad = ws.n_pad;
+  bp.scale_log2 = softmax_scale * 1.4426950408889634f;
+  bp.scale = softmax_scale;
+  bp.lse2 = lse2;
+  bp.dvec = dvec;
+  bp.dq_acc = dq_acc;
+  bp.dk = static_cast<__nv_bfloat16*>(dk);
+  bp.dv = static_cast<__nv_bfloat16*>(dv);
+  bp.err = di->err;
+  const int64_t work = (int64_t)bp.n_kv_units * hkv;
+  if (work > 0) {
+    const int grid = (int)(work < di->sms ? work : di->sms);
+    e = head_dim == 64 ? sap::launch_bwd<64>(tq, tk, tv, tdo, bp, grid, s)
+                       : sap::launch_bwd<128>(tq, tk, tv, tdo, bp, grid, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  e = sap::launch_dq_post(dq_acc, static_cast<__nv_bfloat16*>(dq), p->n * hq * head_dim, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return SAP_OK;
+}
+
+int sap_device_status(int32_t* code) {
+  DeviceInfo* di = nullptr;
+  int rc = device_info(&di);
+  if (rc) return rc;
+  SAP_CUDA(cudaDeviceSynchronize());
+  int v = 0;
+  SAP_CUDA(cudaMemcpyFromSymbol(&v, g_device_err, sizeof(int)));
+  if (code) *code = v;
+  if (v) {
+    const int zero = 0;
+    SAP_CUDA(cudaMemcpyToSymbol(g_device_err, &zero, sizeof(int)));
+    return SAP_ERR_DEVICE;
+  }
+  return SAP_OK;
+}
+
+const char* sap_error_string(int status) {
+  switch (status) {
+    case SAP_OK: return "ok";
+    case SAP_ERR_INVALID_ARG: return "invalid argument";
+    case SAP_ERR_BAD_SEQLENS: return "invalid cu_seqlens";
+    case SAP_ERR_BAD_CHUNKS: return "invalid chunk partition";
+    case SAP_ERR_WORKSPACE: return "workspace missing or too small";
+    case SAP_ERR_CUDA: return "CUDA runtime error";
+    case SAP_ERR_DEVICE: return "device error word set (a kernel wait timed out)";
+    case SAP_ERR_UNSUPPORTED: return "unsupported head_dim or tile size";
+    case SAP_ERR_NOMEM: return "host allocation failed";
+    default: return "unknown status";
+  }
+}
+
+int sap_last_cuda_error(void) { return g_last_cuda_error; }
+
+}  // extern "C"

@@ -1,0 +1,169 @@
+// Memory-bound kernels of the path: the exact LSE merge of partial outputs,
+// the backward pre-pass (D_i and LSE in the log2 domain, zeroed dQ
+// accumulator) and the fp32 -> bf16 conversion of dQ.  One warp per
+// (row, head) keeps every global access coalesced along the head dimension.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "kernels.cuh"
+
+namespace sap {
+
+namespace {
+
+constexpr int kWarpsPerBlock = 8;
+
+template <int E>
+struct Vec;
+template <>
+struct Vec<2> {
+  static __device__ __forceinline__ void load(const float* p, float* v) {
+    float2 t = *reinterpret_cast<const float2*>(p);
+    v[0] = t.x, v[1] = t.y;
+  }
+  static __device__ __forceinline__ void load_bf16(const __nv_bfloat16* p, float* v) {
+    __nv_bfloat162 t = *reinterpret_cast<const __nv_bfloat162*>(p);
+    v[0] = __bfloat162float(t.x), v[1] = __bfloat162float(t.y);
+  }
+  static __device__ __forceinline__ void store_bf16(__nv_bfloat16* p, const float* v) {
+    *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(v[0], v[1]);
+  }
+  static __device__ __forceinline__ void store_zero(float* p) { *reinterpret_cast<float2*>(p) = make_float2(0.f, 0.f); }
+};
+template <>
+struct Vec<4> {
+  static __device__ __forceinline__ void load(const float* p, float* v) {
+    float4 t = *reinterpret_cast<const float4*>(p);
+    v[0] = t.x, v[1] = t.y, v[2] = t.z, v[3] = t.w;
+  }
+  static __device__ __forceinline__ void load_bf16(const __nv_bfloat16* p, float* v) {
+    uint2 t = *reinterpret_cast<const uint2*>(p);
+    __nv_bfloat162 a = *reinterpret_cast<__nv_bfloat162*>(&t.x), b = *reinterpret_cast<__nv_bfloat162*>(&t.y);
+    v[0] = __bfloat162float(a.x), v[1] = __bfloat162float(a.y), v[2] = __bfloat162float(b.x),
+    v[3] = __bfloat162float(b.y);
+  }
+  static __device__ __forceinline__ void store_bf16(__nv_bfloat16* p, const float* v) {
+    __nv_bfloat162 a = __floats2bfloat162_rn(v[0], v[1]), b = __floats2bfloat162_rn(v[2], v[3]);
+    uint2 t;
+    t.x = *reinterpret_cast<uint32_t*>(&a);
+    t.y = *reinterpret_cast<uint32_t*>(&b);
+    *reinterpret_cast<uint2*>(p) = t;
+  }
+  static __device__ __forceinline__ void store_zero(float* p) {
+    *reinterpret_cast<float4*>(p) = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+};
+
+// Merge of the partials of one q-tile: warp = (merge entry, head, row).
+template <int D>
+__global__ void __launch_bounds__(kWarpsPerBlock * 32)
+    merge_kernel(const int32_t* merges, int64_t n_merges, int32_t hq, int64_t n, const float* o_part,
+                 const float* lse_part, __nv_bfloat16* o, float* lse) {
+  constexpr int E = D / 32;
+  const int64_t wid = (int64_t)blockIdx.x * kWarpsPerBlock + threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  if (wid >= n_merges * hq * 128) return;
+  const int64_t mi = wid / (hq * 128);
+  const int h = (int)((wid / 128) % hq), r = (int)(wid % 128);
+  const int qt = merges[3 * mi], s0 = merges[3 * mi + 1], ns = merges[3 * mi + 2];
+  const int64_t i = (int64_t)qt * 128 + r;
+  if (i >= n) return;
+  float mx = -INFINITY;
+  for (int b = 0; b < ns; ++b) mx = fmaxf(mx, lse_part[((size_t)(s0 + b) * hq + h) * 128 + r]);
+  float acc[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) acc[e] = 0.f;
+  float lse_all = -INFINITY;
+  if (mx != -INFINITY) {
+    float sum = 0.f;
+    for (int b = 0; b < ns; ++b) sum += __expf(lse_part[((size_t)(s0 + b) * hq + h) * 128 + r] - mx);
+    lse_all = mx + __logf(sum);
+    for (int b = 0; b < ns; ++b) {
+      const float wgt = __expf(lse_part[((size_t)(s0 + b) * hq + h) * 128 + r] - lse_all);
+      float v[E];
+      Vec<E>::load(o_part + (((size_t)(s0 + b) * hq + h) * 128 + r) * D + lane * E, v);
+#pragma unroll
+      for (int e = 0; e < E; ++e) acc[e] = fmaf(wgt, v[e], acc[e]);
+    }
+  }
+  Vec<E>::store_bf16(o + ((size_t)i * hq + h) * D + lane * E, acc);
+  if (lane == 0) lse[(size_t)h * n + i] = lse_all;
+}
+
+// D_i = <dO_i, O_i>, LSE_i * log2(e), and a zeroed dQ accumulator row: warp = (row, head).
+template <int D>
+__global__ void __launch_bounds__(kWarpsPerBlock * 32)
+    bwd_pre_kernel(const __nv_bfloat16* o, const __nv_bfloat16* dout, const float* lse, int64_t n, int64_t n_pad,
+                   int32_t hq, float* dvec, float* lse2, float* dq_acc) {
+  constexpr int E = D / 32;
+  const int64_t wid = (int64_t)blockIdx.x * kWarpsPerBlock + threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  if (wid >= n_pad * hq) return;
+  const int64_t i = wid / hq;
+  const int h = (int)(wid % hq);
+  Vec<E>::store_zero(dq_acc + (size_t)wid * D + lane * E);
+  float dsum = 0.f;
+  if (i < n) {
+    float a[E], b[E];
+    Vec<E>::load_bf16(o + (size_t)wid * D + lane * E, a);
+    Vec<E>::load_bf16(dout + (size_t)wid * D + lane * E, b);
+#pragma unroll
+    for (int e = 0; e < E; ++e) dsum = fmaf(a[e], b[e], dsum);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, off);
+  }
+  if (lane == 0) {
+    dvec[(size_t)h * n_pad + i] = dsum;
+    lse2[(size_t)h * n_pad + i] = i < n ? lse[(size_t)h * n + i] * 1.4426950408889634f : INFINITY;
+  }
+}
+
+__global__ void dq_post_kernel(const float* dq_acc, __nv_bfloat16* dq, int64_t count4) {
+  const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= count4) return;
+  float v[4];
+  Vec<4>::load(dq_acc + 4 * t, v);
+  Vec<4>::store_bf16(dq + 4 * t, v);
+}
+
+}  // namespace
+
+template <int D>
+cudaError_t launch_merge(const int32_t* merges, int64_t n_merges, int32_t hq, int64_t n, const float* o_part,
+                         const float* lse_part, __nv_bfloat16* o, float* lse, cudaStream_t stream) {
+  const int64_t warps = n_merges * hq * 128;
+  if (warps == 0) return cudaSuccess;
+  const int64_t blocks = (warps + kWarpsPerBlock - 1) / kWarpsPerBlock;
+  merge_kernel<D><<<(unsigned)blocks, kWarpsPerBlock * 32, 0, stream>>>(merges, n_merges, hq, n, o_part, lse_part, o,
+                                                                        lse);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_bwd_pre(const __nv_bfloat16* o, const __nv_bfloat16* dout, const float* lse, int64_t n,
+                           int64_t n_pad, int32_t hq, float* dvec, float* lse2, float* dq_acc, cudaStream_t stream) {
+  const int64_t warps = n_pad * hq;
+  if (warps == 0) return cudaSuccess;
+  const int64_t blocks = (warps + kWarpsPerBlock - 1) / kWarpsPerBlock;
+  bwd_pre_kernel<D><<<(unsigned)blocks, kWarpsPerBlock * 32, 0, stream>>>(o, dout, lse, n, n_pad, hq, dvec, lse2,
+                                                                          dq_acc);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dq_post(const float* dq_acc, __nv_bfloat16* dq, int64_t count, cudaStream_t stream) {
+  const int64_t c4 = count / 4;
+  if (c4 == 0) return cudaSuccess;
+  dq_post_kernel<<<(unsigned)((c4 + 255) / 256), 256, 0, stream>>>(dq_acc, dq, c4);
+  return cudaGetLastError();
+}
+
+template cudaError_t launch_merge<64>(const int32_t*, int64_t, int32_t, int64_t, const float*, const float*,
+                                      __nv_bfloat16*, float*, cudaStream_t);
+template cudaError_t launch_merge<128>(const int32_t*, int64_t, int32_t, int64_t, const float*, const float*,
+                                       __nv_bfloat16*, float*, cudaStream_t);
+template cudaError_t launch_bwd_pre<64>(const __nv_bfloat16*, const __nv_bfloat16*, const float*, int64_t, int64_t,
+                                        int32_t, float*, float*, float*, cudaStream_t);
+template cudaError_t launch_bwd_pre<128>(const __nv_bfloat16*, const __nv_bfloat16*, const float*, int64_t, int64_t,
+                                         int32_t, float*, float*, float*, cudaStream_t);
+
+}  // namespace sap

@@ -1,0 +1,359 @@
+// Forward kernel: partial attention of one q-tile over the kv tiles of one kv
+// chunk ("partial attention computation" of the HSAP / Sequence-Aware
+// Parallelism abstract), for every (forward unit, query head) work item.
+//
+// Persistent CTA, warp-specialised (192 threads):
+//   warp 0      TMA producer: Q tile per work item, K/V tiles through an
+//               NS-stage ring (128-byte swizzled boxes of 64 columns).
+//   warp 1      TMEM owner and tcgen05.mma issuer (one thread):
+//                 S_b = Q K^T   (M=128, N=128, K=D)   into TMEM buffer b = j % 2
+//                 O  += P V     (M=128, N=D,   K=128) into the TMEM O accumulator
+//               S_{j+1} is issued before P_j V_j so QK^T overlaps the softmax.
+//   warps 2..5  softmax warpgroup: thread t owns TMEM lane t = query row t of
+//               the tile.  Per kv tile it reads its S row, masks it (tag != FULL:
+//               keys outside [first token of its document, its own token]),
+//               runs the online softmax in the log2 domain, writes P (bf16)
+//               into a 128-byte swizzled shared tile for the PV MMA, and
+//               rescales O in TMEM when its running max grows by more than
+//               2^8 (lazy rescaling; exact, because the final division uses
+//               the same running max).  The epilogue normalises O and writes
+//               either bf16 O + LSE (single-chunk q-tiles) or an fp32 partial.
+//
+// TMEM columns: S0 [0,128), S1 [128,256), O [256, 256+D).
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "kernels.cuh"
+#include "ptx.cuh"
+
+namespace sap {
+
+template <int D>
+struct FwdCfg {
+  static constexpr int BM = 128, BN = 128;
+  static constexpr int NS = (D == 64) ? 3 : 2;          // K/V ring depth
+  static constexpr int BOX = 128 * 128;                 // bytes of one 128-row x 64-col bf16 box
+  static constexpr int QBYTES = D * BM * 2;
+  static constexpr int KVBYTES = D * BN * 2;
+  static constexpr int PBYTES = BM * BN * 2;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + QBYTES;
+  static constexpr int OFF_V = OFF_K + NS * KVBYTES;
+  static constexpr int OFF_P = OFF_V + NS * KVBYTES;
+  static constexpr int OFF_BAR = OFF_P + PBYTES;
+  static constexpr int NBAR = 2 + 4 * NS + 4 + 2 + 1;
+  static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;  // + tmem slot/abort flag + alignment slack
+  static constexpr int THREADS = 192;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t COL_O = 256;
+};
+
+template <int D>
+__global__ void __launch_bounds__(192, 1)
+    sap_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+  using C = FwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* q_full = bars + 0;
+  uint64_t* q_empty = bars + 1;
+  uint64_t* k_full = bars + 2;
+  uint64_t* k_empty = k_full + C::NS;
+  uint64_t* v_full = k_empty + C::NS;
+  uint64_t* v_empty = v_full + C::NS;
+  uint64_t* s_full = v_empty + C::NS;  // [2]
+  uint64_t* s_empty = s_full + 2;      // [2]
+  uint64_t* p_full = s_empty + 2;
+  uint64_t* pv_done = p_full + 1;
+  uint64_t* mma_drain = pv_done + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBAR);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const Guard guard{abort_flag, p.err};
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    for (int s = 0; s < C::NS; ++s) {
+      mbar_init(k_full + s, 1);
+      mbar_init(k_empty + s, 1);
+      mbar_init(v_full + s, 1);
+      mbar_init(v_empty + s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(s_full + b, 1);
+      mbar_init(s_empty + b, 128);
+    }
+    mbar_init(p_full, 128);
+    mbar_init(pv_done, 1);
+    mbar_init(mma_drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  const int total = p.n_units * p.hq;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ producer
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      uint32_t kv_iter = 0, unit_iter = 0;
+      bool ok = true;
+      for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
+        const int u = p.order[w / p.hq], h = w % p.hq, g = h / p.group;
+        const int qt = p.units[4 * u], ib = p.units[4 * u + 1], ic = p.units[4 * u + 2];
+        if (!mbar_wait(q_empty, (unit_iter & 1) ^ 1, guard, kErrTimeoutLoad)) break;
+        mbar_arrive_expect_tx(q_full, C::QBYTES);
+        for (int b = 0; b < D / 64; ++b) tma_load_3d(smem + C::OFF_Q + b * C::BOX, &tmQ, q_full, 64 * b, h, qt * 128);
+        for (int t = 0; t < ic; ++t) {
+          const int kt = p.items[5 * (ib + t) + 1];
+          const int s = kv_iter % C::NS;
+          const uint32_t ph = (kv_iter / C::NS) & 1;
+          if (!mbar_wait(k_empty + s, ph ^ 1, guard, kErrTimeoutLoad)) { ok = false; break; }
+          mbar_arrive_expect_tx(k_full + s, C::KVBYTES);
+          for (int b = 0; b < D / 64; ++b)
+            tma_load_3d(smem + C::OFF_K + s * C::KVBYTES + b * C::BOX, &tmK, k_full + s, 64 * b, g, kt * 128);
+          if (!mbar_wait(v_empty + s, ph ^ 1, guard, kErrTimeoutLoad)) { ok = false; break; }
+          mbar_arrive_expect_tx(v_full + s, C::KVBYTES);
+          for (int b = 0; b < D / 64; ++b)
+            tma_load_3d(smem + C::OFF_V + s * C::KVBYTES + b * C::BOX, &tmV, v_full + s, 64 * b, g, kt * 128);
+          ++kv_iter;
+        }
+        ++unit_iter;
+      }
+      // Let every copy this thread started land before the CTA can exit.
+      if (unit_iter > 0) drain_wait(q_full, (unit_iter - 1) & 1);
+      for (uint32_t t = (kv_iter > (uint32_t)C::NS ? kv_iter - C::NS : 0); t < kv_iter; ++t) {
+        const int s = t % C::NS;
+        const uint32_t ph = (t / C::NS) & 1;
+        drain_wait(k_full + s, ph);
+        drain_wait(v_full + s, ph);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ----------------------------------------------------------------- MMA
+      constexpr uint32_t idesc_qk = idesc_bf16(128, 128, false, false);
+      constexpr uint32_t idesc_pv = idesc_bf16(128, D, false, true);
+      const uint32_t sQ = smem_u32(smem + C::OFF_Q), sK = smem_u32(smem + C::OFF_K),
+                     sV = smem_u32(smem + C::OFF_V), sP = smem_u32(smem + C::OFF_P);
+      uint32_t kv_iter = 0, unit_iter = 0, s_iter = 0, pv_iter = 0;
+      bool ok = true;
+      for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
+        const int u = p.order[w / p.hq];
+        const int ic = p.units[4 * u + 2];
+        if (!mbar_wait(q_full, unit_iter & 1, guard, kErrTimeoutMma)) break;
+        tc_fence_after();
+        auto issue_pv = [&](uint32_t it) -> bool {  // it = kv_iter index of the tile
+          const int s = it % C::NS;
+          const uint32_t ph = (it / C::NS) & 1;
+          if (!mbar_wait(p_full, pv_iter & 1, guard, kErrTimeoutMma)) return false;
+          if (!mbar_wait(v_full + s, ph, guard, kErrTimeoutMma)) return false;
+          tc_fence_after();
+          const bool first = (it == kv_iter);  // first tile of this unit
+#pragma unroll
+          for (int kk = 0; kk < 128 / 16; ++kk) {
+            const uint64_t a = sdesc_sw128(sP + (kk / 4) * C::BOX + (kk % 4) * 32, 16, 1024);
+            const uint64_t b = sdesc_sw128(sV + s * C::KVBYTES + kk * 2048, C::BOX, 1024);
+            mma_bf16(tmem + C::COL_O, a, b, idesc_pv, (first && kk == 0) ? 0u : 1u);
+          }
+          tc_commit(pv_done);
+          tc_commit(v_empty + s);
+          ++pv_iter;
+          return true;
+        };
+        for (int j = 0; j < ic; ++j) {
+          const uint32_t it = kv_iter + j;
+          const int s = it % C::NS;
+          const uint32_t ph = (it / C::NS) & 1;
+          const int b = s_iter & 1;
+          if (!mbar_wait(k_full + s, ph, guard, kErrTimeoutMma)) { ok = false; break; }
+          if (!mbar_wait(s_empty + b, ((s_iter >> 1) & 1) ^ 1, guard, kErrTimeoutMma)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t a = sdesc_sw128(sQ + (kk / 4) * C::BOX + (kk % 4) * 32, 16, 1024);
+            const uint64_t bd = sdesc_sw128(sK + s * C::KVBYTES + (kk / 4) * C::BOX + (kk % 4) * 32, 16, 1024);
+            mma_bf16(tmem + 128 * b, a, bd, idesc_qk, kk > 0 ? 1u : 0u);
+          }
+          tc_commit(s_full + b);
+          tc_commit(k_empty + s);
+          ++s_iter;
+          if (j >= 1 && !issue_pv(it - 1)) { ok = false; break; }
+        }
+        if (ok && !issue_pv(kv_iter + ic - 1)) ok = false;
+        tc_commit(q_empty);
+        kv_iter += ic;
+        ++unit_iter;
+      }
+      // Wait for every MMA this thread issued before TMEM is released.
+      tc_commit(mma_drain);
+      drain_wait(mma_drain, 0);
+    }
+  } else {
+    // ------------------------------------------------------------- softmax
+    const int quad = warp & 3;            // TMEM lane quadrant this warp may access
+    const int r = quad * 32 + lane;       // query row within the tile
+    const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
+    uint8_t* sP = smem + C::OFF_P;
+    uint32_t s_iter = 0, pv_iter = 0;
+    const float sl2 = p.scale_log2;
+    for (int w = blockIdx.x; w < total; w += gridDim.x) {
+      const int u = p.order[w / p.hq], h = w % p.hq;
+      const int qt = p.units[4 * u], ib = p.units[4 * u + 1], ic = p.units[4 * u + 2], slot = p.units[4 * u + 3];
+      const int64_t i = (int64_t)qt * 128 + r;
+      const bool real_row = i < p.n;
+      const int row_lo = real_row ? p.tok_lo[i] : 1;  // empty key range for rows past N
+      const int row_hi = real_row ? (int)i : 0;
+      float m = -INFINITY, l = 0.f;
+      bool ok = true;
+      for (int j = 0; j < ic; ++j) {
+        const int kt = p.items[5 * (ib + j) + 1], tag = p.items[5 * (ib + j) + 4];
+        const int b = s_iter & 1;
+        if (!mbar_wait_warp(s_full + b, (s_iter >> 1) & 1, guard, kErrTimeoutSoftmax)) { ok = false; break; }
+        tc_fence_after();
+        float sv[128];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(lane_base + 128 * b + 32 * c, sv + 32 * c);
+        tc_fence_before();
+        mbar_arrive(s_empty + b);
+        ++s_iter;
+        if (tag != 0) {
+          const int c_lo = row_lo - kt * 128, c_hi = row_hi - kt * 128;
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            if (c < c_lo || c > c_hi) sv[c] = -INFINITY;
+        }
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 128; ++c) mx = fmaxf(mx, sv[c]);
+        const float m_tile = mx * sl2;
+        // P_{j-1} V_{j-1} must be complete before O is rescaled or P is overwritten.
+        if (j > 0) {
+          if (!mbar_wait_warp(pv_done, pv_iter & 1, guard, kErrTimeoutSoftmax)) { ok = false; break; }
+          ++pv_iter;
+          tc_fence_after();
+        }
+        if (m_tile > m + 8.0f) {
+          const float alpha = ex2(m - m_tile);  // 0 when m = -inf
+          if (j > 0 && l > 0.f) {
+#pragma unroll 1
+            for (int c = 0; c < D / 32; ++c) {
+              float ov[32];
+              tmem_ld32(lane_base + C::COL_O + 32 * c, ov);
+#pragma unroll
+              for (int e = 0; e < 32; ++e) ov[e] *= alpha;
+              tmem_st32(lane_base + C::COL_O + 32 * c, ov);
+            }
+          }
+          l *= alpha;
+          m = m_tile;
+        }
+        const float base = (m == -INFINITY) ? 0.f : m;
+        float rs = 0.f;
+#pragma unroll
+        for (int cc = 0; cc < 16; ++cc) {
+          uint32_t w4[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float p0 = ex2(fmaf(sv[cc * 8 + 2 * e], sl2, -base));
+            const float p1 = ex2(fmaf(sv[cc * 8 + 2 * e + 1], sl2, -base));
+            rs += p0 + p1;
+            w4[e] = pack_bf16x2(p0, p1);
+          }
+          const uint32_t addr = smem_u32(sP + (cc / 8) * C::BOX + sw128_offset(r, cc % 8));
+          st_shared_v4(addr, w4[0], w4[1], w4[2], w4[3]);
+        }
+        l += rs;
+        fence_async_smem();
+        tc_fence_before();
+        mbar_arrive(p_full);
+      }
+      if (!ok) break;
+      // ------------------------------------------------------------ epilogue
+      if (!mbar_wait_warp(pv_done, pv_iter & 1, guard, kErrTimeoutEpilogue)) break;
+      ++pv_iter;
+      tc_fence_after();
+      const float inv_l = l > 0.f ? 1.f / l : 0.f;
+      const float lse_val = l > 0.f ? (m + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
+      if (slot < 0) {
+        __nv_bfloat16* orow = p.o + ((size_t)i * p.hq + h) * D;
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          float ov[32];
+          tmem_ld32(lane_base + C::COL_O + 32 * c, ov);
+          if (real_row) {
+#pragma unroll
+            for (int e = 0; e < 32; e += 8) {
+              uint4 pk;
+              pk.x = pack_bf16x2(ov[e] * inv_l, ov[e + 1] * inv_l);
+              pk.y = pack_bf16x2(ov[e + 2] * inv_l, ov[e + 3] * inv_l);
+              pk.z = pack_bf16x2(ov[e + 4] * inv_l, ov[e + 5] * inv_l);
+              pk.w = pack_bf16x2(ov[e + 6] * inv_l, ov[e + 7] * inv_l);
+              *reinterpret_cast<uint4*>(orow + 32 * c + e) = pk;
+            }
+          }
+        }
+        if (real_row) p.lse[(size_t)h * p.n + i] = lse_val;
+      } else {
+        float* orow = p.o_part + (((size_t)slot * p.hq + h) * 128 + r) * D;
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          float ov[32];
+          tmem_ld32(lane_base + C::COL_O + 32 * c, ov);
+#pragma unroll
+          for (int e = 0; e < 32; e += 4)
+            *reinterpret_cast<float4*>(orow + 32 * c + e) =
+                make_float4(ov[e] * inv_l, ov[e + 1] * inv_l, ov[e + 2] * inv_l, ov[e + 3] * inv_l);
+        }
+        p.lse_part[((size_t)slot * p.hq + h) * 128 + r] = lse_val;
+      }
+      // The next unit's first PV overwrites O only after p_full, which these
+      // threads signal after this point, so the TMEM reads above are ordered
+      // before it by the fence below.
+      tc_fence_before();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+template <int D>
+int fwd_smem_bytes() {
+  return FwdCfg<D>::SMEM;
+}
+
+template <int D>
+cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
+                       int grid, cudaStream_t stream) {
+  auto kern = sap_fwd_kernel<D>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, FwdCfg<D>::SMEM);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, FwdCfg<D>::THREADS, FwdCfg<D>::SMEM, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError();
+}
+
+template cudaError_t launch_fwd<64>(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const FwdParams&,
+                                    int, cudaStream_t);
+template cudaError_t launch_fwd<128>(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const FwdParams&,
+                                     int, cudaStream_t);
+
+}  // namespace sap

@@ -1,0 +1,153 @@
+// Host planner: cu_seqlens + chunk partition -> non-empty tile items and the
+// forward / backward work schedules.
+//
+// This is the single-GPU counterpart of the schedule that the HSAP paper
+// generates ahead of time for the irregular attention of packed sequences
+// (HSAP / Sequence-Aware Parallelism page, abstract and method details: the
+// JIT-generated instruction sequences, and the load-balancing scheduler).
+// Here the schedule is a compact list of tiles that the kernels walk, with
+// cross-document tiles skipped entirely.
+//
+// Cost is O(items + N): for a q-tile whose first row starts document-wise at
+// token s, the kv tiles that hold an unmasked pair are exactly
+// floor(s / BN) .. floor((last row) / BN), because the key ranges of the rows
+// of one q-tile are contiguous and together cover [s, last row].  Tags need
+// O(1) work per item because the first key of a row is non-decreasing in the
+// row.
+#include <algorithm>
+#include <numeric>
+
+#include "plan.hpp"
+
+int sap_plan_build(const int32_t* cu, int32_t num_docs, int64_t n, int32_t num_chunks, int32_t block_m,
+                   int32_t block_n, sap_plan_s* p) {
+  if (!cu || !p || num_docs < 0 || n < 0 || block_m <= 0 || block_n <= 0) return SAP_ERR_INVALID_ARG;
+  if (n > INT32_MAX - 256) return SAP_ERR_INVALID_ARG;
+  if (cu[0] != 0) return SAP_ERR_BAD_SEQLENS;
+  for (int32_t k = 0; k < num_docs; ++k)
+    if (cu[k + 1] < cu[k]) return SAP_ERR_BAD_SEQLENS;
+  if ((int64_t)cu[num_docs] != n) return SAP_ERR_BAD_SEQLENS;
+  if (num_chunks < 1) return SAP_ERR_BAD_CHUNKS;
+  int64_t chunk = n > 0 ? n : 1;
+  if (num_chunks > 1) {
+    if (n % num_chunks) return SAP_ERR_BAD_CHUNKS;
+    chunk = n / num_chunks;
+    if (chunk % block_m || chunk % block_n) return SAP_ERR_BAD_CHUNKS;
+  }
+  p->n = n;
+  p->num_docs = num_docs;
+  p->num_chunks = num_chunks;
+  p->block_m = block_m;
+  p->block_n = block_n;
+  p->chunk = chunk;
+  p->cu.assign(cu, cu + num_docs + 1);
+
+  // per-token document bounds
+  p->tok_lo.assign((size_t)n, 0);
+  p->tok_hi.assign((size_t)n, 0);
+  p->unmasked_pairs = 0;
+  std::vector<int32_t> doc_of((size_t)n);
+  for (int32_t k = 0; k < num_docs; ++k) {
+    int64_t L = (int64_t)cu[k + 1] - cu[k];
+    p->unmasked_pairs += L * (L + 1) / 2;
+    for (int64_t i = cu[k]; i < cu[k + 1]; ++i) {
+      p->tok_lo[i] = cu[k];
+      p->tok_hi[i] = cu[k + 1] - 1;
+      doc_of[i] = k;
+    }
+  }
+
+  // items, canonical order
+  p->items.clear();
+  const int64_t ntq = (n + block_m - 1) / block_m;
+  for (int64_t qt = 0; qt < ntq; ++qt) {
+    const int64_t i0 = qt * block_m;
+    const int64_t ilast = std::min<int64_t>(i0 + block_m, n) - 1;  // last real row
+    const bool tile_complete = (i0 + block_m) <= n;
+    const int64_t kt_first = p->tok_lo[i0] / block_n, kt_last = ilast / block_n;
+    for (int64_t kt = kt_first; kt <= kt_last; ++kt) {
+      const int64_t j0 = kt * block_n, j1 = j0 + block_n - 1;
+      int32_t tag;
+      // every nominal row exists, the latest-starting row starts at or before j0,
+      // and the earliest row ends at or after j1
+      if (tile_complete && p->tok_lo[ilast] <= j0 && j1 <= i0)
+        tag = SAP_TAG_FULL;
+      else if (block_m == block_n && kt == qt && doc_of[i0] == doc_of[ilast])
+        tag = SAP_TAG_CAUSAL;
+      else
+        tag = SAP_TAG_MASKED;
+      p->items.push_back(
+          sap_item_t{(int32_t)qt, (int32_t)kt, (int32_t)(i0 / chunk), (int32_t)(j0 / chunk), tag});
+    }
+  }
+
+  // chunk pairs
+  {
+    std::vector<char> seen((size_t)num_chunks * num_chunks, 0);
+    p->n_chunk_pairs = 0;
+    for (const auto& it : p->items) {
+      char& s = seen[(size_t)it.q_chunk * num_chunks + it.kv_chunk];
+      if (!s) s = 1, ++p->n_chunk_pairs;
+    }
+  }
+
+  // forward units: contiguous runs of one q-tile and one kv-chunk
+  p->fwd_units.clear();
+  p->merges.clear();
+  p->n_slots = 0;
+  {
+    size_t a = 0;
+    const size_t ni = p->items.size();
+    while (a < ni) {
+      size_t e = a;
+      while (e < ni && p->items[e].q_tile == p->items[a].q_tile) ++e;  // items of this q-tile: [a, e)
+      std::vector<std::pair<size_t, size_t>> runs;
+      size_t r = a;
+      while (r < e) {
+        size_t s = r;
+        while (s < e && p->items[s].kv_chunk == p->items[r].kv_chunk) ++s;
+        runs.push_back({r, s - r});
+        r = s;
+      }
+      const bool partial = runs.size() > 1;
+      if (partial)
+        p->merges.insert(p->merges.end(),
+                         {p->items[a].q_tile, (int32_t)p->n_slots, (int32_t)runs.size()});
+      for (auto& run : runs) {
+        int32_t slot = partial ? (int32_t)(p->n_slots++) : -1;
+        p->fwd_units.insert(p->fwd_units.end(),
+                            {p->items[a].q_tile, (int32_t)run.first, (int32_t)run.second, slot});
+      }
+      a = e;
+    }
+  }
+  const size_t nu = p->fwd_units.size() / 4;
+  p->fwd_order.resize(nu);
+  std::iota(p->fwd_order.begin(), p->fwd_order.end(), 0);
+  std::stable_sort(p->fwd_order.begin(), p->fwd_order.end(),
+                   [&](int32_t x, int32_t y) { return p->fwd_units[4 * x + 2] > p->fwd_units[4 * y + 2]; });
+
+  // backward: items grouped by kv tile (counting sort keeps q-tile ascending)
+  const int64_t ntk = (n + block_n - 1) / block_n;
+  std::vector<int64_t> cnt((size_t)ntk + 1, 0);
+  for (const auto& it : p->items) cnt[(size_t)it.kv_tile + 1]++;
+  for (int64_t t = 0; t < ntk; ++t) cnt[t + 1] += cnt[t];
+  p->kv_entries.assign(p->items.size() * 2, 0);
+  {
+    std::vector<int64_t> pos(cnt.begin(), cnt.end() - 1);
+    for (const auto& it : p->items) {
+      int64_t w = pos[it.kv_tile]++;
+      p->kv_entries[2 * w] = it.q_tile;
+      p->kv_entries[2 * w + 1] = it.tag;
+    }
+  }
+  std::vector<int32_t> kvs;
+  for (int64_t t = 0; t < ntk; ++t)
+    if (cnt[t + 1] > cnt[t]) kvs.push_back((int32_t)t);
+  std::stable_sort(kvs.begin(), kvs.end(),
+                   [&](int32_t x, int32_t y) { return cnt[x + 1] - cnt[x] > cnt[y + 1] - cnt[y]; });
+  p->kv_units.clear();
+  for (int32_t t : kvs)
+    p->kv_units.insert(p->kv_units.end(), {t, (int32_t)cnt[t], (int32_t)(cnt[t + 1] - cnt[t])});
+  return SAP_OK;
+}

@@ -1,0 +1,147 @@
+"""Shared helpers of the GPU parity tests: run the CUDA path through the C ABI
+and compare with the oracle.
+
+Tolerance (written here and derived in the design doc): for O, dQ, dK, dV the
+bound max-abs 2e-2 / mean-abs 2e-3 applies on top of the half-ulp of the bf16
+output format, i.e. every element satisfies
+    |out - ref| <= 2e-2 + 2^-8 |ref|
+and mean |out - ref| <= 2e-3; for LSE, max-abs 1e-3.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import torch
+
+import oracle
+import packed_sequence_causal_b200 as sap
+
+ATOL = 2e-2
+MEAN_ATOL = 2e-3
+LSE_ATOL = 1e-3
+BF16_HALF_ULP = 2.0 ** -8
+
+
+def assert_close(out, ref, what: str):
+    out = out.detach().double().cpu().numpy() if hasattr(out, "detach") else np.asarray(out, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert out.shape == ref.shape, (what, out.shape, ref.shape)
+    assert np.all(np.isfinite(out)), f"{what}: non-finite output"
+    err = np.abs(out - ref)
+    excess = err - (ATOL + BF16_HALF_ULP * np.abs(ref))
+    worst = int(np.argmax(excess)) if excess.size else 0
+    assert excess.size == 0 or excess.max() <= 0, (
+        f"{what}: |err| {err.flat[worst]:.4g} at {np.unravel_index(worst, err.shape)} "
+        f"(ref {ref.flat[worst]:.4g}, out {out.flat[worst]:.4g})")
+    assert err.size == 0 or err.mean() <= MEAN_ATOL, f"{what}: mean |err| {err.mean():.4g}"
+
+
+def assert_lse(out, ref, what="lse"):
+    out = out.detach().double().cpu().numpy() if hasattr(out, "detach") else np.asarray(out)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert np.all(np.isfinite(out)), f"{what}: non-finite"
+    err = np.abs(out - ref)
+    assert err.size == 0 or err.max() <= LSE_ATOL, f"{what}: max |err| {err.max():.4g}"
+
+
+class Run:
+    """One fwd (+merge) and optionally bwd pass of a batch through the C ABI."""
+
+    def __init__(self, batch, nchunks: int, scale: float | None = None, device="cuda"):
+        b = batch
+        self.batch = b
+        n, hq, d = b.q.shape
+        hkv = b.k.shape[1]
+        self.n, self.hq, self.hkv, self.d = n, hq, hkv, d
+        self.scale = scale if scale is not None else 1.0 / math.sqrt(d)
+        self.plan = sap.sap_plan(b.cu_seqlens, n, nchunks)
+        self.q, self.k, self.v = (t.to(device).contiguous() for t in (b.q, b.k, b.v))
+        self.do = b.do.to(device).contiguous() if b.do is not None else None
+        self.o = torch.full((n, hq, d), float("nan"), dtype=torch.bfloat16, device=device)
+        self.lse = torch.full((hq, max(n, 1)), float("nan"), dtype=torch.float32, device=device)
+        self.ws_fwd = sap.alloc_workspace(self.plan, hq, hkv, d, sap.SAP_WS_FWD, device)
+
+    def fwd(self):
+        sap.sap_attn_fwd(self.plan, self.q, self.k, self.v, self.scale, self.o, self.lse, self.ws_fwd)
+        sap.sap_merge(self.plan, self.ws_fwd, self.hq, self.d, self.o, self.lse)
+        assert sap.sap_device_status() == 0
+        return self.o, self.lse[:, : self.n]
+
+    def bwd(self):
+        n, hq, hkv, d = self.n, self.hq, self.hkv, self.d
+        dev = self.q.device
+        self.dq = torch.full((n, hq, d), float("nan"), dtype=torch.bfloat16, device=dev)
+        self.dk = torch.full((n, hkv, d), float("nan"), dtype=torch.bfloat16, device=dev)
+        self.dv = torch.full((n, hkv, d), float("nan"), dtype=torch.bfloat16, device=dev)
+        ws = sap.alloc_workspace(self.plan, hq, hkv, d, sap.SAP_WS_BWD, dev)
+        sap.sap_attn_bwd(self.plan, self.q, self.k, self.v, self.o, self.lse, self.do, self.scale, self.dq, self.dk,
+                         self.dv, ws)
+        assert sap.sap_device_status() == 0
+        return self.dq, self.dk, self.dv
+
+
+def sample_rows(cu, n: int, nchunks: int, k_random: int = 24, seed: int = 0) -> np.ndarray:
+    """Rows at document starts/ends, chunk and tile boundaries, plus random rows."""
+    rows = set()
+    for s, e in zip(cu[:-1], cu[1:]):
+        if e > s:
+            rows |= {s, min(s + 1, e - 1), e - 1, max(s, e - 2)}
+    c = n // nchunks if nchunks > 1 else n
+    for b in range(nchunks):
+        rows |= {b * c, b * c + 127, b * c + 128}
+    rows |= {0, n - 1, 127, 128, 129}
+    rng = np.random.default_rng(seed)
+    rows |= set(rng.integers(0, n, size=k_random).tolist())
+    return np.array(sorted(r for r in rows if 0 <= r < n), dtype=np.int64)
+
+
+def cheap_kv_rows(cu, rows, d: int, G: int, budget: float = 3e10) -> np.ndarray:
+    """The subset of candidate kv rows whose dK/dV the sampled oracle computes within a flop budget."""
+    doc_of = np.searchsorted(np.asarray(cu), rows, side="right") - 1
+    chosen, need = [], {}
+    spent = 0.0
+    for j, dk in zip(rows, doc_of):
+        s, e = int(cu[dk]), int(cu[dk + 1])
+        lo = need.get(dk, e)
+        new_lo = min(lo, int(j))
+        # stats for rows [new_lo, lo) cost ~ sum (i - s + 1) d G each, plus the row's own sum
+        cost = sum_range(new_lo - s + 1, lo - s + 1) * 4.0 * d * G + (e - j) * 4.0 * d * G
+        if spent + cost > budget:
+            continue
+        spent += cost
+        need[dk] = new_lo
+        chosen.append(int(j))
+    return np.array(chosen, dtype=np.int64)
+
+
+def sum_range(a: int, b: int) -> float:
+    """sum of x for x in [a, b)."""
+    if b <= a:
+        return 0.0
+    return (a + b - 1) * (b - a) / 2.0
+
+
+def doc_sum_identities(dk, dv, do, cu, hq: int, hkv: int, what: str):
+    """Properties that hold at any size: per document and kv head,
+    sum_j dK[j] = 0 and sum_j dV[j] = sum over the group's heads and the document's rows of dO."""
+    G = hq // hkv
+    cu_t = torch.as_tensor(np.asarray(cu, dtype=np.int64), device=dk.device)
+    lens = (cu_t[1:] - cu_t[:-1])
+    doc_id = torch.repeat_interleave(torch.arange(len(lens), device=dk.device), lens)
+    ndoc = len(lens)
+
+    def seg_sum(x):  # x [N, hkv, d] -> [ndoc, hkv, d] in fp64
+        out = torch.zeros((ndoc,) + tuple(x.shape[1:]), dtype=torch.float64, device=x.device)
+        out.index_add_(0, doc_id, x.double())
+        return out
+
+    sk = seg_sum(dk)
+    sv = seg_sum(dv)
+    dog = do.double().reshape(do.shape[0], hkv, G, do.shape[2]).sum(2)
+    ref_v = seg_sum(dog)
+    # tolerance from bf16 rounding of the summed elements: 6 sigma of a random walk of half-ulps
+    tol_k = 6 * torch.sqrt(seg_sum((dk.double() * 2.0 ** -8) ** 2)) + 2e-2
+    tol_v = 6 * torch.sqrt(seg_sum((dv.double() * 2.0 ** -8) ** 2)) + 2e-2
+    assert torch.all(sk.abs() <= tol_k), f"{what}: sum dK per doc {sk.abs().max().item():.4g}"
+    assert torch.all((sv - ref_v).abs() <= tol_v), f"{what}: sum dV per doc {(sv - ref_v).abs().max().item():.4g}"

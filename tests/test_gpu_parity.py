@@ -1,0 +1,151 @@
+"""CUDA path (through the C ABI) against the fp64 oracle, element by element,
+on sizes the oracle finishes in seconds: several tiles, GQA and MHA, d = 64
+and 128, multiple chunks, ragged documents and a ragged tail, and the
+degenerate cases (empty batch, one-token documents, one document, tile-aligned
+documents, zero-length documents)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import packed_sequence_causal_b200 as sap
+import workloads
+from gpu_helpers import Run, assert_close, assert_lse
+
+pytestmark = pytest.mark.gpu
+
+
+def _fwd_bwd_full(lens, hq, hkv, d, nchunks, seed=0, scale=None, bwd=True):
+    b = workloads.custom_batch(lens, hq, hkv, d, seed=seed, with_do=bwd)
+    r = Run(b, nchunks, scale)
+    o, lse = r.fwd()
+    ro, rl = oracle.attn_fwd(b.q, b.k, b.v, b.cu_seqlens, r.scale)
+    assert_close(o, ro, "O")
+    assert_lse(lse, rl)
+    if bwd:
+        dq, dk, dv = r.bwd()
+        rdq, rdk, rdv = oracle.attn_bwd(b.q, b.k, b.v, b.do, b.cu_seqlens, r.scale)
+        assert_close(dq, rdq, "dQ")
+        assert_close(dk, rdk, "dK")
+        assert_close(dv, rdv, "dV")
+    return r
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_tiny_workload_fwd_merge(seed):
+    """1024 tokens, 4 documents (each >= 64), MHA 4 heads, d = 64, P = 2: fwd + merge."""
+    b = workloads.make_batch("tiny", seed)
+    r = Run(b, b.workload.p)
+    o, lse = r.fwd()
+    ro, rl = oracle.attn_fwd(b.q, b.k, b.v, b.cu_seqlens, r.scale)
+    assert_close(o, ro, "O")
+    assert_lse(lse, rl)
+
+
+def test_partials_match_chunked_oracle():
+    """The fp32 partials left in the workspace equal the oracle's per-chunk partial attention."""
+    lens = [700, 60, 500, 788]
+    b = workloads.custom_batch(lens, 2, 1, 64, seed=3, with_do=False)
+    nchunks = 4
+    r = Run(b, nchunks)
+    sap.sap_attn_fwd(r.plan, r.q, r.k, r.v, r.scale, r.o, r.lse, r.ws_fwd)
+    torch.cuda.synchronize()
+    _, _, op, lp = oracle.attn_fwd_chunked(b.q, b.k, b.v, b.cu_seqlens, r.scale, nchunks)
+    units, _, merges = sap.sap_plan_fwd_schedule(r.plan)
+    items = sap.sap_plan_items(r.plan)
+    slots = sap.sap_plan_stats(r.plan)["n_partial_slots"]
+    assert slots > 0
+    hq, d = 2, 64
+    ws = r.ws_fwd
+    o_part = ws[: slots * hq * 128 * d * 4].view(torch.float32).reshape(slots, hq, 128, d).cpu().double().numpy()
+    off = ((slots * hq * 128 * d * 4 + 255) // 256) * 256
+    l_part = ws[off: off + slots * hq * 128 * 4].view(torch.float32).reshape(slots, hq, 128).cpu().double().numpy()
+    for qt, ib, ic, slot in units:
+        if slot < 0:
+            continue
+        kc = items[ib, 3]
+        rows = slice(qt * 128, qt * 128 + 128)
+        ref_o = op[kc][rows].transpose(1, 0, 2)      # [hq, 128, d]
+        ref_l = lp[kc][:, rows]                      # [hq, 128]
+        empty = np.isneginf(ref_l)
+        assert np.array_equal(np.isneginf(l_part[slot]), empty)
+        np.testing.assert_allclose(l_part[slot][~empty], ref_l[~empty], atol=1e-3)
+        np.testing.assert_allclose(o_part[slot], ref_o, atol=5e-3)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_gqa_multichunk(d):
+    _fwd_bwd_full([300, 1, 129, 594, 512, 300, 212], 4, 2, d, 4)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_gqa4_three_chunks(d):
+    _fwd_bwd_full([1000, 37, 200, 299], 4, 1, d, 3, seed=2)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_mha_ragged_tail(d):
+    """N = 1000 is not a multiple of the 128 tile (P = 1)."""
+    _fwd_bwd_full([10, 500, 490], 2, 2, d, 1, seed=4)
+
+
+def test_ragged_smaller_than_a_tile():
+    _fwd_bwd_full([30, 47], 2, 1, 128, 1, seed=5)
+
+
+def test_one_document_is_plain_causal():
+    _fwd_bwd_full([640], 2, 1, 64, 5, seed=6)
+
+
+def test_single_token_documents():
+    _fwd_bwd_full([1] * 256, 2, 2, 128, 2, seed=7)
+
+
+def test_tile_aligned_documents():
+    """Documents of exactly 128 tokens: only CAUSAL diagonal tiles."""
+    _fwd_bwd_full([128] * 6, 2, 1, 64, 3, seed=8)
+
+
+def test_zero_length_documents():
+    _fwd_bwd_full([0, 200, 0, 0, 312, 0], 2, 2, 64, 2, seed=9)
+
+
+def test_custom_scale():
+    _fwd_bwd_full([400, 112], 2, 1, 128, 2, seed=10, scale=0.37)
+
+
+def test_large_scores_are_stable():
+    """Scale 1.0 on d = 128 gives scores of magnitude ~ 30: exercises the lazy rescaling."""
+    _fwd_bwd_full([256, 384], 2, 2, 128, 1, seed=11, scale=1.0 / math.sqrt(8.0))
+
+
+def test_empty_batch_is_a_no_op():
+    plan = sap.sap_plan([0], 0, 1)
+    z = torch.zeros((0, 2, 64), dtype=torch.bfloat16, device="cuda")
+    lse = torch.zeros((2, 1), dtype=torch.float32, device="cuda")
+    ws = sap.alloc_workspace(plan, 2, 2, 64, sap.SAP_WS_BWD)
+    sap.sap_attn_fwd(plan, z, z, z, 0.125, z, lse, ws)
+    sap.sap_merge(plan, ws, 2, 64, z, lse)
+    sap.sap_attn_bwd(plan, z, z, z, z, lse, z, 0.125, z, z, z, ws)
+    assert sap.sap_device_status() == 0
+
+
+def test_repeat_calls_are_identical_forward():
+    """Forward has no atomics: two calls give identical bytes."""
+    b = workloads.custom_batch([300, 700, 24], 4, 2, 64, seed=12, with_do=False)
+    r = Run(b, 1)
+    o1, l1 = r.fwd()
+    o1, l1 = o1.clone(), l1.clone()
+    o2, l2 = r.fwd()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_workspace_too_small_is_rejected():
+    b = workloads.custom_batch([700, 324], 2, 1, 64, seed=13, with_do=True)
+    r = Run(b, 8)
+    small = torch.empty(16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(sap.SapError) as e:
+        sap.sap_attn_fwd(r.plan, r.q, r.k, r.v, r.scale, r.o, r.lse, small)
+    assert e.value.status == -4

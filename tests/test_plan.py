@@ -1,0 +1,159 @@
+"""Host planner (libsap.so, no GPU needed): bit-exact tile list against the
+oracle, schedule invariants, statistics and argument errors."""
+import numpy as np
+import pytest
+
+import oracle
+import packed_sequence_causal_b200 as sap
+import workloads
+
+
+def _plan_and_check(cu, n, nchunks, bm=128, bn=128):
+    plan = sap.sap_plan(cu, n, nchunks, bm, bn)
+    items = sap.sap_plan_items(plan)
+    ref = oracle.tile_list(cu, n, nchunks, bm, bn)
+    np.testing.assert_array_equal(items, ref)
+    st = sap.sap_plan_stats(plan)
+    assert st["unmasked_pairs"] == oracle.unmasked_pairs(cu)
+    assert st["n_chunk_pairs"] == len({(int(a), int(b)) for a, b in ref[:, 2:4]}) if len(ref) else True
+    _check_schedules(plan, items, n, nchunks, bm, bn)
+    return plan, items
+
+
+def _check_schedules(plan, items, n, nchunks, bm, bn):
+    units, order, merges = sap.sap_plan_fwd_schedule(plan)
+    # units tile the item list contiguously, one (q-tile, kv-chunk) each
+    pos = 0
+    slots_of_tile = {}
+    for qt, b, c, slot in units:
+        assert b == pos and c > 0
+        run = items[b:b + c]
+        assert np.all(run[:, 0] == qt) and len(set(run[:, 3].tolist())) == 1
+        pos += c
+        slots_of_tile.setdefault(int(qt), []).append(int(slot))
+    assert pos == len(items)
+    # a q-tile with several units gets consecutive partial slots; one unit writes directly
+    mi = 0
+    next_slot = 0
+    for qt in sorted(slots_of_tile):
+        s = slots_of_tile[qt]
+        if len(s) == 1:
+            assert s == [-1]
+        else:
+            assert s == list(range(next_slot, next_slot + len(s)))
+            assert tuple(merges[mi]) == (qt, next_slot, len(s))
+            next_slot += len(s)
+            mi += 1
+    assert mi == len(merges)
+    assert sap.sap_plan_stats(plan)["n_partial_slots"] == next_slot
+    # heavy-first order: a permutation, non-increasing item counts, stable on ties
+    assert sorted(order.tolist()) == list(range(len(units)))
+    counts = units[order, 2]
+    assert np.all(np.diff(counts) <= 0)
+    for a, b in zip(order[:-1], order[1:]):
+        if units[a, 2] == units[b, 2]:
+            assert a < b
+    # backward: every item once, grouped by kv tile, q-tile ascending, heavy-first
+    kv_units, entries = sap.sap_plan_bwd_schedule(plan)
+    seen = set()
+    prev_cnt = None
+    for kt, e0, ne in kv_units:
+        grp = entries[e0:e0 + ne]
+        assert np.all(np.diff(grp[:, 0]) > 0)
+        for qt, tag in grp:
+            seen.add((int(qt), int(kt), int(tag)))
+        if prev_cnt is not None:
+            assert ne <= prev_cnt
+        prev_cnt = ne
+    assert seen == {(int(a), int(b), int(t)) for a, b, _, _, t in items}
+
+
+@pytest.mark.parametrize("name", ["tiny", "llama32_1b_32k", "llama31_8b_128k", "llama2_13b_64k_short"])
+def test_planner_matches_oracle_on_workloads(name):
+    w = workloads.WORKLOADS[name]
+    cu = workloads.cu_seqlens_from_lengths(workloads.doc_lengths(w, 0))
+    _plan_and_check(cu, w.n, w.p)
+
+
+def test_planner_matches_oracle_512k():
+    w = workloads.WORKLOADS["hybrid_512k"]
+    cu = workloads.cu_seqlens_from_lengths(workloads.doc_lengths(w, 0))
+    _plan_and_check(cu, w.n, w.p)
+
+
+@pytest.mark.parametrize("seed", range(20))
+def test_planner_matches_oracle_random(seed):
+    rng = np.random.default_rng(100 + seed)
+    bm = int(rng.choice([16, 32, 128]))
+    nchunks = int(rng.choice([1, 2, 4, 8]))
+    n = bm * nchunks * int(rng.integers(1, 8))
+    lens = []
+    while sum(lens) < n:
+        lens.append(int(min(n - sum(lens), rng.integers(1, 4 * bm))))
+        if rng.random() < 0.1:
+            lens.append(0)
+    _plan_and_check(workloads.cu_seqlens_from_lengths(lens), n, nchunks, bm, bm)
+
+
+@pytest.mark.parametrize("n", [1, 5, 127, 129, 300, 1000])
+def test_planner_ragged_single_chunk(n):
+    lens = [max(1, n // 4), n - max(1, n // 4)] if n > 1 else [1]
+    _plan_and_check(workloads.cu_seqlens_from_lengths(lens), n, 1)
+
+
+def test_planner_rectangular_tiles():
+    cu = workloads.cu_seqlens_from_lengths([100, 28, 200, 56])
+    _plan_and_check(cu, 384, 3, 32, 64)
+
+
+def test_planner_empty_batch():
+    plan = sap.sap_plan([0], 0, 1)
+    assert len(sap.sap_plan_items(plan)) == 0
+    assert sap.sap_plan_stats(plan)["unmasked_pairs"] == 0
+
+
+def test_planner_single_token_docs_only_diagonal():
+    n = 512
+    plan, items = _plan_and_check(np.arange(n + 1, dtype=np.int32), n, 4)
+    assert len(items) == n // 128 and np.all(items[:, 0] == items[:, 1])
+
+
+def test_planner_errors():
+    with pytest.raises(sap.SapError) as e:
+        sap.sap_plan([0, 10, 9, 20], 20, 1)
+    assert e.value.status == -2
+    with pytest.raises(sap.SapError) as e:
+        sap.sap_plan([1, 20], 20, 1)
+    assert e.value.status == -2
+    with pytest.raises(sap.SapError) as e:
+        sap.sap_plan([0, 20], 21, 1)
+    assert e.value.status == -2
+    with pytest.raises(sap.SapError) as e:
+        sap.sap_plan([0, 300], 300, 3)       # chunk 100 not a multiple of 128
+    assert e.value.status == -3
+    with pytest.raises(sap.SapError) as e:
+        sap.sap_plan([0, 512], 512, 0)
+    assert e.value.status == -3
+    with pytest.raises(sap.SapError) as e:
+        sap.sap_plan([0, 512], 512, 3)       # N not divisible by P
+    assert e.value.status == -3
+    with pytest.raises(sap.SapError) as e:
+        sap.sap_plan([0, 512], 512, 1, 0, 128)
+    assert e.value.status == -1
+
+
+def test_workspace_sizes_and_head_checks():
+    w = workloads.WORKLOADS["tiny"]
+    cu = workloads.cu_seqlens_from_lengths(workloads.doc_lengths(w, 0))
+    plan = sap.sap_plan(cu, w.n, w.p)
+    slots = sap.sap_plan_stats(plan)["n_partial_slots"]
+    fwd = sap.sap_workspace_size(plan, 4, 4, 64, sap.SAP_WS_FWD)
+    assert fwd >= slots * 4 * 128 * (64 + 1) * 4
+    bwd = sap.sap_workspace_size(plan, 4, 4, 64, sap.SAP_WS_BWD)
+    assert bwd >= 1024 * 4 * 64 * 4 + 2 * 4 * 1024 * 4
+    with pytest.raises(sap.SapError) as e:
+        sap.sap_workspace_size(plan, 6, 4, 64, sap.SAP_WS_FWD)   # hq % hkv != 0
+    assert e.value.status == -1
+    with pytest.raises(sap.SapError) as e:
+        sap.sap_workspace_size(plan, 4, 4, 96, sap.SAP_WS_FWD)   # unsupported head_dim
+    assert e.value.status == -7
