@@ -246,18 +246,22 @@ __global__ void __launch_bounds__(192, 1)
           ++pv_iter;
           tc_fence_after();
         }
-        if (m_tile > m + 8.0f) {
-          const float alpha = ex2(m - m_tile);  // 0 when m = -inf
-          if (j > 0 && l > 0.f) {
+        // Rows decide independently whether their max moved; the TMEM
+        // load/store of O is warp-collective, so the warp rescales together
+        // when any of its rows needs it (alpha = 1 for the others).
+        const bool grow = m_tile > m + 8.0f;
+        const float alpha = grow ? ex2(m - m_tile) : 1.f;  // 0 when m = -inf
+        if (j > 0 && __any_sync(0xffffffffu, grow && l > 0.f)) {
 #pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
-              float ov[32];
-              tmem_ld32(lane_base + C::COL_O + 32 * c, ov);
+          for (int c = 0; c < D / 32; ++c) {
+            float ov[32];
+            tmem_ld32(lane_base + C::COL_O + 32 * c, ov);
 #pragma unroll
-              for (int e = 0; e < 32; ++e) ov[e] *= alpha;
-              tmem_st32(lane_base + C::COL_O + 32 * c, ov);
-            }
+            for (int e = 0; e < 32; ++e) ov[e] *= alpha;
+            tmem_st32(lane_base + C::COL_O + 32 * c, ov);
           }
+        }
+        if (grow) {
           l *= alpha;
           m = m_tile;
         }
