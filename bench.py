@@ -1,0 +1,390 @@
+#!/usr/bin/env python
+"""Benchmark of the packed causal attention hot path (SAP, one GPU per rank).
+
+One step = the whole path over one packed batch: sap_attn_fwd (partial
+attention per (q-tile, kv-chunk)), sap_merge (exact LSE merge), sap_attn_bwd
+(D, dK/dV/dQ, dQ conversion).  Prints one JSON line (rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Metric: TFLOP/s on unmasked FLOPs, 14 * head_dim * pairs * hq per step
+(forward 4, backward 10), pairs = sum over documents of L(L+1)/2.  Under
+torchrun every rank runs its own independent batch (seed + rank): data
+parallel replicas, weak scaling, no collective on the data path.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import workloads  # noqa: E402
+
+METRIC = "packed causal attn fwd+bwd TFLOP/s (unmasked FLOPs), tokens/s; % bf16 peak"
+DEFAULT_WORKLOAD = "llama31_8b_128k"
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]), float(d["bf16_tflops_sustained"]), float(d["hbm_gbs"]), "measured"
+    return 1590.0, 1400.0, 6650.0, "fallback"
+
+
+def _flops(w, pairs):
+    return 4.0 * w.d * pairs * w.hq, 10.0 * w.d * pairs * w.hq
+
+
+# ----------------------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    """nvidia-smi samples (200 ms) during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                                          "-lms", "200", "-i", str(self.gpu_index)], stdout=self.f,
+                                         stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, power, reasons = [], [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx.append(float(parts[2]))
+                    power.append(float(parts[3]))
+                except ValueError:
+                    continue
+                for nm, val in zip(names, parts[5:9]):
+                    if val.lower().startswith("active"):
+                        reasons.add(nm)
+        os.unlink(self.path)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        under_load = [s for s, p in zip(sm, power) if p > 0.3 * max(power)] or sm
+        return {"sm_mhz": statistics.median(under_load), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm), "power_w_max": max(power)}
+
+
+# --------------------------------------------------------------------- cpu oracle
+
+
+def _doc_sample(b, budget_flops: float):
+    """The shortest documents of the batch, shortest first, while their oracle cost fits the budget.
+
+    Returns (token index list, cu_seqlens of the sub-batch, unmasked FLOPs, number of documents)."""
+    w = b.workload
+    cu = b.cu_seqlens
+    lens = np.diff(cu)
+    order = np.argsort(lens, kind="stable")
+    picked, spent = [], 0.0
+    for dk in order:
+        L = int(lens[dk])
+        if L == 0:
+            continue
+        f = 14.0 * w.d * w.hq * L * (L + 1) / 2
+        if picked and spent + f > budget_flops:
+            break
+        picked.append(int(dk))
+        spent += f
+        if spent >= budget_flops:
+            break
+    picked.sort()
+    idx = np.concatenate([np.arange(cu[dk], cu[dk + 1]) for dk in picked])
+    sub_cu = np.concatenate([[0], np.cumsum([lens[dk] for dk in picked])]).astype(np.int32)
+    return idx, sub_cu, spent, len(picked)
+
+
+def run_oracle_sample(b, budget_flops: float):
+    """Times the fp64 oracle (forward + backward) on a bounded document sample. Returns (tflops, seconds, desc)."""
+    import torch
+
+    import oracle  # the CPU baseline leg is the one place the benchmark runs the oracle
+
+    w = b.workload
+    idx, sub_cu, flops, ndocs = _doc_sample(b, budget_flops)
+    ti = torch.as_tensor(idx, device=b.q.device)
+    q, k, v, do = (t.index_select(0, ti).cpu() for t in (b.q, b.k, b.v, b.do))
+    scale = 1.0 / math.sqrt(w.d)
+    t0 = time.perf_counter()
+    oracle.attn_fwd(q, k, v, sub_cu, scale)
+    oracle.attn_bwd(q, k, v, do, sub_cu, scale)
+    dt = time.perf_counter() - t0
+    desc = (f"oracle fwd+bwd (fp64, all {w.hq} heads) on the {ndocs} shortest documents of the workload "
+            f"({len(idx)} tokens, {flops:.3g} unmasked FLOPs)")
+    return flops / dt / 1e12, dt, desc
+
+
+# ------------------------------------------------------------------------- main
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=1e11, help="unmasked FLOPs of the CPU-baseline sample")
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    w = workloads.WORKLOADS[args.workload]
+
+    if args.impl == "reference":
+        return run_reference(args, w, rank, world)
+
+    import torch
+    import torch.distributed as dist
+
+    import packed_sequence_causal_b200 as sap
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    b = workloads.make_batch(w.name, args.seed + rank, device=str(dev), with_do=True)
+    n, hq, hkv, d = w.n, w.hq, w.hkv, w.d
+    scale = 1.0 / math.sqrt(d)
+    t_plan = time.perf_counter()
+    plan = sap.sap_plan(b.cu_seqlens, n, w.p)
+    t_plan = time.perf_counter() - t_plan
+    sap.sap_plan_upload(plan)
+    stats = sap.sap_plan_stats(plan)
+    pairs = stats["unmasked_pairs"]
+    n_items = len(sap.sap_plan_items(plan))
+    _, _, merges = sap.sap_plan_fwd_schedule(plan)
+    q, k, v, do = b.q, b.k, b.v, b.do
+    o = torch.empty_like(q)
+    lse = torch.empty((hq, n), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws_f = sap.alloc_workspace(plan, hq, hkv, d, sap.SAP_WS_FWD, dev)
+    ws_b = sap.alloc_workspace(plan, hq, hkv, d, sap.SAP_WS_BWD, dev)
+    stream = torch.cuda.current_stream()
+    launches_per_step = 1 + (1 if len(merges) else 0) + 3
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        sap.sap_attn_fwd(plan, q, k, v, scale, o, lse, ws_f, stream)
+        if ev:
+            ev[1].record(stream)
+        sap.sap_merge(plan, ws_f, hq, d, o, lse, stream)
+        if ev:
+            ev[2].record(stream)
+        sap.sap_attn_bwd(plan, q, k, v, o, lse, do, scale, dq, dk, dv, ws_b, stream)
+        if ev:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    status = sap.sap_device_status()
+    if status != 0:
+        raise RuntimeError(f"device error word {status} after warm-up")
+
+    gpu_index = local_rank
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    if vis and "," not in vis and vis.strip().isdigit():
+        gpu_index = int(vis)
+    sampler = ClockSampler(gpu_index)
+    sampler.start()
+    time.sleep(0.4)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    elapsed_ms = start.elapsed_time(end)
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    status = sap.sap_device_status()
+    if status != 0:
+        raise RuntimeError(f"device error word {status} after the timed steps")
+
+    f_fwd, f_bwd = _flops(w, pairs)
+    f_step = f_fwd + f_bwd
+    ms_step = elapsed_ms / args.steps
+    value = world * f_step * args.steps / (elapsed_ms / 1e3) / 1e12
+    tokens_s = world * n * args.steps / (elapsed_ms / 1e3)
+    burst, sustained, hbm, peak_src = _peaks()
+    # per-call device times from the events recorded on the launching stream
+    t_fwd, t_merge, t_bwd = (sum(e[c].elapsed_time(e[c + 1]) for e in evs) / args.steps for c in range(3))
+
+    # end to end through the public API: pinned host inputs -> device, the path, results -> pinned host
+    e2e = None
+    if not args.no_e2e:
+        hq_in = [t.cpu().pin_memory() for t in (q, k, v, do)]
+        h_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (o, lse, dq, dk, dv)]
+        dev_in = (q, k, v, do)
+        h2d = sum(t.numel() * t.element_size() for t in hq_in)
+        d2h = sum(t.numel() * t.element_size() for t in h_out)
+
+        def e2e_step():
+            for dst, src in zip(dev_in, hq_in):
+                dst.copy_(src, non_blocking=True)
+            step()
+            for dst, src in zip(h_out, (o, lse, dq, dk, dv)):
+                dst.copy_(src, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s2.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e2.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = s2.elapsed_time(e2)
+        if world > 1:
+            t = torch.tensor([e2e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        e2e = {"value": round(world * f_step * args.steps / (e2e_ms / 1e3) / 1e12, 2), "unit": "TFLOP/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "ms_per_step": round(e2e_ms / args.steps, 3),
+               "tokens_per_s": round(world * n * args.steps / (e2e_ms / 1e3), 1)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tf, secs, desc = run_oracle_sample(b, args.cpu_budget)
+        import oracle
+        cpu = {"value": tf, "unit": "TFLOP/s", "cores": oracle.max_threads(), "kind": "oracle", "sample": desc,
+               "seconds": round(secs, 2)}
+
+    if rank == 0:
+        achieved = f_bwd / (t_bwd / 1e3) / 1e12
+        line = {
+            "metric": METRIC,
+            "value": round(value, 2),
+            "unit": "TFLOP/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": round(ms_step, 3),
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic (seeded packed documents, bf16 N(0,1) Q/K/V/dO)",
+            "config": {"workload": w.name, "tokens": n, "docs": int(len(b.cu_seqlens) - 1), "hq": hq, "hkv": hkv,
+                       "head_dim": d, "chunks": w.p, "tiles": n_items, "unmasked_pairs_per_head": pairs,
+                       "flops_per_step": f_step, "parallelism": f"dp{world}" if world > 1 else "single",
+                       "l2": "inputs larger than L2 (Q, dO, O 1 GiB each); no flush"},
+            "tokens_per_s": round(tokens_s, 1),
+            "pct_bf16_peak": round(100 * value / world / burst, 2),
+            "pct_bf16_peak_sustained": round(100 * value / world / sustained, 2),
+            "peak_source": peak_src,
+            "kernels_ms": {"fwd": round(t_fwd, 3), "merge": round(t_merge, 3), "bwd": round(t_bwd, 3),
+                           "fwd_tflops": round(f_fwd / (t_fwd / 1e3) / 1e12, 1),
+                           "bwd_tflops": round(f_bwd / (t_bwd / 1e3) / 1e12, 1),
+                           "plan_host_ms": round(1e3 * t_plan, 2)},
+            "roofline": {"bound": "tensor", "kernel": "sap_attn_bwd (bwd_pre + sap_bwd_kernel + dq_post)",
+                         "achieved": round(achieved, 1), "peak": sustained, "unit": "TFLOP/s",
+                         "frac": round(achieved / sustained, 4), "frac_of_burst_peak": round(achieved / burst, 4),
+                         "traffic": None},
+            "clocks": clocks,
+            "gpu_launches": launches_per_step * args.steps,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_reference(args, w, rank, world):
+    """The oracle as the reference arm: fp64 on the host cores, bounded sample per step."""
+    if rank != 0:
+        return
+    import oracle
+    b = workloads.make_batch(w.name, args.seed, device="cpu", with_do=True)
+    budget = args.cpu_budget / 3
+    for _ in range(args.warmup):
+        run_oracle_sample(b, budget / 4)
+    times, desc, tf_all = [], "", []
+    for _ in range(args.steps):
+        tf, secs, desc = run_oracle_sample(b, budget)
+        times.append(secs)
+        tf_all.append(tf)
+    _, _, flops, _ = _doc_sample(b, budget)
+    value = flops * len(times) / sum(times) / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(1e3 * sum(times) / len(times), 1), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded packed documents, bf16 N(0,1) Q/K/V/dO)",
+        "config": {"workload": w.name, "tokens": w.n, "hq": w.hq, "hkv": w.hkv, "head_dim": w.d, "chunks": w.p},
+        "impl": "reference",
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.max_threads(), "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

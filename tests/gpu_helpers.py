@@ -124,7 +124,15 @@ def sum_range(a: int, b: int) -> float:
 
 def doc_sum_identities(dk, dv, do, cu, hq: int, hkv: int, what: str):
     """Properties that hold at any size: per document and kv head,
-    sum_j dK[j] = 0 and sum_j dV[j] = sum over the group's heads and the document's rows of dO."""
+    sum_j dK[j] = 0 and sum_j dV[j] = sum over the group's heads and the document's rows of dO.
+
+    Tolerance: 0.1 + 2e-3 * (natural scale of the sum), the natural scale being
+    sqrt(sum of squares) of the summed terms (dO for dV, dK for dK).  Against the
+    full oracle on a 16K-token batch with an 8K-token document the kernel's
+    per-document sums deviate from the exact sums by at most 3e-4 of that scale
+    (fp32 accumulation over long reductions plus bf16 operands), so the bound
+    leaves headroom; a dropped near-diagonal tile moves a sum by O(1).
+    """
     G = hq // hkv
     cu_t = torch.as_tensor(np.asarray(cu, dtype=np.int64), device=dk.device)
     lens = (cu_t[1:] - cu_t[:-1])
@@ -138,10 +146,11 @@ def doc_sum_identities(dk, dv, do, cu, hq: int, hkv: int, what: str):
 
     sk = seg_sum(dk)
     sv = seg_sum(dv)
-    dog = do.double().reshape(do.shape[0], hkv, G, do.shape[2]).sum(2)
-    ref_v = seg_sum(dog)
-    # tolerance from bf16 rounding of the summed elements: 6 sigma of a random walk of half-ulps
-    tol_k = 6 * torch.sqrt(seg_sum((dk.double() * 2.0 ** -8) ** 2)) + 2e-2
-    tol_v = 6 * torch.sqrt(seg_sum((dv.double() * 2.0 ** -8) ** 2)) + 2e-2
+    dog = do.double().reshape(do.shape[0], hkv, G, do.shape[2])
+    ref_v = seg_sum(dog.sum(2))
+    scale_v = torch.sqrt(seg_sum((dog ** 2).sum(2)))
+    scale_k = torch.sqrt(seg_sum(dk.double() ** 2))
+    tol_k = 0.1 + 2e-3 * scale_k
+    tol_v = 0.1 + 2e-3 * scale_v
     assert torch.all(sk.abs() <= tol_k), f"{what}: sum dK per doc {sk.abs().max().item():.4g}"
     assert torch.all((sv - ref_v).abs() <= tol_v), f"{what}: sum dV per doc {(sv - ref_v).abs().max().item():.4g}"
