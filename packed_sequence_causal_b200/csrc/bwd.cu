@@ -5,28 +5,33 @@
 // already, so the pairs of different chunks are independent and their
 // gradients simply add.
 //
-// Persistent CTA, warp-specialised (320 threads), everything transposed so
-// that a TMEM lane is a key/value row:
-//   warp 0      TMA producer: K, V tile per work item; per iteration the Q and
-//               dO tiles plus the 128 LSE*log2(e) and D values of the q tile.
-//   warp 1      TMEM owner and tcgen05.mma issuer (one thread), per iteration
-//                 S^T  = K Q^T        (M=128 kv, N=128 q, K=D)   -> TMEM S
-//                 dP^T = V dO^T       (M=128 kv, N=128 q, K=D)   -> TMEM dP
-//                 dV  += P^T dO       (M=128 kv, N=D, K=128 q)   -> TMEM dV
-//                 dK  += dS^T Q       (M=128 kv, N=D, K=128 q)   -> TMEM dK
-//                 dQ   = dS K         (M=128 q,  N=D, K=128 kv)  -> TMEM dQ
-//               (dS^T is read as a K-major operand for dK and as an M-major
-//               operand for dQ from the same shared tile).
-//   warps 2..5  thread t owns kv row j = kt*128 + t: P^T_ji = exp2(S*c - LSE2_i)
-//               on the pairs of its document with i >= j (all pairs for FULL
-//               tiles), dS^T = P^T (dP^T - D_i) * scale; both go to 128-byte
-//               swizzled shared tiles as bf16.
-//   warps 6..9  drain dQ from TMEM into the fp32 accumulator with vector
-//               reductions, and write dK, dV (bf16) at the end of a work item.
+// Persistent CTA, warp-specialised (448 threads), transposed so that a TMEM
+// lane is a key/value row:
+//   warp 0       TMA producer: K, V per work item; per iteration Q, dO and the
+//                128 LSE*log2(e) and D values of the q tile, through an
+//                NSQ-stage ring.
+//   warp 1       TMEM owner and tcgen05.mma issuer (one thread), per iteration j
+//                  S^T_j  = K Q_j^T   (M=128 kv, N=128 q, K=D)        -> R1
+//                  dP^T_j = V dO_j^T  (M=128 kv, N=128 q, K=D)        -> R2
+//                  dV    += P^T_j dO_j  (A = P^T from TMEM R1)         -> dV
+//                  S^T_{j+1}          (issued here: R1 is free once dV_j has read P^T_j)
+//                  dK    += dS^T_j Q_j  (A = dS^T from shared memory) -> dK
+//                  dQ_j               (D=128: dQ^T = K^T dS^T -> R2; D=64: dQ = dS K -> DQ)
+//   warps 2..9   two warpgroups, one per half of the 128 q columns; thread t
+//                owns kv row j = kt*128 + t.  P^T = exp2(S^T c - LSE2_i) on the
+//                pairs of its document with i >= j (all pairs for FULL tiles),
+//                written back to TMEM as packed bf16 over its own S columns;
+//                dS^T = P^T (dP^T - D_i) * scale written to a 128-byte swizzled
+//                shared tile as bf16 (read as a K-major operand by dK and as an
+//                MN-major operand by dQ).
+//   warps 10..13 drain dQ from TMEM into the fp32 accumulator (global
+//                reductions, one 128-byte row per warp instruction for D=128),
+//                and write dK, dV (bf16) at the end of a work item.
 //
-// TMEM columns: dK [0,D), dV [D,2D), S [2D,2D+128), dP [2D+128,2D+256),
-// dQ at 384 for D = 64, aliased onto S for D = 128 (S is consumed before dQ
-// is produced; the next S waits until dQ has been drained).
+// TMEM columns: dK [0,D), dV [D,2D), R1 = S^T/P^T [2D, 2D+128),
+// R2 = dP^T [2D+128, 2D+256); dQ shares R2 for D = 128 (dP^T is consumed
+// before dQ is produced, and the next dP^T waits for the drain) and has its
+// own columns [384, 448) for D = 64.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -37,43 +42,48 @@ namespace sap {
 
 template <int D>
 struct BwdCfg {
-  static constexpr int NSQ = (D == 64) ? 2 : 1;  // Q/dO ring depth
-  static constexpr int BOX = 128 * 128;
-  static constexpr int TILE = D * 128 * 2;       // bytes of one 128-row bf16 tile of width D
+  static constexpr int NSQ = (D == 64) ? 3 : 2;  // Q/dO ring depth
+  static constexpr int BOX = 128 * 128;          // one 128-row x 64-column bf16 box
+  static constexpr int TILE = D * 128 * 2;       // one 128-row bf16 tile of width D
   static constexpr int VEC = 128 * 4;            // 128 fp32 values
   static constexpr int STAGE = 2 * TILE + 2 * VEC;
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + TILE;
-  static constexpr int OFF_P = OFF_V + TILE;
-  static constexpr int OFF_DS = OFF_P + 128 * 128 * 2;
+  static constexpr int OFF_DS = OFF_V + TILE;
   static constexpr int OFF_ST = OFF_DS + 128 * 128 * 2;  // stages: Q, dO, lse2, dvec
   static constexpr int OFF_BAR = OFF_ST + NSQ * STAGE;
   static constexpr int NBAR = 2 + 2 * NSQ + 10;
-  static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
-  static constexpr int THREADS = 320;
-  static constexpr uint32_t COL_DK = 0, COL_DV = D, COL_S = 2 * D, COL_DP = 2 * D + 128;
-  static constexpr bool ALIAS_DQ = (D == 128);
-  static constexpr uint32_t COL_DQ = ALIAS_DQ ? COL_S : 384;
+  // The dynamic shared window starts 1024-byte aligned (checked at run time),
+  // so no alignment slack is reserved: the D = 128 layout needs 231,568 bytes.
+  static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16;
+  static constexpr int THREADS = 448;
+  static constexpr uint32_t COL_DK = 0, COL_DV = D, COL_R1 = 2 * D, COL_R2 = 2 * D + 128;
+  static constexpr bool DQ_T = (D == 128);  // dQ^T in R2 (coalesced drain) vs dQ in its own columns
+  static constexpr uint32_t COL_DQ = DQ_T ? COL_R2 : 384;
 };
 
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(448, 1)
     sap_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                    const BwdParams p) {
   using C = BwdCfg<D>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem[];
+  if (smem_u32(smem) & 1023u) {  // TMA 128-byte swizzle and the descriptors need 1024-byte alignment
+    if (threadIdx.x == 0) atomicOr(p.err, kErrSmemAlign);
+    return;
+  }
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* kv_full = bars + 0;
   uint64_t* kv_empty = bars + 1;
-  uint64_t* q_full = bars + 2;           // [NSQ]
-  uint64_t* q_empty = q_full + C::NSQ;   // [NSQ]
+  uint64_t* q_full = bars + 2;          // [NSQ]
+  uint64_t* q_empty = q_full + C::NSQ;  // [NSQ]
   uint64_t* s_full = q_empty + C::NSQ;
   uint64_t* dp_full = s_full + 1;
-  uint64_t* pds_ready = dp_full + 1;
-  uint64_t* pds_free = pds_ready + 1;
-  uint64_t* dq_full = pds_free + 1;
+  uint64_t* p_ready = dp_full + 1;
+  uint64_t* ds_ready = p_ready + 1;
+  uint64_t* ds_free = ds_ready + 1;
+  uint64_t* dq_full = ds_free + 1;
   uint64_t* dq_free = dq_full + 1;
   uint64_t* dkdv_full = dq_free + 1;
   uint64_t* dkdv_free = dkdv_full + 1;
@@ -93,8 +103,9 @@ __global__ void __launch_bounds__(320, 1)
     }
     mbar_init(s_full, 1);
     mbar_init(dp_full, 1);
-    mbar_init(pds_ready, 128);
-    mbar_init(pds_free, 1);
+    mbar_init(p_ready, 256);
+    mbar_init(ds_ready, 256);
+    mbar_init(ds_free, 1);
     mbar_init(dq_full, 1);
     mbar_init(dq_free, 128);
     mbar_init(dkdv_full, 1);
@@ -162,71 +173,79 @@ __global__ void __launch_bounds__(320, 1)
     if (lane == 0) {
       // ----------------------------------------------------------------- MMA
       constexpr uint32_t id_sq = idesc_bf16(128, 128, false, false);  // S^T, dP^T
-      constexpr uint32_t id_kv = idesc_bf16(128, D, false, true);     // dV, dK
-      constexpr uint32_t id_dq = idesc_bf16(128, D, true, true);      // dQ
+      constexpr uint32_t id_kv = idesc_bf16(128, D, false, true);     // dV (A in TMEM), dK
+      constexpr uint32_t id_dq = C::DQ_T ? idesc_bf16(128, 128, true, true) : idesc_bf16(128, D, true, true);
       const uint32_t sK = smem_u32(smem + C::OFF_K), sV = smem_u32(smem + C::OFF_V);
-      const uint32_t sP = smem_u32(smem + C::OFF_P), sDS = smem_u32(smem + C::OFF_DS);
+      const uint32_t sDS = smem_u32(smem + C::OFF_DS);
       const uint32_t sST = smem_u32(smem + C::OFF_ST);
-      uint32_t unit_iter = 0, it = 0;  // it: global iteration counter
+      const uint32_t R1 = tmem + C::COL_R1, R2 = tmem + C::COL_R2;
+      uint32_t unit_iter = 0, it = 0;  // it: global iteration counter (all barriers below count per iteration)
       bool ok = true;
+      auto stage_q = [&](uint32_t i) { return sST + (i % C::NSQ) * C::STAGE; };
+      auto issue_s = [&](uint32_t i) -> bool {  // S^T_i = K Q_i^T -> R1
+        if (!mbar_wait(q_full + i % C::NSQ, (i / C::NSQ) & 1, guard, kErrTimeoutMma)) return false;
+        tc_fence_after();
+        const uint32_t sQ = stage_q(i);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t ko = (kk / 4) * C::BOX + (kk % 4) * 32;
+          mma_bf16(R1, sdesc_sw128(sK + ko, 16, 1024), sdesc_sw128(sQ + ko, 16, 1024), id_sq, kk > 0);
+        }
+        tc_commit(s_full);
+        return true;
+      };
       for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
         const int u = w / p.hkv;
-        const int ne = p.kv_units[3 * u + 2];
-        const int n_it = ne * G;
+        const int n_it = p.kv_units[3 * u + 2] * G;
         if (!mbar_wait(kv_full, unit_iter & 1, guard, kErrTimeoutMma)) break;
+        tc_fence_after();
+        if (!issue_s(it)) break;
         for (int j = 0; j < n_it; ++j, ++it) {
-          const int s = it % C::NSQ;
-          const uint32_t ph = (it / C::NSQ) & 1;
-          const uint32_t sQ = sST + s * C::STAGE, sDO = sQ + C::TILE;
-          if (!mbar_wait(q_full + s, ph, guard, kErrTimeoutMma)) { ok = false; break; }
-          // S^T may overwrite the dQ of the previous iteration when they share columns.
-          if (C::ALIAS_DQ && it > 0 && !mbar_wait(dq_free, (it - 1) & 1, guard, kErrTimeoutMma)) { ok = false; break; }
+          const uint32_t sQ = stage_q(it), sDO = sQ + C::TILE;
+          // dP^T_j -> R2 once the previous dQ (D = 128: same columns) has been drained
+          if (C::DQ_T && it > 0 && !mbar_wait(dq_free, (it - 1) & 1, guard, kErrTimeoutMma)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t ko = (kk / 4) * C::BOX + (kk % 4) * 32;
-            mma_bf16(tmem + C::COL_S, sdesc_sw128(sK + ko, 16, 1024), sdesc_sw128(sQ + ko, 16, 1024), id_sq,
-                     kk > 0);
-          }
-          tc_commit(s_full);
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t ko = (kk / 4) * C::BOX + (kk % 4) * 32;
-            mma_bf16(tmem + C::COL_DP, sdesc_sw128(sV + ko, 16, 1024), sdesc_sw128(sDO + ko, 16, 1024), id_sq,
-                     kk > 0);
+            mma_bf16(R2, sdesc_sw128(sV + ko, 16, 1024), sdesc_sw128(sDO + ko, 16, 1024), id_sq, kk > 0);
           }
           tc_commit(dp_full);
-          // P^T and dS^T of this iteration are in shared memory.
-          if (!mbar_wait(pds_ready, it & 1, guard, kErrTimeoutMma)) { ok = false; break; }
-          // dK/dV of the previous work item must have been read out before they restart.
+          // dV += P^T_j dO_j, P^T in TMEM (packed bf16 over the S^T columns of each half)
+          if (!mbar_wait(p_ready, it & 1, guard, kErrTimeoutMma)) { ok = false; break; }
           if (j == 0 && unit_iter > 0 && !mbar_wait(dkdv_free, (unit_iter - 1) & 1, guard, kErrTimeoutMma)) {
             ok = false;
             break;
           }
           tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < 128 / 16; ++kk) {  // dV += P^T dO
-            const uint64_t a = sdesc_sw128(sP + (kk / 4) * C::BOX + (kk % 4) * 32, 16, 1024);
-            const uint64_t b = sdesc_sw128(sDO + kk * 2048, C::BOX, 1024);
-            mma_bf16(tmem + C::COL_DV, a, b, id_kv, (j > 0 || kk > 0) ? 1u : 0u);
-          }
-#pragma unroll
-          for (int kk = 0; kk < 128 / 16; ++kk) {  // dK += dS^T Q
-            const uint64_t a = sdesc_sw128(sDS + (kk / 4) * C::BOX + (kk % 4) * 32, 16, 1024);
-            const uint64_t b = sdesc_sw128(sQ + kk * 2048, C::BOX, 1024);
-            mma_bf16(tmem + C::COL_DK, a, b, id_kv, (j > 0 || kk > 0) ? 1u : 0u);
-          }
-          if (!C::ALIAS_DQ && it > 0 && !mbar_wait(dq_free, (it - 1) & 1, guard, kErrTimeoutMma)) { ok = false; break; }
+          for (int kk = 0; kk < 128 / 16; ++kk)
+            mma_bf16_tmem_a(tmem + C::COL_DV, R1 + (kk / 4) * 64 + (kk % 4) * 8,
+                            sdesc_sw128(sDO + kk * 2048, C::BOX, 1024), id_kv, (j > 0 || kk > 0) ? 1u : 0u);
+          // S^T_{j+1}: R1 is rewritten only after dV_j (issued above) has read P^T_j
+          if (j + 1 < n_it && !issue_s(it + 1)) { ok = false; break; }
+          // dK += dS^T_j Q_j ; dQ_j
+          if (!mbar_wait(ds_ready, it & 1, guard, kErrTimeoutMma)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < 128 / 16; ++kk) {  // dQ = dS K
-            const uint64_t a = sdesc_sw128(sDS + kk * 2048, C::BOX, 1024);
-            const uint64_t b = sdesc_sw128(sK + kk * 2048, C::BOX, 1024);
-            mma_bf16(tmem + C::COL_DQ, a, b, id_dq, kk > 0);
+          for (int kk = 0; kk < 128 / 16; ++kk) {
+            const uint64_t a = sdesc_sw128(sDS + (kk / 4) * C::BOX + (kk % 4) * 32, 16, 1024);
+            mma_bf16(tmem + C::COL_DK, a, sdesc_sw128(sQ + kk * 2048, C::BOX, 1024), id_kv,
+                     (j > 0 || kk > 0) ? 1u : 0u);
+          }
+          if (!C::DQ_T && it > 0 && !mbar_wait(dq_free, (it - 1) & 1, guard, kErrTimeoutMma)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 128 / 16; ++kk) {
+            // D=128: dQ^T[d][q] = sum_kv K[kv][d] dS^T[kv][q]  (A = K, B = dS^T, both MN-major)
+            // D=64 : dQ[q][d]   = sum_kv dS^T[kv][q] K[kv][d]  (A = dS^T, B = K, both MN-major)
+            const uint64_t kd = sdesc_sw128(sK + kk * 2048, C::BOX, 1024);
+            const uint64_t sd = sdesc_sw128(sDS + kk * 2048, C::BOX, 1024);
+            mma_bf16(tmem + C::COL_DQ, C::DQ_T ? kd : sd, C::DQ_T ? sd : kd, id_dq, kk > 0);
           }
           tc_commit(dq_full);
-          tc_commit(pds_free);
-          tc_commit(q_empty + s);
+          tc_commit(ds_free);
+          tc_commit(q_empty + it % C::NSQ);
         }
         if (!ok) break;
         tc_commit(dkdv_full);
@@ -236,13 +255,14 @@ __global__ void __launch_bounds__(320, 1)
       tc_commit(mma_drain);
       drain_wait(mma_drain, 0);
     }
-  } else if (warp < 6) {
-    // ------------------------------------------------------- P^T and dS^T
+  } else if (warp < 10) {
+    // ----------------------------------------------------- P^T and dS^T
     const int quad = warp & 3;
-    const int t = quad * 32 + lane;  // kv row within the tile
+    const int half = (warp - 2) >> 2;  // q columns [64*half, 64*half + 64)
+    const int t = quad * 32 + lane;    // kv row within the tile
     const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
-    uint8_t* sPt = smem + C::OFF_P;
-    uint8_t* sDSt = smem + C::OFF_DS;
+    const uint32_t R1 = lane_base + C::COL_R1 + 64 * half, R2 = lane_base + C::COL_R2 + 64 * half;
+    uint8_t* sDSt = smem + C::OFF_DS + half * C::BOX;
     const float sl2 = p.scale_log2, scale = p.scale;
     uint32_t it = 0;
     bool ok = true;
@@ -251,53 +271,62 @@ __global__ void __launch_bounds__(320, 1)
       const int kt = p.kv_units[3 * u], e0 = p.kv_units[3 * u + 1], ne = p.kv_units[3 * u + 2];
       const int64_t jrow = (int64_t)kt * 128 + t;
       const bool real_row = jrow < p.n;
-      const int j_lo = real_row ? (int)jrow : 1;              // queries i with j <= i <= last token of the doc
+      const int j_lo = real_row ? (int)jrow : 1;  // queries i with j <= i <= last token of the document
       const int j_hi = real_row ? p.tok_hi[jrow] : 0;
       for (int hh = 0; hh < G && ok; ++hh) {
         for (int e = 0; e < ne; ++e, ++it) {
           const int qt = p.entries[2 * (e0 + e)], tag = p.entries[2 * (e0 + e) + 1];
-          const int s = it % C::NSQ;
-          const uint32_t ph = (it / C::NSQ) & 1;
-          const float* lse2 = reinterpret_cast<const float*>(smem + C::OFF_ST + s * C::STAGE + 2 * C::TILE);
+          const float* lse2 =
+              reinterpret_cast<const float*>(smem + C::OFF_ST + (it % C::NSQ) * C::STAGE + 2 * C::TILE) + 64 * half;
           const float* dvec = lse2 + 128;
-          if (!mbar_wait_warp(q_full + s, ph, guard, kErrTimeoutSoftmax)) { ok = false; break; }
+          const int c_lo = j_lo - qt * 128 - 64 * half, c_hi = j_hi - qt * 128 - 64 * half;
+          if (!mbar_wait_warp(q_full + it % C::NSQ, (it / C::NSQ) & 1, guard, kErrTimeoutSoftmax)) { ok = false; break; }
           if (!mbar_wait_warp(s_full, it & 1, guard, kErrTimeoutSoftmax)) { ok = false; break; }
-          if (!mbar_wait_warp(dp_full, it & 1, guard, kErrTimeoutSoftmax)) { ok = false; break; }
-          if (it > 0 && !mbar_wait_warp(pds_free, (it - 1) & 1, guard, kErrTimeoutSoftmax)) { ok = false; break; }
           tc_fence_after();
-          const int c_lo = j_lo - qt * 128, c_hi = j_hi - qt * 128;
-#pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
-            float sv[32], dpv[32];
-            tmem_ld32(lane_base + C::COL_S + 32 * c, sv);
-            tmem_ld32(lane_base + C::COL_DP + 32 * c, dpv);
-            uint32_t pw[16], dw[16];
+          float pr[64];
+          {
+            float sv[32];
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+              tmem_ld32(R1 + 32 * c, sv);
+#pragma unroll
+              for (int e2 = 0; e2 < 32; ++e2) {
+                const int col = 32 * c + e2;
+                const bool valid = (tag == 0) || (col >= c_lo && col <= c_hi);
+                pr[col] = valid ? ex2(fmaf(sv[e2], sl2, -lse2[col])) : 0.f;
+              }
+            }
+            uint32_t pk[32];
+#pragma unroll
+            for (int e2 = 0; e2 < 32; ++e2) pk[e2] = pack_bf16x2(pr[2 * e2], pr[2 * e2 + 1]);
+            tmem_st32_u(R1, pk);  // P^T over this half's first 32 S^T columns (already read)
+          }
+          tc_fence_before();
+          mbar_arrive(p_ready);
+          if (!mbar_wait_warp(dp_full, it & 1, guard, kErrTimeoutSoftmax)) { ok = false; break; }
+          if (it > 0 && !mbar_wait_warp(ds_free, (it - 1) & 1, guard, kErrTimeoutSoftmax)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            float dpv[32];
+            tmem_ld32(R2 + 32 * c, dpv);
+            uint32_t dw[16];
 #pragma unroll
             for (int e2 = 0; e2 < 32; e2 += 2) {
-              float pp[2], dd[2];
-#pragma unroll
-              for (int q = 0; q < 2; ++q) {
-                const int col = 32 * c + e2 + q;
-                const bool valid = (tag == 0) || (col >= c_lo && col <= c_hi);
-                const float pr = valid ? ex2(fmaf(sv[e2 + q], sl2, -lse2[col])) : 0.f;
-                pp[q] = pr;
-                dd[q] = pr * (dpv[e2 + q] - dvec[col]) * scale;
-              }
-              pw[e2 / 2] = pack_bf16x2(pp[0], pp[1]);
-              dw[e2 / 2] = pack_bf16x2(dd[0], dd[1]);
+              const int col = 32 * c + e2;
+              const float d0 = pr[col] * (dpv[e2] - dvec[col]) * scale;
+              const float d1 = pr[col + 1] * (dpv[e2 + 1] - dvec[col + 1]) * scale;
+              dw[e2 / 2] = pack_bf16x2(d0, d1);
             }
-            // columns 32c .. 32c+31 = 16-byte chunks 4c .. 4c+3 of the 128-column row
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-              const int cc = 4 * c + q4;
-              const uint32_t off = (cc / 8) * C::BOX + sw128_offset(t, cc % 8);
-              st_shared_v4(smem_u32(sPt + off), pw[4 * q4], pw[4 * q4 + 1], pw[4 * q4 + 2], pw[4 * q4 + 3]);
+            for (int q4 = 0; q4 < 4; ++q4) {  // 16-byte chunks 4c .. 4c+3 of this half's 64 columns
+              const uint32_t off = sw128_offset(t, 4 * c + q4);
               st_shared_v4(smem_u32(sDSt + off), dw[4 * q4], dw[4 * q4 + 1], dw[4 * q4 + 2], dw[4 * q4 + 3]);
             }
           }
           fence_async_smem();
           tc_fence_before();
-          mbar_arrive(pds_ready);
+          mbar_arrive(ds_ready);
         }
       }
     }
@@ -317,14 +346,29 @@ __global__ void __launch_bounds__(320, 1)
           const int qt = p.entries[2 * (e0 + e)];
           if (!mbar_wait_warp(dq_full, it & 1, guard, kErrTimeoutEpilogue)) { ok = false; break; }
           tc_fence_after();
-          float* dst = p.dq_acc + (((size_t)qt * 128 + t) * p.hq + h) * D;
+          if (C::DQ_T) {
+            // lane t = feature t of dQ; a warp's reductions for one q row cover 32 consecutive floats
+            float* dst = p.dq_acc + ((size_t)qt * 128 * p.hq + h) * D + t;
+            const size_t row_stride = (size_t)p.hq * D;
 #pragma unroll 1
-          for (int c = 0; c < D / 32; ++c) {
-            float v[32];
-            tmem_ld32(lane_base + C::COL_DQ + 32 * c, v);
+            for (int c = 0; c < 4; ++c) {
+              float v[32];
+              tmem_ld32(lane_base + C::COL_DQ + 32 * c, v);
 #pragma unroll
-            for (int e4 = 0; e4 < 32; e4 += 4)
-              atomicAdd(reinterpret_cast<float4*>(dst + 32 * c + e4), make_float4(v[e4], v[e4 + 1], v[e4 + 2], v[e4 + 3]));
+              for (int e2 = 0; e2 < 32; ++e2) atomicAdd(dst + (size_t)(32 * c + e2) * row_stride, v[e2]);
+            }
+          } else {
+            // lane t = q row t of the tile
+            float* dst = p.dq_acc + (((size_t)qt * 128 + t) * p.hq + h) * D;
+#pragma unroll 1
+            for (int c = 0; c < D / 32; ++c) {
+              float v[32];
+              tmem_ld32(lane_base + C::COL_DQ + 32 * c, v);
+#pragma unroll
+              for (int e4 = 0; e4 < 32; e4 += 4)
+                atomicAdd(reinterpret_cast<float4*>(dst + 32 * c + e4),
+                          make_float4(v[e4], v[e4 + 1], v[e4 + 2], v[e4 + 3]));
+            }
           }
           tc_fence_before();
           mbar_arrive(dq_free);

@@ -36,7 +36,7 @@ def _check_workload(name, seed=0, kv_heads=(0,), q_heads_fwd=None, budget=3e10):
     if not w.backward:
         return
     dq, dk, dv = r.bwd()
-    doc_sum_identities(dk, dv, r.do, cu, w.hq, w.hkv, name)
+    doc_sum_identities(dk, dv, r.do, r.q, r.scale, cu, w.hq, w.hkv, name)
     for g in kv_heads:
         heads = list(range(g * G, (g + 1) * G))
         arrays = oracle.widen(b.q[:, heads].cpu(), b.k[:, g:g + 1].cpu(), b.v[:, g:g + 1].cpu(),
