@@ -171,12 +171,17 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=1e11, help="unmasked FLOPs of the CPU-baseline sample")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="run the workload's recipe at a smaller token count (profiling captures only)")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     w = workloads.WORKLOADS[args.workload]
+    if args.tokens:
+        import dataclasses
+        w = dataclasses.replace(w, n=args.tokens, big=min(w.big, args.tokens), name=f"{w.name}@{args.tokens}")
 
     if args.impl == "reference":
         return run_reference(args, w, rank, world)
@@ -191,7 +196,7 @@ def main():
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
-    b = workloads.make_batch(w.name, args.seed + rank, device=str(dev), with_do=True)
+    b = workloads.make_batch(w, args.seed + rank, device=str(dev), with_do=True)
     n, hq, hkv, d = w.n, w.hq, w.hkv, w.d
     scale = 1.0 / math.sqrt(d)
     t_plan = time.perf_counter()
@@ -361,7 +366,7 @@ def run_reference(args, w, rank, world):
     if rank != 0:
         return
     import oracle
-    b = workloads.make_batch(w.name, args.seed, device="cpu", with_do=True)
+    b = workloads.make_batch(w, args.seed, device="cpu", with_do=True)
     budget = args.cpu_budget / 3
     for _ in range(args.warmup):
         run_oracle_sample(b, budget / 4)

@@ -130,10 +130,13 @@ def doc_sum_identities(dk, dv, do, q, scale: float, cu, hq: int, hkv: int, what:
     in exact arithmetic; sum_j P_ij is 1 only in exact arithmetic), so its
     natural scale is that of a random walk over the document's rows and heads:
     sqrt(sum dO^2) for dV and softmax_scale * sqrt(sum Q^2) for dK (per
-    element).  Tolerance: 0.1 + 2e-3 * that scale.  Against the full oracle on
-    a 16K-token batch with an 8K-token document the per-document sums deviate
-    from the exact sums by at most 3e-4 of the dV scale, so the bound leaves
-    headroom; a dropped near-diagonal tile moves a sum by O(1).
+    element).  Tolerance: 0.1 + 4e-3 * that scale.  Measured deviations of the
+    kernel's per-document sums: at most 3e-4 of the dV scale against the full
+    oracle on a 16K-token batch with an 8K-token document, and 1.4e-3 of it
+    for the 256K-token document of the 512K batch, whose individual dK/dV rows
+    (its first keys included) are all within the element bound against an
+    independent fp64 computation; a dropped near-diagonal tile moves a sum by
+    O(1).
     """
     G = hq // hkv
     cu_t = torch.as_tensor(np.asarray(cu, dtype=np.int64), device=dk.device)
@@ -153,7 +156,7 @@ def doc_sum_identities(dk, dv, do, q, scale: float, cu, hq: int, hkv: int, what:
     scale_v = torch.sqrt(seg_sum((dog ** 2).sum(2)))
     qg = q.double().reshape(q.shape[0], hkv, G, q.shape[2])
     scale_k = scale * torch.sqrt(seg_sum((qg ** 2).sum(2)))
-    tol_k = 0.1 + 2e-3 * scale_k
-    tol_v = 0.1 + 2e-3 * scale_v
+    tol_k = 0.1 + 4e-3 * scale_k
+    tol_v = 0.1 + 4e-3 * scale_v
     assert torch.all(sk.abs() <= tol_k), f"{what}: sum dK per doc {sk.abs().max().item():.4g}"
     assert torch.all((sv - ref_v).abs() <= tol_v), f"{what}: sum dV per doc {(sv - ref_v).abs().max().item():.4g}"
