@@ -106,7 +106,7 @@ int sap_plan_fwd_schedule(sap_plan_t plan, const int32_t** units, int64_t* n_uni
 
 /* Backward schedule, host memory owned by the plan:
  *   kv_units: int32[n_kv_units][3] = (kv_tile, first_entry, n_entries), heavy-first;
- *   entries:  int32[n_items][2] = (q_tile, tag), grouped by kv tile, q-tile ascending. */
+ *   entries:  int32[n_items][2] = (q_tile, tag), grouped by kv tile, q-tile descending. */
 int sap_plan_bwd_schedule(sap_plan_t plan, const int32_t** kv_units, int64_t* n_kv_units, const int32_t** entries);
 
 /* Copy the plan's device arrays to the current device on `stream`.  Called

@@ -144,10 +144,13 @@ __global__ void __launch_bounds__(448, 1)
           tma_load_3d(smem + C::OFF_K + b * C::BOX, &tmK, kv_full, 64 * b, g, kt * 128);
           tma_load_3d(smem + C::OFF_V + b * C::BOX, &tmV, kv_full, 64 * b, g, kt * 128);
         }
-        for (int hh = 0; hh < G && ok; ++hh) {
-          const int h = g * G + hh;
-          for (int e = 0; e < ne; ++e) {
-            const int qt = p.entries[2 * (e0 + e)];
+        // entries are walked q-tile outer, head inner; the next q tile is fetched one entry ahead
+        int qt_next = p.entries[2 * e0];
+        for (int e = 0; e < ne && ok; ++e) {
+          const int qt = qt_next;
+          if (e + 1 < ne) qt_next = p.entries[2 * (e0 + e + 1)];
+          for (int hh = 0; hh < G; ++hh) {
+            const int h = g * G + hh;
             const int s = q_iter % C::NSQ;
             const uint32_t ph = (q_iter / C::NSQ) & 1;
             if (!mbar_wait(q_empty + s, ph ^ 1, guard, kErrTimeoutLoad)) { ok = false; break; }
@@ -273,9 +276,11 @@ __global__ void __launch_bounds__(448, 1)
       const bool real_row = jrow < p.n;
       const int j_lo = real_row ? (int)jrow : 1;  // queries i with j <= i <= last token of the document
       const int j_hi = real_row ? p.tok_hi[jrow] : 0;
-      for (int hh = 0; hh < G && ok; ++hh) {
-        for (int e = 0; e < ne; ++e, ++it) {
-          const int qt = p.entries[2 * (e0 + e)], tag = p.entries[2 * (e0 + e) + 1];
+      int qt_next = p.entries[2 * e0], tag_next = p.entries[2 * e0 + 1];
+      for (int e = 0; e < ne && ok; ++e) {
+        const int qt = qt_next, tag = tag_next;
+        if (e + 1 < ne) qt_next = p.entries[2 * (e0 + e + 1)], tag_next = p.entries[2 * (e0 + e + 1) + 1];
+        for (int hh = 0; hh < G; ++hh, ++it) {
           const float* lse2 =
               reinterpret_cast<const float*>(smem + C::OFF_ST + (it % C::NSQ) * C::STAGE + 2 * C::TILE) + 64 * half;
           const float* dvec = lse2 + 128;
@@ -340,10 +345,12 @@ __global__ void __launch_bounds__(448, 1)
     for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
       const int u = w / p.hkv, g = w % p.hkv;
       const int kt = p.kv_units[3 * u], e0 = p.kv_units[3 * u + 1], ne = p.kv_units[3 * u + 2];
-      for (int hh = 0; hh < G && ok; ++hh) {
-        const int h = g * G + hh;
-        for (int e = 0; e < ne; ++e, ++it) {
-          const int qt = p.entries[2 * (e0 + e)];
+      int qt_next = p.entries[2 * e0];
+      for (int e = 0; e < ne && ok; ++e) {
+        const int qt = qt_next;
+        if (e + 1 < ne) qt_next = p.entries[2 * (e0 + e + 1)];
+        for (int hh = 0; hh < G; ++hh, ++it) {
+          const int h = g * G + hh;
           if (!mbar_wait_warp(dq_full, it & 1, guard, kErrTimeoutEpilogue)) { ok = false; break; }
           tc_fence_after();
           if (C::DQ_T) {

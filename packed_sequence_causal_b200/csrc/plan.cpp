@@ -127,16 +127,19 @@ int sap_plan_build(const int32_t* cu, int32_t num_docs, int64_t n, int32_t num_c
   std::stable_sort(p->fwd_order.begin(), p->fwd_order.end(),
                    [&](int32_t x, int32_t y) { return p->fwd_units[4 * x + 2] > p->fwd_units[4 * y + 2]; });
 
-  // backward: items grouped by kv tile (counting sort keeps q-tile ascending)
+  // backward: items grouped by kv tile, q-tile descending within a kv tile.
+  // The backward kernel walks each list in this order, so the persistent CTAs
+  // (which start their heavy kv tiles together) sweep the q tiles from the
+  // top down roughly in step and share Q, dO and dQ rows in L2.
   const int64_t ntk = (n + block_n - 1) / block_n;
   std::vector<int64_t> cnt((size_t)ntk + 1, 0);
   for (const auto& it : p->items) cnt[(size_t)it.kv_tile + 1]++;
   for (int64_t t = 0; t < ntk; ++t) cnt[t + 1] += cnt[t];
   p->kv_entries.assign(p->items.size() * 2, 0);
   {
-    std::vector<int64_t> pos(cnt.begin(), cnt.end() - 1);
+    std::vector<int64_t> pos(cnt.begin() + 1, cnt.end());  // fill each group from its end
     for (const auto& it : p->items) {
-      int64_t w = pos[it.kv_tile]++;
+      int64_t w = --pos[it.kv_tile];
       p->kv_entries[2 * w] = it.q_tile;
       p->kv_entries[2 * w + 1] = it.tag;
     }

@@ -53,13 +53,13 @@ def _check_schedules(plan, items, n, nchunks, bm, bn):
     for a, b in zip(order[:-1], order[1:]):
         if units[a, 2] == units[b, 2]:
             assert a < b
-    # backward: every item once, grouped by kv tile, q-tile ascending, heavy-first
+    # backward: every item once, grouped by kv tile, q-tile descending, heavy-first
     kv_units, entries = sap.sap_plan_bwd_schedule(plan)
     seen = set()
     prev_cnt = None
     for kt, e0, ne in kv_units:
         grp = entries[e0:e0 + ne]
-        assert np.all(np.diff(grp[:, 0]) > 0)
+        assert np.all(np.diff(grp[:, 0]) < 0)
         for qt, tag in grp:
             seen.add((int(qt), int(kt), int(tag)))
         if prev_cnt is not None:
