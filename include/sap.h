@@ -149,6 +149,31 @@ int sap_attn_bwd(sap_plan_t plan, const void* q, const void* k, const void* v, c
                  const void* dout, int32_t hq, int32_t hkv, int32_t head_dim, float softmax_scale, void* dq,
                  void* dk, void* dv, void* workspace, size_t ws_bytes, void* stream);
 
+/* Forward + merge (the same kernels as sap_attn_fwd followed by sap_merge)
+ * without any device allocation: the partial outputs and LSEs live in a
+ * 16 MiB array compiled into the library instead of a caller-owned workspace.
+ * The paper has no counterpart; this call exists for callers that cannot call
+ * cudaMalloc -- for example code whose framework owns all device memory
+ * through its own pool, or a plugin that is handed only its input and output
+ * pointers.
+ *   - The plan must already be uploaded to the current device
+ *     (sap_plan_upload, or any earlier device call with it), because uploading
+ *     allocates; otherwise SAP_ERR_INVALID_ARG.
+ *   - Plans whose forward workspace (sap_workspace_size with SAP_WS_FWD)
+ *     exceeds 16 MiB are rejected with SAP_ERR_WORKSPACE.
+ *   - The first call on a device looks up the array's device address (and the
+ *     library's other per-device handles); make that first call before any
+ *     stream capture begins.
+ *   - All calls on a device share that device's one array, which keeps the
+ *     last call's contents.  Calls that may run at the same time on one GPU
+ *     (for example on two streams) race on it: serialise them.
+ *   - Every device on which the library's kernels are loaded holds the 16 MiB
+ *     until the process exits.
+ * Arguments, layouts and errors are otherwise those of sap_attn_fwd. */
+int sap_attn_fwd_static_scratch(sap_plan_t plan, const void* q, const void* k, const void* v, int32_t hq,
+                                int32_t hkv, int32_t head_dim, float softmax_scale, void* o, float* lse,
+                                void* stream);
+
 /* Synchronise the current device and return SAP_OK, or SAP_ERR_DEVICE if a
  * kernel set the device error word (its code is stored in *code, then the word
  * is cleared). */

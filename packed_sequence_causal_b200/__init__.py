@@ -19,6 +19,7 @@ from ._capi import (  # noqa: F401
     load_library,
     sap_attn_bwd,
     sap_attn_fwd,
+    sap_attn_fwd_static_scratch,
     sap_device_status,
     sap_error_string,
     sap_merge,

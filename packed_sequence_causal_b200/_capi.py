@@ -63,6 +63,8 @@ def load_library():
     L.sap_merge.argtypes = [P, P, sz, i32, i32, P, P, P]
     L.sap_attn_bwd.restype = ctypes.c_int
     L.sap_attn_bwd.argtypes = [P, P, P, P, P, P, P, i32, i32, i32, f32, P, P, P, P, sz, P]
+    L.sap_attn_fwd_static_scratch.restype = ctypes.c_int
+    L.sap_attn_fwd_static_scratch.argtypes = [P, P, P, P, i32, i32, i32, f32, P, P, P]
     L.sap_device_status.restype = ctypes.c_int
     L.sap_device_status.argtypes = [ctypes.POINTER(i32)]
     L.sap_error_string.restype = ctypes.c_char_p
@@ -211,6 +213,21 @@ def sap_attn_bwd(plan: Plan, q, k, v, o, lse, dout, softmax_scale: float, dq, dk
     _check(load_library().sap_attn_bwd(plan.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), hq,
                                        hkv, d, float(softmax_scale), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace),
                                        _nbytes(workspace), ctypes.c_void_p(_stream_ptr(stream))), "sap_attn_bwd")
+
+
+def sap_attn_fwd_static_scratch(plan: Plan, q, k, v, softmax_scale: float, o, lse, stream=None):
+    """Forward + merge with the partials in the library's own 16 MiB device array (no allocation).
+
+    For callers that cannot allocate device memory; the plan must already be
+    uploaded to the current device, and calls must not overlap on one GPU."""
+    for t, nme in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
+        _bf16_3d(t, nme)
+    _, hq, d = q.shape
+    hkv = k.shape[1]
+    _check(load_library().sap_attn_fwd_static_scratch(plan.handle, _ptr(q), _ptr(k), _ptr(v), hq, hkv, d,
+                                                      float(softmax_scale), _ptr(o), _ptr(lse),
+                                                      ctypes.c_void_p(_stream_ptr(stream))),
+           "sap_attn_fwd_static_scratch")
 
 
 def sap_device_status() -> int:

@@ -120,6 +120,31 @@ BwdWs bwd_ws(const sap_plan_s* p, int32_t hq, int32_t hd) {
   return w;
 }
 
+// Scratch for sap_attn_fwd_static_scratch: the forward's partial outputs and
+// LSEs live here instead of in a caller-allocated workspace.  Every GPU that
+// loads the library holds these 16 MiB until the process exits.
+constexpr size_t kStaticScratchBytes = size_t(16) << 20;
+static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
+
+// Device address of g_static_scratch per device, looked up once with that
+// device current (host code must not use the symbol itself as a pointer).
+void* g_static_scratch_addr[kMaxDevices] = {};
+std::mutex g_static_scratch_mu;
+
+int static_scratch_address(void** out) {
+  int dev = 0;
+  SAP_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) return SAP_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lk(g_static_scratch_mu);
+  if (!g_static_scratch_addr[dev]) {
+    void* ptr = nullptr;
+    SAP_CUDA(cudaGetSymbolAddress(&ptr, g_static_scratch));
+    g_static_scratch_addr[dev] = ptr;
+  }
+  *out = g_static_scratch_addr[dev];
+  return SAP_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -418,5 +443,67 @@ const char* sap_error_string(int status) {
 }
 
 int sap_last_cuda_error(void) { return g_last_cuda_error; }
+
+int sap_attn_fwd_static_scratch(sap_plan_t p, const void* q, const void* k, const void* v, int32_t hq, int32_t hkv,
+                                int32_t head_dim, float softmax_scale, void* o, float* lse, void* stream) {
+  int rc = check_kernel_plan(p);
+  if (rc) return rc;
+  if ((rc = check_heads(hq, hkv, head_dim))) return rc;
+  if (p->n == 0) return SAP_OK;
+  if (!q || !k || !v || !o || !lse) return SAP_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return SAP_ERR_INVALID_ARG;
+  // Uploading a plan allocates device memory, so this call only accepts a plan
+  // already uploaded to the current device.
+  int dev = 0;
+  SAP_CUDA(cudaGetDevice(&dev));
+  if (!p->dev || p->dev_id != dev) return SAP_ERR_INVALID_ARG;
+  const FwdWs ws = fwd_ws(p, hq, head_dim);
+  if (ws.total > kStaticScratchBytes) return SAP_ERR_WORKSPACE;
+  DeviceInfo* di = nullptr;
+  if ((rc = device_info(&di))) return rc;
+  void* scratch = nullptr;
+  if ((rc = static_scratch_address(&scratch))) return rc;
+  CUtensorMap tq, tk, tv;
+  if ((rc = make_map(&tq, q, p->n, hq, head_dim))) return rc;
+  if ((rc = make_map(&tk, k, p->n, hkv, head_dim))) return rc;
+  if ((rc = make_map(&tv, v, p->n, hkv, head_dim))) return rc;
+  const int32_t* base = static_cast<const int32_t*>(p->dev);
+  uint8_t* wsb = static_cast<uint8_t*>(scratch);
+  sap::FwdParams fp;
+  fp.items = base + p->off_items;
+  fp.units = base + p->off_units;
+  fp.order = base + p->off_order;
+  fp.tok_lo = base + p->off_tok_lo;
+  fp.n_units = (int32_t)(p->fwd_units.size() / 4);
+  fp.hq = hq;
+  fp.group = hq / hkv;
+  fp.n = p->n;
+  fp.scale_log2 = softmax_scale * 1.4426950408889634f;
+  fp.o = static_cast<__nv_bfloat16*>(o);
+  fp.lse = lse;
+  // Every (slot, head, row) partial that the merge reads is written by this
+  // call's forward kernel first, so nothing in the scratch needs clearing.
+  fp.o_part = reinterpret_cast<float*>(wsb + ws.o_part);
+  fp.lse_part = reinterpret_cast<float*>(wsb + ws.lse_part);
+  fp.err = di->err;
+  const int64_t work = (int64_t)fp.n_units * hq;
+  if (work == 0) return SAP_OK;
+  if (work > INT32_MAX) return SAP_ERR_INVALID_ARG;
+  const int grid = (int)(work < di->sms ? work : di->sms);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = head_dim == 64 ? sap::launch_fwd<64>(tq, tk, tv, fp, grid, s)
+                                 : sap::launch_fwd<128>(tq, tk, tv, fp, grid, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  const int64_t n_merges = (int64_t)p->merges.size() / 3;
+  if (n_merges > 0) {
+    e = head_dim == 64 ? sap::launch_merge<64>(base + p->off_merges, n_merges, hq, p->n, fp.o_part, fp.lse_part,
+                                               fp.o, lse, s)
+                       : sap::launch_merge<128>(base + p->off_merges, n_merges, hq, p->n, fp.o_part, fp.lse_part,
+                                                fp.o, lse, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  return SAP_OK;
+}
 
 }  // extern "C"
