@@ -78,6 +78,20 @@ int make_map(CUtensorMap* map, const void* base, int64_t rows, int32_t heads, in
   return SAP_OK;
 }
 
+// fp32 dQ accumulator [rows][heads][hd] -> 3-D map whose box is one q tile of one head
+// (128 rows x hd features, no swizzle): the target of the backward's bulk reductions.
+int make_map_f32_tile(CUtensorMap* map, void* base, int64_t rows, int32_t heads, int32_t hd) {
+  cuuint64_t dims[3] = {(cuuint64_t)hd, (cuuint64_t)heads, (cuuint64_t)rows};
+  cuuint64_t strides[2] = {(cuuint64_t)hd * 4, (cuuint64_t)heads * hd * 4};
+  cuuint32_t box[3] = {(cuuint32_t)hd, 1, 128};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
+  return SAP_OK;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
@@ -372,6 +386,8 @@ int sap_attn_bwd(sap_plan_t p, const void* q, const void* k, const void* v, cons
   if ((rc = make_map(&tdo, dout, p->n, hq, head_dim))) return rc;
   uint8_t* wsb = static_cast<uint8_t*>(workspace);
   float* dq_acc = reinterpret_cast<float*>(wsb + ws.dq_acc);
+  CUtensorMap tdq;
+  if ((rc = make_map_f32_tile(&tdq, dq_acc, ws.n_pad, hq, head_dim))) return rc;
   float* dvec = reinterpret_cast<float*>(wsb + ws.dvec);
   float* lse2 = reinterpret_cast<float*>(wsb + ws.lse2);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -402,8 +418,8 @@ int sap_attn_bwd(sap_plan_t p, const void* q, const void* k, const void* v, cons
   const int64_t work = (int64_t)bp.n_kv_units * hkv;
   if (work > 0) {
     const int grid = (int)(work < di->sms ? work : di->sms);
-    e = head_dim == 64 ? sap::launch_bwd<64>(tq, tk, tv, tdo, bp, grid, s)
-                       : sap::launch_bwd<128>(tq, tk, tv, tdo, bp, grid, s);
+    e = head_dim == 64 ? sap::launch_bwd<64>(tq, tk, tv, tdo, tdq, bp, grid, s)
+                       : sap::launch_bwd<128>(tq, tk, tv, tdo, tdq, bp, grid, s);
     if (e != cudaSuccess) return cuda_fail(e);
   }
   e = sap::launch_dq_post(dq_acc, static_cast<__nv_bfloat16*>(dq), p->n * hq * head_dim, s);

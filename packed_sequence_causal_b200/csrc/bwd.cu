@@ -52,7 +52,7 @@ struct BwdCfg {
   static constexpr int OFF_DS = OFF_V + TILE;
   static constexpr int OFF_ST = OFF_DS + 128 * 128 * 2;  // stages: Q, dO, lse2, dvec
   static constexpr int OFF_BAR = OFF_ST + NSQ * STAGE;
-  static constexpr int NBAR = 2 + 2 * NSQ + 10;
+  static constexpr int NBAR = 2 + 2 * NSQ + 11;
   // The dynamic shared window starts 1024-byte aligned (checked at run time),
   // so no alignment slack is reserved: the D = 128 layout needs 231,568 bytes.
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16;
@@ -66,7 +66,7 @@ template <int D>
 __global__ void __launch_bounds__(448, 1)
     sap_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-                   const BwdParams p) {
+                   const __grid_constant__ CUtensorMap tmDQ, const BwdParams p) {
   using C = BwdCfg<D>;
   extern __shared__ __align__(1024) uint8_t smem[];
   if (smem_u32(smem) & 1023u) {  // TMA 128-byte swizzle and the descriptors need 1024-byte alignment
@@ -88,6 +88,7 @@ __global__ void __launch_bounds__(448, 1)
   uint64_t* dkdv_full = dq_free + 1;
   uint64_t* dkdv_free = dkdv_full + 1;
   uint64_t* mma_drain = dkdv_free + 1;
+  uint64_t* stg_ready = mma_drain + 1;  // dQ tile staged in shared memory (d = 128)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBAR);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -111,6 +112,7 @@ __global__ void __launch_bounds__(448, 1)
     mbar_init(dkdv_full, 1);
     mbar_init(dkdv_free, 128);
     mbar_init(mma_drain, 1);
+    mbar_init(stg_ready, 128);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -248,7 +250,8 @@ __global__ void __launch_bounds__(448, 1)
           }
           tc_commit(dq_full);
           tc_commit(ds_free);
-          tc_commit(q_empty + it % C::NSQ);
+          // d = 128: the dQ drain stages its tile in this stage and releases it after the reduction has read it
+          if (!C::DQ_T) tc_commit(q_empty + it % C::NSQ);
         }
         if (!ok) break;
         tc_commit(dkdv_full);
@@ -354,16 +357,32 @@ __global__ void __launch_bounds__(448, 1)
           if (!mbar_wait_warp(dq_full, it & 1, guard, kErrTimeoutEpilogue)) { ok = false; break; }
           tc_fence_after();
           if (C::DQ_T) {
-            // lane t = feature t of dQ; a warp's reductions for one q row cover 32 consecutive floats
-            float* dst = p.dq_acc + ((size_t)qt * 128 * p.hq + h) * D + t;
-            const size_t row_stride = (size_t)p.hq * D;
+            // Lane t holds feature t of dQ^T (one column per q row).  The fp32 tile is staged,
+            // row-major [q][d], over this iteration's Q/dO stage (no MMA reads it any more once
+            // dq_full has fired) and added to the accumulator by one TMA bulk reduction.
+            const int s = it % C::NSQ;
+            float* stg = reinterpret_cast<float*>(smem + C::OFF_ST + s * C::STAGE);
 #pragma unroll 1
             for (int c = 0; c < 4; ++c) {
               float v[32];
               tmem_ld32(lane_base + C::COL_DQ + 32 * c, v);
+              if (c == 3) {  // all of dQ^T is in registers: R2 may take the next dP^T
+                tc_fence_before();
+                mbar_arrive(dq_free);
+              }
 #pragma unroll
-              for (int e2 = 0; e2 < 32; ++e2) atomicAdd(dst + (size_t)(32 * c + e2) * row_stride, v[e2]);
+              for (int e2 = 0; e2 < 32; ++e2) stg[(32 * c + e2) * 128 + t] = v[e2];
             }
+            fence_async_smem();
+            mbar_arrive(stg_ready);
+            if (!mbar_wait_warp(stg_ready, it & 1, guard, kErrTimeoutEpilogue)) { ok = false; break; }
+            if (t == 0) {
+              tma_reduce_add_3d(&tmDQ, stg, 0, h, qt * 128);
+              bulk_commit_group();
+              bulk_wait_group_read0();
+              mbar_arrive(q_empty + s);
+            }
+            continue;
           } else {
             // lane t = q row t of the tile
             float* dst = p.dq_acc + (((size_t)qt * 128 + t) * p.hq + h) * D;
@@ -412,6 +431,7 @@ __global__ void __launch_bounds__(448, 1)
     }
   }
 
+  if (warp >= 10) bulk_wait_group0();  // the dQ reductions issued by this thread have completed
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -423,17 +443,17 @@ __global__ void __launch_bounds__(448, 1)
 
 template <int D>
 cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
-                       const BwdParams& p, int grid, cudaStream_t stream) {
+                       const CUtensorMap& tdq, const BwdParams& p, int grid, cudaStream_t stream) {
   auto kern = sap_bwd_kernel<D>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, BwdCfg<D>::SMEM);
   if (e != cudaSuccess) return e;
-  kern<<<grid, BwdCfg<D>::THREADS, BwdCfg<D>::SMEM, stream>>>(tq, tk, tv, tdo, p);
+  kern<<<grid, BwdCfg<D>::THREADS, BwdCfg<D>::SMEM, stream>>>(tq, tk, tv, tdo, tdq, p);
   return cudaGetLastError();
 }
 
 template cudaError_t launch_bwd<64>(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
-                                    const BwdParams&, int, cudaStream_t);
+                                    const CUtensorMap&, const BwdParams&, int, cudaStream_t);
 template cudaError_t launch_bwd<128>(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
-                                     const BwdParams&, int, cudaStream_t);
+                                     const CUtensorMap&, const BwdParams&, int, cudaStream_t);
 
 }  // namespace sap

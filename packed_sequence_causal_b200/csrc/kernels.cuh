@@ -47,7 +47,7 @@ cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
 
 template <int D>
 cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
-                       const BwdParams& p, int grid, cudaStream_t stream);
+                       const CUtensorMap& tdq, const BwdParams& p, int grid, cudaStream_t stream);
 
 template <int D>
 cudaError_t launch_merge(const int32_t* merges, int64_t n_merges, int32_t hq, int64_t n, const float* o_part,
