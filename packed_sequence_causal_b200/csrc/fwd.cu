@@ -340,6 +340,324 @@ __global__ void __launch_bounds__(192, 1)
   }
 }
 
+// Two-tile variant for an even GQA group: one CTA computes the same q tile for
+// two query heads of one kv group, so both tiles walk the same kv tiles and
+// share every K/V load.  P is written back into TMEM (packed bf16 over the S
+// columns) and read from there by the PV MMA, and the MMA thread interleaves
+// the tiles -- S0, S1, PV0, S0', PV1, S1', ... -- so that while one softmax
+// warpgroup exponentiates its tile the tensor core works on the other.
+//
+// Threads: warp 0 TMA, warp 1 MMA, warps 2..5 softmax of tile 0 (head 2p),
+// warps 6..9 softmax of tile 1 (head 2p+1).
+// TMEM columns: S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [256+D,256+2D).
+template <int D>
+struct Fwd2Cfg {
+  static constexpr int NS = (D == 64) ? 3 : 2;
+  static constexpr int BOX = 128 * 128;
+  static constexpr int QBYTES = D * 128 * 2;
+  static constexpr int KVBYTES = D * 128 * 2;
+  static constexpr int OFF_Q0 = 0;
+  static constexpr int OFF_Q1 = QBYTES;
+  static constexpr int OFF_K = 2 * QBYTES;
+  static constexpr int OFF_V = OFF_K + NS * KVBYTES;
+  static constexpr int OFF_BAR = OFF_V + NS * KVBYTES;
+  static constexpr int NBAR = 2 + 4 * NS + 2 + 2 + 2;
+  static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16;
+  static constexpr int THREADS = 320;
+  static constexpr uint32_t COL_O = 256;
+};
+
+template <int D>
+__global__ void __launch_bounds__(320, 1)
+    sap_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                        const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+  using C = Fwd2Cfg<D>;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  if (smem_u32(smem) & 1023u) {
+    if (threadIdx.x == 0) atomicOr(p.err, kErrSmemAlign);
+    return;
+  }
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* q_full = bars + 0;
+  uint64_t* q_empty = bars + 1;
+  uint64_t* k_full = bars + 2;
+  uint64_t* k_empty = k_full + C::NS;
+  uint64_t* v_full = k_empty + C::NS;
+  uint64_t* v_empty = v_full + C::NS;
+  uint64_t* s_full = v_empty + C::NS;  // [2], one per tile
+  uint64_t* p_full = s_full + 2;       // [2]
+  uint64_t* o_done = p_full + 2;
+  uint64_t* mma_drain = o_done + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBAR);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const Guard guard{abort_flag, p.err};
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    for (int s = 0; s < C::NS; ++s) {
+      mbar_init(k_full + s, 1);
+      mbar_init(k_empty + s, 1);
+      mbar_init(v_full + s, 1);
+      mbar_init(v_empty + s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(s_full + b, 1);
+      mbar_init(p_full + b, 128);
+    }
+    mbar_init(o_done, 1);
+    mbar_init(mma_drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  const int pairs = p.hq / 2;
+  const int total = p.n_units * pairs;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ producer
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      uint32_t kv_iter = 0, unit_iter = 0;
+      bool ok = true;
+      for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
+        const int u = p.order[w / pairs], h0 = 2 * (w % pairs), g = h0 / p.group;
+        const int qt = p.units[4 * u], ib = p.units[4 * u + 1], ic = p.units[4 * u + 2];
+        if (!mbar_wait(q_empty, (unit_iter & 1) ^ 1, guard, kErrTimeoutLoad)) break;
+        mbar_arrive_expect_tx(q_full, 2 * C::QBYTES);
+        for (int b = 0; b < D / 64; ++b) {
+          tma_load_3d(smem + C::OFF_Q0 + b * C::BOX, &tmQ, q_full, 64 * b, h0, qt * 128);
+          tma_load_3d(smem + C::OFF_Q1 + b * C::BOX, &tmQ, q_full, 64 * b, h0 + 1, qt * 128);
+        }
+        int kt_next = p.items[5 * ib + 1];
+        for (int t = 0; t < ic; ++t) {
+          const int kt = kt_next;
+          if (t + 1 < ic) kt_next = p.items[5 * (ib + t + 1) + 1];
+          const int s = kv_iter % C::NS;
+          const uint32_t ph = (kv_iter / C::NS) & 1;
+          if (!mbar_wait(k_empty + s, ph ^ 1, guard, kErrTimeoutLoad)) { ok = false; break; }
+          mbar_arrive_expect_tx(k_full + s, C::KVBYTES);
+          for (int b = 0; b < D / 64; ++b)
+            tma_load_3d(smem + C::OFF_K + s * C::KVBYTES + b * C::BOX, &tmK, k_full + s, 64 * b, g, kt * 128);
+          if (!mbar_wait(v_empty + s, ph ^ 1, guard, kErrTimeoutLoad)) { ok = false; break; }
+          mbar_arrive_expect_tx(v_full + s, C::KVBYTES);
+          for (int b = 0; b < D / 64; ++b)
+            tma_load_3d(smem + C::OFF_V + s * C::KVBYTES + b * C::BOX, &tmV, v_full + s, 64 * b, g, kt * 128);
+          ++kv_iter;
+        }
+        ++unit_iter;
+      }
+      if (unit_iter > 0) drain_wait(q_full, (unit_iter - 1) & 1);
+      for (uint32_t t = (kv_iter > (uint32_t)C::NS ? kv_iter - C::NS : 0); t < kv_iter; ++t) {
+        drain_wait(k_full + t % C::NS, (t / C::NS) & 1);
+        drain_wait(v_full + t % C::NS, (t / C::NS) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ----------------------------------------------------------------- MMA
+      constexpr uint32_t idesc_qk = idesc_bf16(128, 128, false, false);
+      constexpr uint32_t idesc_pv = idesc_bf16(128, D, false, true);
+      const uint32_t sQ0 = smem_u32(smem + C::OFF_Q0), sQ1 = smem_u32(smem + C::OFF_Q1);
+      const uint32_t sK = smem_u32(smem + C::OFF_K), sV = smem_u32(smem + C::OFF_V);
+      uint32_t kv_iter = 0, unit_iter = 0, tile_iter = 0;  // tile_iter counts kv tiles (per tile barrier phases)
+      bool ok = true;
+      auto issue_s = [&](int tile, uint32_t it) {  // S_tile = Q_tile K_it^T
+        const uint32_t sQ = tile ? sQ1 : sQ0;
+        const int s = it % C::NS;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t ko = (kk / 4) * C::BOX + (kk % 4) * 32;
+          mma_bf16(tmem + 128 * tile, sdesc_sw128(sQ + ko, 16, 1024),
+                   sdesc_sw128(sK + s * C::KVBYTES + ko, 16, 1024), idesc_qk, kk > 0);
+        }
+        tc_commit(s_full + tile);
+      };
+      auto issue_pv = [&](int tile, uint32_t it, bool first) {  // O_tile += P_tile V_it, P from TMEM
+        const int s = it % C::NS;
+#pragma unroll
+        for (int kk = 0; kk < 128 / 16; ++kk)
+          mma_bf16_tmem_a(tmem + C::COL_O + D * tile, tmem + 128 * tile + kk * 8,
+                          sdesc_sw128(sV + s * C::KVBYTES + kk * 2048, C::BOX, 1024), idesc_pv,
+                          (first && kk == 0) ? 0u : 1u);
+      };
+      for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
+        const int u = p.order[w / pairs];
+        const int ic = p.units[4 * u + 2];
+        if (!mbar_wait(q_full, unit_iter & 1, guard, kErrTimeoutMma)) break;
+        if (!mbar_wait(k_full + kv_iter % C::NS, (kv_iter / C::NS) & 1, guard, kErrTimeoutMma)) break;
+        tc_fence_after();
+        issue_s(0, kv_iter);
+        issue_s(1, kv_iter);
+        tc_commit(k_empty + kv_iter % C::NS);
+        for (int j = 0; j < ic; ++j, ++tile_iter) {
+          const uint32_t it = kv_iter + j;
+          if (!mbar_wait(v_full + it % C::NS, (it / C::NS) & 1, guard, kErrTimeoutMma)) { ok = false; break; }
+          if (!mbar_wait(p_full + 0, tile_iter & 1, guard, kErrTimeoutMma)) { ok = false; break; }
+          tc_fence_after();
+          issue_pv(0, it, j == 0);
+          const bool more = j + 1 < ic;
+          if (more) {
+            if (!mbar_wait(k_full + (it + 1) % C::NS, ((it + 1) / C::NS) & 1, guard, kErrTimeoutMma)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_s(0, it + 1);  // rewrites S0/P0 only after PV0 (issued above) has read P0
+          }
+          if (!mbar_wait(p_full + 1, tile_iter & 1, guard, kErrTimeoutMma)) { ok = false; break; }
+          tc_fence_after();
+          issue_pv(1, it, j == 0);
+          tc_commit(v_empty + it % C::NS);
+          if (more) {
+            issue_s(1, it + 1);
+            tc_commit(k_empty + (it + 1) % C::NS);
+          }
+        }
+        if (!ok) break;
+        tc_commit(o_done);
+        tc_commit(q_empty);
+        kv_iter += ic;
+        ++unit_iter;
+      }
+      tc_commit(mma_drain);
+      drain_wait(mma_drain, 0);
+    }
+  } else {
+    // ------------------------------------------------------------- softmax
+    const int tile = (warp - 2) >> 2;
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;
+    const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
+    const uint32_t colS = 128 * tile, colO = C::COL_O + D * tile;
+    uint32_t tile_iter = 0, unit_iter = 0;
+    const float sl2 = p.scale_log2;
+    bool ok = true;
+    for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
+      const int u = p.order[w / pairs], h = 2 * (w % pairs) + tile;
+      const int qt = p.units[4 * u], ib = p.units[4 * u + 1], ic = p.units[4 * u + 2], slot = p.units[4 * u + 3];
+      const int64_t i = (int64_t)qt * 128 + r;
+      const bool real_row = i < p.n;
+      const int row_lo = real_row ? p.tok_lo[i] : 1;
+      const int row_hi = real_row ? (int)i : 0;
+      float m = -INFINITY, l = 0.f;
+      for (int j = 0; j < ic; ++j, ++tile_iter) {
+        const int kt = p.items[5 * (ib + j) + 1], tag = p.items[5 * (ib + j) + 4];
+        if (!mbar_wait_warp(s_full + tile, tile_iter & 1, guard, kErrTimeoutSoftmax)) { ok = false; break; }
+        tc_fence_after();
+        float sv[128];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(lane_base + colS + 32 * c, sv + 32 * c);
+        if (tag != 0) {
+          const int c_lo = row_lo - kt * 128, c_hi = row_hi - kt * 128;
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            if (c < c_lo || c > c_hi) sv[c] = -INFINITY;
+        }
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 128; ++c) mx = fmaxf(mx, sv[c]);
+        const float m_tile = mx * sl2;
+        // s_full of this tile also means the previous PV into O has completed.
+        const bool grow = m_tile > m + 8.0f;
+        const float alpha = grow ? ex2(m - m_tile) : 1.f;
+        if (j > 0 && __any_sync(0xffffffffu, grow && l > 0.f)) {
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            float ov[32];
+            tmem_ld32(lane_base + colO + 32 * c, ov);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) ov[e] *= alpha;
+            tmem_st32(lane_base + colO + 32 * c, ov);
+          }
+        }
+        if (grow) {
+          l *= alpha;
+          m = m_tile;
+        }
+        const float base = (m == -INFINITY) ? 0.f : m;
+        float rs = 0.f;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const float p0 = ex2(fmaf(sv[64 * half + 2 * e], sl2, -base));
+            const float p1 = ex2(fmaf(sv[64 * half + 2 * e + 1], sl2, -base));
+            rs += p0 + p1;
+            pk[e] = pack_bf16x2(p0, p1);
+          }
+          tmem_st32_u(lane_base + colS + 32 * half, pk);  // P over the S columns already read
+        }
+        l += rs;
+        tc_fence_before();
+        mbar_arrive(p_full + tile);
+      }
+      if (!ok) break;
+      // ------------------------------------------------------------ epilogue
+      if (!mbar_wait_warp(o_done, unit_iter & 1, guard, kErrTimeoutEpilogue)) break;
+      ++unit_iter;
+      tc_fence_after();
+      const float inv_l = l > 0.f ? 1.f / l : 0.f;
+      const float lse_val = l > 0.f ? (m + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
+      if (slot < 0) {
+        __nv_bfloat16* orow = p.o + ((size_t)i * p.hq + h) * D;
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          float ov[32];
+          tmem_ld32(lane_base + colO + 32 * c, ov);
+          if (real_row) {
+#pragma unroll
+            for (int e = 0; e < 32; e += 8) {
+              uint4 pk;
+              pk.x = pack_bf16x2(ov[e] * inv_l, ov[e + 1] * inv_l);
+              pk.y = pack_bf16x2(ov[e + 2] * inv_l, ov[e + 3] * inv_l);
+              pk.z = pack_bf16x2(ov[e + 4] * inv_l, ov[e + 5] * inv_l);
+              pk.w = pack_bf16x2(ov[e + 6] * inv_l, ov[e + 7] * inv_l);
+              *reinterpret_cast<uint4*>(orow + 32 * c + e) = pk;
+            }
+          }
+        }
+        if (real_row) p.lse[(size_t)h * p.n + i] = lse_val;
+      } else {
+        float* orow = p.o_part + (((size_t)slot * p.hq + h) * 128 + r) * D;
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          float ov[32];
+          tmem_ld32(lane_base + colO + 32 * c, ov);
+#pragma unroll
+          for (int e = 0; e < 32; e += 4)
+            *reinterpret_cast<float4*>(orow + 32 * c + e) =
+                make_float4(ov[e] * inv_l, ov[e + 1] * inv_l, ov[e + 2] * inv_l, ov[e + 3] * inv_l);
+        }
+        p.lse_part[((size_t)slot * p.hq + h) * 128 + r] = lse_val;
+      }
+      // The next unit's first PV into O waits for this warpgroup's next p_full.
+      tc_fence_before();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
 template <int D>
 int fwd_smem_bytes() {
   return FwdCfg<D>::SMEM;
@@ -348,6 +666,15 @@ int fwd_smem_bytes() {
 template <int D>
 cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
                        int grid, cudaStream_t stream) {
+  if (p.group % 2 == 0) {  // two heads of one kv group per CTA
+    const int64_t work = (int64_t)p.n_units * (p.hq / 2);
+    const int g2 = (int)(work < grid ? work : grid);
+    auto kern2 = sap_fwd_pair_kernel<D>;
+    cudaError_t e = cudaFuncSetAttribute(kern2, cudaFuncAttributeMaxDynamicSharedMemorySize, Fwd2Cfg<D>::SMEM);
+    if (e != cudaSuccess) return e;
+    if (g2 > 0) kern2<<<g2, Fwd2Cfg<D>::THREADS, Fwd2Cfg<D>::SMEM, stream>>>(tq, tk, tv, p);
+    return cudaGetLastError();
+  }
   auto kern = sap_fwd_kernel<D>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, FwdCfg<D>::SMEM);
   if (e != cudaSuccess) return e;
