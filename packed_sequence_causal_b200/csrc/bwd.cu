@@ -21,7 +21,8 @@
 //                owns kv row j = kt*128 + t.  P^T = exp2(S^T c - LSE2_i) on the
 //                pairs of its document with i >= j (all pairs for FULL tiles),
 //                written back to TMEM as packed bf16 over its own S columns;
-//                dS^T = P^T (dP^T - D_i) * scale written to a 128-byte swizzled
+//                dS^T = P^T (dP^T - D_i) (the softmax scale is applied to dK and dQ
+//                as they are drained) written to a 128-byte swizzled
 //                shared tile as bf16 (read as a K-major operand by dK and as an
 //                MN-major operand by dQ).
 //   warps 10..13 drain dQ from TMEM into the fp32 accumulator (global
@@ -269,7 +270,7 @@ __global__ void __launch_bounds__(448, 1)
     const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
     const uint32_t R1 = lane_base + C::COL_R1 + 64 * half, R2 = lane_base + C::COL_R2 + 64 * half;
     uint8_t* sDSt = smem + C::OFF_DS + half * C::BOX;
-    const float sl2 = p.scale_log2, scale = p.scale;
+    const float sl2 = p.scale_log2;
     uint32_t it = 0;
     bool ok = true;
     for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
@@ -293,15 +294,27 @@ __global__ void __launch_bounds__(448, 1)
           tc_fence_after();
           float pr[64];
           {
+            const float4* l4 = reinterpret_cast<const float4*>(lse2);
             float sv[32];
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
               tmem_ld32(R1 + 32 * c, sv);
+              if (tag == 0) {  // FULL tile: no pair is masked
 #pragma unroll
-              for (int e2 = 0; e2 < 32; ++e2) {
-                const int col = 32 * c + e2;
-                const bool valid = (tag == 0) || (col >= c_lo && col <= c_hi);
-                pr[col] = valid ? ex2(fmaf(sv[e2], sl2, -lse2[col])) : 0.f;
+                for (int e4 = 0; e4 < 32; e4 += 4) {
+                  const float4 l = l4[(32 * c + e4) / 4];
+                  pr[32 * c + e4] = ex2(fmaf(sv[e4], sl2, -l.x));
+                  pr[32 * c + e4 + 1] = ex2(fmaf(sv[e4 + 1], sl2, -l.y));
+                  pr[32 * c + e4 + 2] = ex2(fmaf(sv[e4 + 2], sl2, -l.z));
+                  pr[32 * c + e4 + 3] = ex2(fmaf(sv[e4 + 3], sl2, -l.w));
+                }
+              } else {
+#pragma unroll
+                for (int e2 = 0; e2 < 32; ++e2) {
+                  const int col = 32 * c + e2;
+                  const bool valid = col >= c_lo && col <= c_hi;
+                  pr[col] = valid ? ex2(fmaf(sv[e2], sl2, -lse2[col])) : 0.f;
+                }
               }
             }
             uint32_t pk[32];
@@ -314,17 +327,19 @@ __global__ void __launch_bounds__(448, 1)
           if (!mbar_wait_warp(dp_full, it & 1, guard, kErrTimeoutSoftmax)) { ok = false; break; }
           if (it > 0 && !mbar_wait_warp(ds_free, (it - 1) & 1, guard, kErrTimeoutSoftmax)) { ok = false; break; }
           tc_fence_after();
+          const float4* d4 = reinterpret_cast<const float4*>(dvec);
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
             float dpv[32];
             tmem_ld32(R2 + 32 * c, dpv);
             uint32_t dw[16];
+            // dS^T without the softmax scale; the scale is applied to dK and dQ when they are drained
 #pragma unroll
-            for (int e2 = 0; e2 < 32; e2 += 2) {
-              const int col = 32 * c + e2;
-              const float d0 = pr[col] * (dpv[e2] - dvec[col]) * scale;
-              const float d1 = pr[col + 1] * (dpv[e2 + 1] - dvec[col + 1]) * scale;
-              dw[e2 / 2] = pack_bf16x2(d0, d1);
+            for (int e4 = 0; e4 < 32; e4 += 4) {
+              const int col = 32 * c + e4;
+              const float4 dd = d4[col / 4];
+              dw[e4 / 2] = pack_bf16x2(pr[col] * (dpv[e4] - dd.x), pr[col + 1] * (dpv[e4 + 1] - dd.y));
+              dw[e4 / 2 + 1] = pack_bf16x2(pr[col + 2] * (dpv[e4 + 2] - dd.z), pr[col + 3] * (dpv[e4 + 3] - dd.w));
             }
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4) {  // 16-byte chunks 4c .. 4c+3 of this half's 64 columns
@@ -371,7 +386,7 @@ __global__ void __launch_bounds__(448, 1)
                 mbar_arrive(dq_free);
               }
 #pragma unroll
-              for (int e2 = 0; e2 < 32; ++e2) stg[(32 * c + e2) * 128 + t] = v[e2];
+              for (int e2 = 0; e2 < 32; ++e2) stg[(32 * c + e2) * 128 + t] = v[e2] * p.scale;
             }
             fence_async_smem();
             mbar_arrive(stg_ready);
@@ -393,7 +408,8 @@ __global__ void __launch_bounds__(448, 1)
 #pragma unroll
               for (int e4 = 0; e4 < 32; e4 += 4)
                 atomicAdd(reinterpret_cast<float4*>(dst + 32 * c + e4),
-                          make_float4(v[e4], v[e4 + 1], v[e4 + 2], v[e4 + 3]));
+                          make_float4(v[e4] * p.scale, v[e4 + 1] * p.scale, v[e4 + 2] * p.scale,
+                                      v[e4 + 3] * p.scale));
             }
           }
           tc_fence_before();
@@ -408,6 +424,7 @@ __global__ void __launch_bounds__(448, 1)
       for (int which = 0; which < 2; ++which) {
         __nv_bfloat16* out = (which == 0 ? p.dk : p.dv) + ((size_t)jrow * p.hkv + g) * D;
         const uint32_t col = which == 0 ? C::COL_DK : C::COL_DV;
+        const float f = which == 0 ? p.scale : 1.f;  // dK carries the softmax scale left out of dS
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
           float v[32];
@@ -416,10 +433,10 @@ __global__ void __launch_bounds__(448, 1)
 #pragma unroll
             for (int e8 = 0; e8 < 32; e8 += 8) {
               uint4 pk;
-              pk.x = pack_bf16x2(v[e8], v[e8 + 1]);
-              pk.y = pack_bf16x2(v[e8 + 2], v[e8 + 3]);
-              pk.z = pack_bf16x2(v[e8 + 4], v[e8 + 5]);
-              pk.w = pack_bf16x2(v[e8 + 6], v[e8 + 7]);
+              pk.x = pack_bf16x2(v[e8] * f, v[e8 + 1] * f);
+              pk.y = pack_bf16x2(v[e8 + 2] * f, v[e8 + 3] * f);
+              pk.z = pack_bf16x2(v[e8 + 4] * f, v[e8 + 5] * f);
+              pk.w = pack_bf16x2(v[e8 + 6] * f, v[e8 + 7] * f);
               *reinterpret_cast<uint4*>(out + 32 * c + e8) = pk;
             }
           }
