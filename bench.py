@@ -108,6 +108,29 @@ class ClockSampler:
                 "samples": len(sm), "power_w_max": max(power)}
 
 
+# ------------------------------------------------------------------ ranks
+
+
+def rank_seed(base_seed: int, rank: int) -> int:
+    """Each rank runs its own independent packed batch (data-parallel replicas)."""
+    return base_seed + rank
+
+
+def max_over_ranks(value: float, dist=None, device=None) -> float:
+    """The job's time is the slowest rank's device time (no collective on the data path)."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(flops_per_step: float, steps: int, world: int, elapsed_ms: float) -> float:
+    """Whole-job TFLOP/s: the units all ranks processed over the slowest rank's time."""
+    return world * flops_per_step * steps / (elapsed_ms / 1e3) / 1e12
+
+
 # --------------------------------------------------------------------- cpu oracle
 
 
@@ -196,7 +219,7 @@ def main():
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
-    b = workloads.make_batch(w, args.seed + rank, device=str(dev), with_do=True)
+    b = workloads.make_batch(w, rank_seed(args.seed, rank), device=str(dev), with_do=True)
     n, hq, hkv, d = w.n, w.hq, w.hkv, w.d
     scale = 1.0 / math.sqrt(d)
     t_plan = time.perf_counter()
@@ -257,11 +280,7 @@ def main():
     if world > 1:
         dist.barrier()
     clocks = sampler.stop()
-    elapsed_ms = start.elapsed_time(end)
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(start.elapsed_time(end), dist if world > 1 else None, dev)
     status = sap.sap_device_status()
     if status != 0:
         raise RuntimeError(f"device error word {status} after the timed steps")
@@ -269,7 +288,7 @@ def main():
     f_fwd, f_bwd = _flops(w, pairs)
     f_step = f_fwd + f_bwd
     ms_step = elapsed_ms / args.steps
-    value = world * f_step * args.steps / (elapsed_ms / 1e3) / 1e12
+    value = job_throughput(f_step, args.steps, world, elapsed_ms)
     tokens_s = world * n * args.steps / (elapsed_ms / 1e3)
     burst, sustained, hbm, peak_src = _peaks()
     # per-call device times from the events recorded on the launching stream
@@ -302,12 +321,8 @@ def main():
             e2e_step()
         e2.record(stream)
         torch.cuda.synchronize()
-        e2e_ms = s2.elapsed_time(e2)
-        if world > 1:
-            t = torch.tensor([e2e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
-        e2e = {"value": round(world * f_step * args.steps / (e2e_ms / 1e3) / 1e12, 2), "unit": "TFLOP/s",
+        e2e_ms = max_over_ranks(s2.elapsed_time(e2), dist if world > 1 else None, dev)
+        e2e = {"value": round(job_throughput(f_step, args.steps, world, e2e_ms), 2), "unit": "TFLOP/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": round(e2e_ms / args.steps, 3),
                "tokens_per_s": round(world * n * args.steps / (e2e_ms / 1e3), 1)}
