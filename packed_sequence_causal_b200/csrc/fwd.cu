@@ -236,9 +236,15 @@ __global__ void __launch_bounds__(192, 1)
           for (int c = 0; c < 128; ++c)
             if (c < c_lo || c > c_hi) sv[c] = -INFINITY;
         }
-        float mx = -INFINITY;
+        // row max as 8 independent chains (a single 128-long chain is latency-bound)
+        float mx8[8];
 #pragma unroll
-        for (int c = 0; c < 128; ++c) mx = fmaxf(mx, sv[c]);
+        for (int e = 0; e < 8; ++e) mx8[e] = sv[e];
+#pragma unroll
+        for (int c = 8; c < 128; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], sv[c]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) mx8[e] = fmaxf(mx8[e], mx8[e + 4]);
+        const float mx = fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3]));
         const float m_tile = mx * sl2;
         // P_{j-1} V_{j-1} must be complete before O is rescaled or P is overwritten.
         if (j > 0) {
@@ -266,7 +272,7 @@ __global__ void __launch_bounds__(192, 1)
           m = m_tile;
         }
         const float base = (m == -INFINITY) ? 0.f : m;
-        float rs = 0.f;
+        float rs4[4] = {0.f, 0.f, 0.f, 0.f};  // row sum as 4 independent chains
 #pragma unroll
         for (int cc = 0; cc < 16; ++cc) {
           uint32_t w4[4];
@@ -274,13 +280,13 @@ __global__ void __launch_bounds__(192, 1)
           for (int e = 0; e < 4; ++e) {
             const float p0 = ex2(fmaf(sv[cc * 8 + 2 * e], sl2, -base));
             const float p1 = ex2(fmaf(sv[cc * 8 + 2 * e + 1], sl2, -base));
-            rs += p0 + p1;
+            rs4[e] += p0 + p1;
             w4[e] = pack_bf16x2(p0, p1);
           }
           const uint32_t addr = smem_u32(sP + (cc / 8) * C::BOX + sw128_offset(r, cc % 8));
           st_shared_v4(addr, w4[0], w4[1], w4[2], w4[3]);
         }
-        l += rs;
+        l += (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
         fence_async_smem();
         tc_fence_before();
         mbar_arrive(p_full);
@@ -566,9 +572,15 @@ __global__ void __launch_bounds__(320, 1)
           for (int c = 0; c < 128; ++c)
             if (c < c_lo || c > c_hi) sv[c] = -INFINITY;
         }
-        float mx = -INFINITY;
+        // row max as 8 independent chains (a single 128-long chain is latency-bound)
+        float mx8[8];
 #pragma unroll
-        for (int c = 0; c < 128; ++c) mx = fmaxf(mx, sv[c]);
+        for (int e = 0; e < 8; ++e) mx8[e] = sv[e];
+#pragma unroll
+        for (int c = 8; c < 128; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], sv[c]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) mx8[e] = fmaxf(mx8[e], mx8[e + 4]);
+        const float mx = fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3]));
         const float m_tile = mx * sl2;
         // s_full of this tile also means the previous PV into O has completed.
         const bool grow = m_tile > m + 8.0f;
@@ -588,7 +600,7 @@ __global__ void __launch_bounds__(320, 1)
           m = m_tile;
         }
         const float base = (m == -INFINITY) ? 0.f : m;
-        float rs = 0.f;
+        float rs4[4] = {0.f, 0.f, 0.f, 0.f};  // row sum as 4 independent chains
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           uint32_t pk[32];
@@ -596,12 +608,12 @@ __global__ void __launch_bounds__(320, 1)
           for (int e = 0; e < 32; ++e) {
             const float p0 = ex2(fmaf(sv[64 * half + 2 * e], sl2, -base));
             const float p1 = ex2(fmaf(sv[64 * half + 2 * e + 1], sl2, -base));
-            rs += p0 + p1;
+            rs4[e & 3] += p0 + p1;
             pk[e] = pack_bf16x2(p0, p1);
           }
           tmem_st32_u(lane_base + colS + 32 * half, pk);  // P over the S columns already read
         }
-        l += rs;
+        l += (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
         tc_fence_before();
         mbar_arrive(p_full + tile);
       }
