@@ -194,6 +194,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=1e11, help="unmasked FLOPs of the CPU-baseline sample")
+    ap.add_argument("--fused-merge", action="store_true",
+                    help="one forward pass over all kv chunks of a q tile (no partials, no merge kernel)")
     ap.add_argument("--tokens", type=int, default=None,
                     help="run the workload's recipe at a smaller token count (profiling captures only)")
     args = ap.parse_args()
@@ -224,6 +226,8 @@ def main():
     scale = 1.0 / math.sqrt(d)
     t_plan = time.perf_counter()
     plan = sap.sap_plan(b.cu_seqlens, n, w.p)
+    if args.fused_merge:
+        sap.sap_plan_set_fused_merge(plan, True)
     t_plan = time.perf_counter() - t_plan
     sap.sap_plan_upload(plan)
     stats = sap.sap_plan_stats(plan)
@@ -352,6 +356,7 @@ def main():
             "config": {"workload": w.name, "tokens": n, "docs": int(len(b.cu_seqlens) - 1), "hq": hq, "hkv": hkv,
                        "head_dim": d, "chunks": w.p, "tiles": n_items, "unmasked_pairs_per_head": pairs,
                        "flops_per_step": f_step, "parallelism": f"dp{world}" if world > 1 else "single",
+                       "fused_merge": bool(args.fused_merge),
                        "l2": "inputs larger than L2 (Q, dO, O 1 GiB each); no flush"},
             "tokens_per_s": round(tokens_s, 1),
             "pct_bf16_peak": round(100 * value / world / burst, 2),

@@ -109,6 +109,17 @@ int sap_plan_fwd_schedule(sap_plan_t plan, const int32_t** units, int64_t* n_uni
  *   entries:  int32[n_items][2] = (q_tile, tag), grouped by kv tile, q-tile descending. */
 int sap_plan_bwd_schedule(sap_plan_t plan, const int32_t** kv_units, int64_t* n_kv_units, const int32_t** entries);
 
+/* Fused-merge mode (enable != 0): the forward schedule gets one unit per
+ * q-tile spanning all of its kv chunks, so sap_attn_fwd carries the online
+ * softmax across chunk boundaries and writes O and LSE directly -- no fp32
+ * partials, no forward workspace, and sap_merge has nothing to do.  The result
+ * is the merged result of the chunked path (the merge is exact), computed in
+ * one pass; the per-(q-chunk, kv-chunk) partials are not produced.  enable = 0
+ * restores the chunked schedule.  Host-side only: the device copy of the plan
+ * is released (the device is synchronised) and uploaded again by the next
+ * device call. */
+int sap_plan_set_fused_merge(sap_plan_t plan, int enable);
+
 /* Copy the plan's device arrays to the current device on `stream`.  Called
  * implicitly by the first device call that needs them; calling it first keeps
  * the one host-to-device transfer out of later timed calls. */

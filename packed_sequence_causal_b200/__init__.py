@@ -28,6 +28,7 @@ from ._capi import (  # noqa: F401
     sap_plan_destroy,
     sap_plan_fwd_schedule,
     sap_plan_items,
+    sap_plan_set_fused_merge,
     sap_plan_stats,
     sap_plan_upload,
     sap_workspace_size,

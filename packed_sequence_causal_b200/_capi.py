@@ -51,6 +51,8 @@ def load_library():
     L.sap_plan_fwd_schedule.argtypes = [P, PP, ctypes.POINTER(i64), PP, PP, ctypes.POINTER(i64)]
     L.sap_plan_bwd_schedule.restype = ctypes.c_int
     L.sap_plan_bwd_schedule.argtypes = [P, PP, ctypes.POINTER(i64), PP]
+    L.sap_plan_set_fused_merge.restype = ctypes.c_int
+    L.sap_plan_set_fused_merge.argtypes = [P, ctypes.c_int]
     L.sap_plan_upload.restype = ctypes.c_int
     L.sap_plan_upload.argtypes = [P, P]
     L.sap_plan_destroy.restype = None
@@ -156,6 +158,10 @@ def _stream_ptr(stream) -> Optional[int]:
     if stream is None:
         stream = torch.cuda.current_stream()
     return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def sap_plan_set_fused_merge(plan: Plan, enable: bool = True):
+    _check(load_library().sap_plan_set_fused_merge(plan.handle, int(bool(enable))), "sap_plan_set_fused_merge")
 
 
 def sap_plan_upload(plan: Plan, stream=None):

@@ -271,6 +271,23 @@ int sap_plan_upload(sap_plan_t p, void* stream) {
   return SAP_OK;
 }
 
+int sap_plan_set_fused_merge(sap_plan_t plan, int enable) {
+  if (!plan) return SAP_ERR_INVALID_ARG;
+  if (plan->fused_merge == (enable != 0)) return SAP_OK;
+  try {
+    sap_plan_build_fwd_schedule(plan, enable != 0);
+  } catch (const std::bad_alloc&) {
+    return SAP_ERR_NOMEM;
+  }
+  if (plan->dev) {  // the device copy no longer matches: drop it, the next device call uploads again
+    cudaError_t e = cudaFree(plan->dev);
+    plan->dev = nullptr;
+    plan->dev_id = -1;
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  return SAP_OK;
+}
+
 void sap_plan_destroy(sap_plan_t plan) {
   if (!plan) return;
   if (plan->dev) cudaFree(plan->dev);

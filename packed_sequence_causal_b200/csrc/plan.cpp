@@ -19,6 +19,48 @@
 
 #include "plan.hpp"
 
+// Forward schedule.  Default: one unit per (q-tile, kv-chunk) run of items, a
+// partial slot for each unit of a q-tile that sees several kv chunks, and a
+// merge entry per such q-tile.  Fused: one unit per q-tile over all its items
+// (every kv chunk), written directly, so there are no partials and no merges.
+void sap_plan_build_fwd_schedule(sap_plan_s* p, bool fused) {
+  p->fused_merge = fused;
+  p->fwd_units.clear();
+  p->merges.clear();
+  p->n_slots = 0;
+  {
+    size_t a = 0;
+    const size_t ni = p->items.size();
+    while (a < ni) {
+      size_t e = a;
+      while (e < ni && p->items[e].q_tile == p->items[a].q_tile) ++e;  // items of this q-tile: [a, e)
+      std::vector<std::pair<size_t, size_t>> runs;
+      size_t r = a;
+      while (r < e) {
+        size_t s = r;
+        while (s < e && (fused || p->items[s].kv_chunk == p->items[r].kv_chunk)) ++s;
+        runs.push_back({r, s - r});
+        r = s;
+      }
+      const bool partial = runs.size() > 1;
+      if (partial)
+        p->merges.insert(p->merges.end(),
+                         {p->items[a].q_tile, (int32_t)p->n_slots, (int32_t)runs.size()});
+      for (auto& run : runs) {
+        int32_t slot = partial ? (int32_t)(p->n_slots++) : -1;
+        p->fwd_units.insert(p->fwd_units.end(),
+                            {p->items[a].q_tile, (int32_t)run.first, (int32_t)run.second, slot});
+      }
+      a = e;
+    }
+  }
+  const size_t nu = p->fwd_units.size() / 4;
+  p->fwd_order.resize(nu);
+  std::iota(p->fwd_order.begin(), p->fwd_order.end(), 0);
+  std::stable_sort(p->fwd_order.begin(), p->fwd_order.end(),
+                   [&](int32_t x, int32_t y) { return p->fwd_units[4 * x + 2] > p->fwd_units[4 * y + 2]; });
+}
+
 int sap_plan_build(const int32_t* cu, int32_t num_docs, int64_t n, int32_t num_chunks, int32_t block_m,
                    int32_t block_n, sap_plan_s* p) {
   if (!cu || !p || num_docs < 0 || n < 0 || block_m <= 0 || block_n <= 0) return SAP_ERR_INVALID_ARG;
@@ -91,41 +133,7 @@ int sap_plan_build(const int32_t* cu, int32_t num_docs, int64_t n, int32_t num_c
     }
   }
 
-  // forward units: contiguous runs of one q-tile and one kv-chunk
-  p->fwd_units.clear();
-  p->merges.clear();
-  p->n_slots = 0;
-  {
-    size_t a = 0;
-    const size_t ni = p->items.size();
-    while (a < ni) {
-      size_t e = a;
-      while (e < ni && p->items[e].q_tile == p->items[a].q_tile) ++e;  // items of this q-tile: [a, e)
-      std::vector<std::pair<size_t, size_t>> runs;
-      size_t r = a;
-      while (r < e) {
-        size_t s = r;
-        while (s < e && p->items[s].kv_chunk == p->items[r].kv_chunk) ++s;
-        runs.push_back({r, s - r});
-        r = s;
-      }
-      const bool partial = runs.size() > 1;
-      if (partial)
-        p->merges.insert(p->merges.end(),
-                         {p->items[a].q_tile, (int32_t)p->n_slots, (int32_t)runs.size()});
-      for (auto& run : runs) {
-        int32_t slot = partial ? (int32_t)(p->n_slots++) : -1;
-        p->fwd_units.insert(p->fwd_units.end(),
-                            {p->items[a].q_tile, (int32_t)run.first, (int32_t)run.second, slot});
-      }
-      a = e;
-    }
-  }
-  const size_t nu = p->fwd_units.size() / 4;
-  p->fwd_order.resize(nu);
-  std::iota(p->fwd_order.begin(), p->fwd_order.end(), 0);
-  std::stable_sort(p->fwd_order.begin(), p->fwd_order.end(),
-                   [&](int32_t x, int32_t y) { return p->fwd_units[4 * x + 2] > p->fwd_units[4 * y + 2]; });
+  sap_plan_build_fwd_schedule(p, false);
 
   // backward: items grouped by kv tile, q-tile descending within a kv tile.
   // The backward kernel walks each list in this order, so the persistent CTAs

@@ -25,6 +25,7 @@ struct sap_plan_s {
   std::vector<int32_t> fwd_order;   // [U]
   std::vector<int32_t> merges;      // [M][3] (q_tile, first_slot, n_slots)
   int64_t n_slots = 0;
+  bool fused_merge = false;  // forward units span all kv chunks of a q-tile (no partials)
 
   // backward schedule
   std::vector<int32_t> kv_units;    // [V][3] (kv_tile, first_entry, n_entries), heavy-first
@@ -43,6 +44,8 @@ struct sap_plan_s {
   size_t off_items = 0, off_units = 0, off_order = 0, off_merges = 0, off_kv_units = 0, off_kv_entries = 0,
          off_tok_lo = 0, off_tok_hi = 0, dev_words = 0;
 };
+
+void sap_plan_build_fwd_schedule(sap_plan_s* p, bool fused);
 
 int sap_plan_build(const int32_t* cu, int32_t num_docs, int64_t n, int32_t num_chunks, int32_t block_m,
                    int32_t block_n, sap_plan_s* p);

@@ -164,3 +164,24 @@ def test_long_document_elementwise():
     element of O, LSE, dQ, dK, dV against the full oracle, with kv tiles that
     loop over 32 q tiles x 4 heads."""
     _fwd_bwd_full([4096, 300, 1200, 1700, 896], 8, 2, 128, 4, seed=21)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_fused_merge_mode(d):
+    """Fused-merge schedule (one pass over all kv chunks of a q-tile): same result as the oracle,
+    and within rounding of the chunked path."""
+    b = workloads.custom_batch([1500, 300, 248], 4, 2, d, seed=41, with_do=True)
+    r = Run(b, 4)
+    o_c, l_c = r.fwd()
+    o_c, l_c = o_c.clone(), l_c.clone()
+    sap.sap_plan_set_fused_merge(r.plan, True)
+    o, lse = r.fwd()
+    ro, rl = oracle.attn_fwd(b.q, b.k, b.v, b.cu_seqlens, r.scale)
+    assert_close(o, ro, "O (fused merge)")
+    assert_lse(lse, rl)
+    assert_close(o, o_c.double().cpu().numpy(), "O fused vs chunked")
+    dq, dk, dv = r.bwd()
+    rdq, rdk, rdv = oracle.attn_bwd(b.q, b.k, b.v, b.do, b.cu_seqlens, r.scale)
+    assert_close(dq, rdq, "dQ")
+    assert_close(dk, rdk, "dK")
+    assert_close(dv, rdv, "dV")

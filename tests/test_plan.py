@@ -157,3 +157,29 @@ def test_workspace_sizes_and_head_checks():
     with pytest.raises(sap.SapError) as e:
         sap.sap_workspace_size(plan, 4, 4, 96, sap.SAP_WS_FWD)   # unsupported head_dim
     assert e.value.status == -7
+
+
+@pytest.mark.parametrize("name", ["tiny", "llama31_8b_128k"])
+def test_fused_merge_schedule(name):
+    """Fused-merge mode: one forward unit per q-tile covering all its items, no slots, no merges;
+    switching back restores the chunked schedule exactly."""
+    w = workloads.WORKLOADS[name]
+    cu = workloads.cu_seqlens_from_lengths(workloads.doc_lengths(w, 0))
+    plan = sap.sap_plan(cu, w.n, w.p)
+    items = sap.sap_plan_items(plan)
+    chunked = sap.sap_plan_fwd_schedule(plan)
+    sap.sap_plan_set_fused_merge(plan, True)
+    units, order, merges = sap.sap_plan_fwd_schedule(plan)
+    qts = np.unique(items[:, 0])
+    assert len(units) == len(qts) and len(merges) == 0
+    assert np.all(units[:, 3] == -1) and sap.sap_plan_stats(plan)["n_partial_slots"] == 0
+    pos = 0
+    for qt, b, c, _ in units:
+        assert b == pos and np.all(items[b:b + c, 0] == qt) and (b + c == len(items) or items[b + c, 0] != qt)
+        pos += c
+    assert pos == len(items)
+    assert sorted(order.tolist()) == list(range(len(units)))
+    assert sap.sap_workspace_size(plan, w.hq, w.hkv, w.d, sap.SAP_WS_FWD) == 0
+    sap.sap_plan_set_fused_merge(plan, False)
+    for a, b in zip(chunked, sap.sap_plan_fwd_schedule(plan)):
+        np.testing.assert_array_equal(a, b)
