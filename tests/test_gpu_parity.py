@@ -185,3 +185,9 @@ def test_fused_merge_mode(d):
     assert_close(dq, rdq, "dQ")
     assert_close(dk, rdk, "dK")
     assert_close(dv, rdv, "dV")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_odd_gqa_group_uses_one_tile_forward(d):
+    """Group size 3 (odd): the one-tile forward kernel with GQA, plus the backward."""
+    _fwd_bwd_full([700, 200, 124], 6, 2, d, 2, seed=42)
