@@ -126,9 +126,6 @@ __global__ void __launch_bounds__(448, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  // Work items are kv-head-major (all kv tiles of kv head 0, heavy-first, then kv head 1, ...):
-  // the CTAs running at the same time then share one head group's Q, dO and dQ rows, so a sweep
-  // of the q tiles touches an eighth of the data that an all-heads-at-once order would.
   const int total = p.n_kv_units * p.hkv;
   const int G = p.group;
 
@@ -142,7 +139,7 @@ __global__ void __launch_bounds__(448, 1)
       uint32_t unit_iter = 0, q_iter = 0;
       bool ok = true;
       for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
-        const int g = w / p.n_kv_units, u = w % p.n_kv_units;
+        const int u = w / p.hkv, g = w % p.hkv;
         const int kt = p.kv_units[3 * u], e0 = p.kv_units[3 * u + 1], ne = p.kv_units[3 * u + 2];
         if (!mbar_wait(kv_empty, (unit_iter & 1) ^ 1, guard, kErrTimeoutLoad)) break;
         mbar_arrive_expect_tx(kv_full, 2 * C::TILE);
@@ -204,7 +201,7 @@ __global__ void __launch_bounds__(448, 1)
         return true;
       };
       for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
-        const int u = w % p.n_kv_units;
+        const int u = w / p.hkv;
         const int n_it = p.kv_units[3 * u + 2] * G;
         if (!mbar_wait(kv_full, unit_iter & 1, guard, kErrTimeoutMma)) break;
         tc_fence_after();
@@ -277,7 +274,7 @@ __global__ void __launch_bounds__(448, 1)
     uint32_t it = 0;
     bool ok = true;
     for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
-      const int u = w % p.n_kv_units;
+      const int u = w / p.hkv;
       const int kt = p.kv_units[3 * u], e0 = p.kv_units[3 * u + 1], ne = p.kv_units[3 * u + 2];
       const int64_t jrow = (int64_t)kt * 128 + t;
       const bool real_row = jrow < p.n;
@@ -364,7 +361,7 @@ __global__ void __launch_bounds__(448, 1)
     uint32_t it = 0, unit_iter = 0;
     bool ok = true;
     for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
-      const int g = w / p.n_kv_units, u = w % p.n_kv_units;
+      const int u = w / p.hkv, g = w % p.hkv;
       const int kt = p.kv_units[3 * u], e0 = p.kv_units[3 * u + 1], ne = p.kv_units[3 * u + 2];
       int qt_next = p.entries[2 * e0];
       for (int e = 0; e < ne && ok; ++e) {
