@@ -225,8 +225,7 @@ __global__ void __launch_bounds__(192, 1)
         if (!mbar_wait_warp(s_full + b, (s_iter >> 1) & 1, guard, kErrTimeoutSoftmax)) { ok = false; break; }
         tc_fence_after();
         float sv[128];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(lane_base + 128 * b + 32 * c, sv + 32 * c);
+        tmem_ld128(lane_base + 128 * b, sv);
         tc_fence_before();
         mbar_arrive(s_empty + b);
         ++s_iter;
@@ -564,8 +563,7 @@ __global__ void __launch_bounds__(320, 1)
         if (!mbar_wait_warp(s_full + tile, tile_iter & 1, guard, kErrTimeoutSoftmax)) { ok = false; break; }
         tc_fence_after();
         float sv[128];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(lane_base + colS + 32 * c, sv + 32 * c);
+        tmem_ld128(lane_base + colS, sv);
         if (tag != 0) {
           const int c_lo = row_lo - kt * 128, c_hi = row_hi - kt * 128;
 #pragma unroll
