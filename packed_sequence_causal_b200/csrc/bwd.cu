@@ -295,21 +295,26 @@ __global__ void __launch_bounds__(448, 1)
           float pr[64];
           {
             const float4* l4 = reinterpret_cast<const float4*>(lse2);
-            tmem_ld64(R1, pr);  // S^T of this half's 64 columns, turned into P^T in place
-            if (tag == 0) {     // FULL tile: no pair is masked
+            float sv[32];
 #pragma unroll
-              for (int e4 = 0; e4 < 64; e4 += 4) {
-                const float4 l = l4[e4 / 4];
-                pr[e4] = ex2(fmaf(pr[e4], sl2, -l.x));
-                pr[e4 + 1] = ex2(fmaf(pr[e4 + 1], sl2, -l.y));
-                pr[e4 + 2] = ex2(fmaf(pr[e4 + 2], sl2, -l.z));
-                pr[e4 + 3] = ex2(fmaf(pr[e4 + 3], sl2, -l.w));
-              }
-            } else {
+            for (int c = 0; c < 2; ++c) {
+              tmem_ld32(R1 + 32 * c, sv);
+              if (tag == 0) {  // FULL tile: no pair is masked
 #pragma unroll
-              for (int col = 0; col < 64; ++col) {
-                const bool valid = col >= c_lo && col <= c_hi;
-                pr[col] = valid ? ex2(fmaf(pr[col], sl2, -lse2[col])) : 0.f;
+                for (int e4 = 0; e4 < 32; e4 += 4) {
+                  const float4 l = l4[(32 * c + e4) / 4];
+                  pr[32 * c + e4] = ex2(fmaf(sv[e4], sl2, -l.x));
+                  pr[32 * c + e4 + 1] = ex2(fmaf(sv[e4 + 1], sl2, -l.y));
+                  pr[32 * c + e4 + 2] = ex2(fmaf(sv[e4 + 2], sl2, -l.z));
+                  pr[32 * c + e4 + 3] = ex2(fmaf(sv[e4 + 3], sl2, -l.w));
+                }
+              } else {
+#pragma unroll
+                for (int e2 = 0; e2 < 32; ++e2) {
+                  const int col = 32 * c + e2;
+                  const bool valid = col >= c_lo && col <= c_hi;
+                  pr[col] = valid ? ex2(fmaf(sv[e2], sl2, -lse2[col])) : 0.f;
+                }
               }
             }
             uint32_t pk[32];
