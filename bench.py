@@ -108,6 +108,24 @@ class ClockSampler:
                 "samples": len(sm), "power_w_max": max(power)}
 
 
+# ------------------------------------------------------------------ traffic
+
+
+def measured_traffic(workload: str):
+    """DRAM bytes per launch of the backward kernel from the committed ncu capture, or None when the
+    capture is of another workload or the kernel source has changed since it was taken."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", f"traffic_sap_bwd_kernel_{workload}.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        rec = json.load(f)
+    src = os.path.join(ROOT, rec["source"])
+    if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest() != rec["source_sha256"]:
+        return None
+    return rec["dram_bytes_read"] + rec["dram_bytes_write"]
+
+
 # ------------------------------------------------------------------ ranks
 
 
@@ -369,7 +387,8 @@ def main():
             "roofline": {"bound": "tensor", "kernel": "sap_attn_bwd (bwd_pre + sap_bwd_kernel + dq_post)",
                          "achieved": round(achieved, 1), "peak": sustained, "unit": "TFLOP/s",
                          "frac": round(achieved / sustained, 4), "frac_of_burst_peak": round(achieved / burst, 4),
-                         "traffic": None},
+                         "traffic": None if args.tokens else measured_traffic(w.name),
+                         "traffic_unit": "bytes per sap_bwd_kernel launch (dram__bytes_read + dram__bytes_write)"},
             "clocks": clocks,
             "gpu_launches": launches_per_step * args.steps,
             "e2e": e2e,
