@@ -83,7 +83,7 @@ int make_map(CUtensorMap* map, const void* base, int64_t rows, int32_t heads, in
 int make_map_f32_tile(CUtensorMap* map, void* base, int64_t rows, int32_t heads, int32_t hd) {
   cuuint64_t dims[3] = {(cuuint64_t)hd, (cuuint64_t)heads, (cuuint64_t)rows};
   cuuint64_t strides[2] = {(cuuint64_t)hd * 4, (cuuint64_t)heads * hd * 4};
-  cuuint32_t box[3] = {(cuuint32_t)hd, 1, 128};
+  cuuint32_t box[3] = {(cuuint32_t)hd, 1, 64};  // half a q tile: the kernel stages and reduces 64 rows at a time
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,

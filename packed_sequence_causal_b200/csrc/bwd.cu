@@ -50,10 +50,12 @@ struct BwdCfg {
   static constexpr int STAGE = 2 * TILE + 2 * VEC;
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + TILE;
+  // d = 64: dS^T (128 x 128 bf16).  d = 128: dS^T lives in the dO half of its iteration's stage and this
+  // region stages half a dQ tile (64 q rows x 128 fp32) for the TMA reduction.
   static constexpr int OFF_DS = OFF_V + TILE;
   static constexpr int OFF_ST = OFF_DS + 128 * 128 * 2;  // stages: Q, dO, lse2, dvec
   static constexpr int OFF_BAR = OFF_ST + NSQ * STAGE;
-  static constexpr int NBAR = 2 + 2 * NSQ + 11;
+  static constexpr int NBAR = 2 + 2 * NSQ + 13;
   // The dynamic shared window starts 1024-byte aligned (checked at run time),
   // so no alignment slack is reserved: the D = 128 layout needs 231,568 bytes.
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16;
@@ -89,7 +91,9 @@ __global__ void __launch_bounds__(448, 1)
   uint64_t* dkdv_full = dq_free + 1;
   uint64_t* dkdv_free = dkdv_full + 1;
   uint64_t* mma_drain = dkdv_free + 1;
-  uint64_t* stg_ready = mma_drain + 1;  // dQ tile staged in shared memory (d = 128)
+  uint64_t* stg_ready = mma_drain + 1;  // half dQ tile staged in shared memory (d = 128)
+  uint64_t* stg_free = stg_ready + 1;   // its reduction has read the staging buffer (d = 128)
+  uint64_t* dv_done = stg_free + 1;     // dV has read dO: dS^T may go over it (d = 128)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBAR);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -114,6 +118,8 @@ __global__ void __launch_bounds__(448, 1)
     mbar_init(dkdv_free, 128);
     mbar_init(mma_drain, 1);
     mbar_init(stg_ready, 128);
+    mbar_init(stg_free, 1);
+    mbar_init(dv_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -228,6 +234,8 @@ __global__ void __launch_bounds__(448, 1)
           for (int kk = 0; kk < 128 / 16; ++kk)
             mma_bf16_tmem_a(tmem + C::COL_DV, R1 + (kk / 4) * 64 + (kk % 4) * 8,
                             sdesc_sw128(sDO + kk * 2048, C::BOX, 1024), id_kv, (j > 0 || kk > 0) ? 1u : 0u);
+          if (C::DQ_T) tc_commit(dv_done);
+          const uint32_t sDSj = C::DQ_T ? sDO : sDS;  // d = 128: dS^T_j over dO_j
           // S^T_{j+1}: R1 is rewritten only after dV_j (issued above) has read P^T_j
           if (j + 1 < n_it && !issue_s(it + 1)) { ok = false; break; }
           // dK += dS^T_j Q_j ; dQ_j
@@ -235,7 +243,7 @@ __global__ void __launch_bounds__(448, 1)
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < 128 / 16; ++kk) {
-            const uint64_t a = sdesc_sw128(sDS + (kk / 4) * C::BOX + (kk % 4) * 32, 16, 1024);
+            const uint64_t a = sdesc_sw128(sDSj + (kk / 4) * C::BOX + (kk % 4) * 32, 16, 1024);
             mma_bf16(tmem + C::COL_DK, a, sdesc_sw128(sQ + kk * 2048, C::BOX, 1024), id_kv,
                      (j > 0 || kk > 0) ? 1u : 0u);
           }
@@ -246,13 +254,12 @@ __global__ void __launch_bounds__(448, 1)
             // D=128: dQ^T[d][q] = sum_kv K[kv][d] dS^T[kv][q]  (A = K, B = dS^T, both MN-major)
             // D=64 : dQ[q][d]   = sum_kv dS^T[kv][q] K[kv][d]  (A = dS^T, B = K, both MN-major)
             const uint64_t kd = sdesc_sw128(sK + kk * 2048, C::BOX, 1024);
-            const uint64_t sd = sdesc_sw128(sDS + kk * 2048, C::BOX, 1024);
+            const uint64_t sd = sdesc_sw128(sDSj + kk * 2048, C::BOX, 1024);
             mma_bf16(tmem + C::COL_DQ, C::DQ_T ? kd : sd, C::DQ_T ? sd : kd, id_dq, kk > 0);
           }
           tc_commit(dq_full);
-          tc_commit(ds_free);
-          // d = 128: the dQ drain stages its tile in this stage and releases it after the reduction has read it
-          if (!C::DQ_T) tc_commit(q_empty + it % C::NSQ);
+          if (!C::DQ_T) tc_commit(ds_free);
+          tc_commit(q_empty + it % C::NSQ);
         }
         if (!ok) break;
         tc_commit(dkdv_full);
@@ -269,7 +276,6 @@ __global__ void __launch_bounds__(448, 1)
     const int t = quad * 32 + lane;    // kv row within the tile
     const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
     const uint32_t R1 = lane_base + C::COL_R1 + 64 * half, R2 = lane_base + C::COL_R2 + 64 * half;
-    uint8_t* sDSt = smem + C::OFF_DS + half * C::BOX;
     const float sl2 = p.scale_log2;
     uint32_t it = 0;
     bool ok = true;
@@ -325,8 +331,16 @@ __global__ void __launch_bounds__(448, 1)
           tc_fence_before();
           mbar_arrive(p_ready);
           if (!mbar_wait_warp(dp_full, it & 1, guard, kErrTimeoutSoftmax)) { ok = false; break; }
-          if (it > 0 && !mbar_wait_warp(ds_free, (it - 1) & 1, guard, kErrTimeoutSoftmax)) { ok = false; break; }
+          // d = 64: dS^T has its own buffer, free once dK/dQ of the previous iteration completed.
+          // d = 128: dS^T goes over dO_j once dV_j (its last reader) has completed.
+          if (C::DQ_T ? !mbar_wait_warp(dv_done, it & 1, guard, kErrTimeoutSoftmax)
+                      : (it > 0 && !mbar_wait_warp(ds_free, (it - 1) & 1, guard, kErrTimeoutSoftmax))) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
+          uint8_t* sDSt = (C::DQ_T ? smem + C::OFF_ST + (it % C::NSQ) * C::STAGE + C::TILE : smem + C::OFF_DS) +
+                          half * C::BOX;
           const float4* d4 = reinterpret_cast<const float4*>(dvec);
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
@@ -358,7 +372,7 @@ __global__ void __launch_bounds__(448, 1)
     const int quad = warp & 3;
     const int t = quad * 32 + lane;
     const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
-    uint32_t it = 0, unit_iter = 0;
+    uint32_t it = 0, unit_iter = 0, hs = 0;  // hs: half-tile stagings (d = 128)
     bool ok = true;
     for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
       const int u = w / p.hkv, g = w % p.hkv;
@@ -372,31 +386,50 @@ __global__ void __launch_bounds__(448, 1)
           if (!mbar_wait_warp(dq_full, it & 1, guard, kErrTimeoutEpilogue)) { ok = false; break; }
           tc_fence_after();
           if (C::DQ_T) {
-            // Lane t holds feature t of dQ^T (one column per q row).  The fp32 tile is staged,
-            // row-major [q][d], over this iteration's Q/dO stage (no MMA reads it any more once
-            // dq_full has fired) and added to the accumulator by one TMA bulk reduction.
-            const int s = it % C::NSQ;
-            float* stg = reinterpret_cast<float*>(smem + C::OFF_ST + s * C::STAGE);
+            // Lane t holds feature t of dQ^T (one column per q row).  Each half of the tile (64 q rows)
+            // is staged row-major [q][d] in the dedicated buffer and added to the accumulator by one TMA
+            // bulk reduction; thread 0 releases the buffer once the reduction has read it.  stg_ready
+            // needs every drain thread and stg_free follows it, so neither parity wait can skip a phase.
+            float* stg = reinterpret_cast<float*>(smem + C::OFF_DS);
+            if (hs > 0 && !mbar_wait_warp(stg_free, (hs - 1) & 1, guard, kErrTimeoutEpilogue)) { ok = false; break; }
 #pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 0; c < 2; ++c) {
               float v[32];
               tmem_ld32(lane_base + C::COL_DQ + 32 * c, v);
-              if (c == 3) {  // all of dQ^T is in registers: R2 may take the next dP^T
-                tc_fence_before();
-                mbar_arrive(dq_free);
-              }
 #pragma unroll
               for (int e2 = 0; e2 < 32; ++e2) stg[(32 * c + e2) * 128 + t] = v[e2] * p.scale;
             }
             fence_async_smem();
             mbar_arrive(stg_ready);
-            if (!mbar_wait_warp(stg_ready, it & 1, guard, kErrTimeoutEpilogue)) { ok = false; break; }
+            float v2[32], v3[32];
+            tmem_ld32(lane_base + C::COL_DQ + 64, v2);
+            tmem_ld32(lane_base + C::COL_DQ + 96, v3);
+            tc_fence_before();
+            mbar_arrive(dq_free);  // all of dQ^T is in registers or staged: R2 may take the next dP^T
+            if (!mbar_wait_warp(stg_ready, hs & 1, guard, kErrTimeoutEpilogue)) { ok = false; break; }
             if (t == 0) {
               tma_reduce_add_3d(&tmDQ, stg, 0, h, qt * 128);
               bulk_commit_group();
               bulk_wait_group_read0();
-              mbar_arrive(q_empty + s);
+              mbar_arrive(stg_free);
             }
+            ++hs;
+            if (!mbar_wait_warp(stg_free, (hs - 1) & 1, guard, kErrTimeoutEpilogue)) { ok = false; break; }
+#pragma unroll
+            for (int e2 = 0; e2 < 32; ++e2) {
+              stg[e2 * 128 + t] = v2[e2] * p.scale;
+              stg[(32 + e2) * 128 + t] = v3[e2] * p.scale;
+            }
+            fence_async_smem();
+            mbar_arrive(stg_ready);
+            if (!mbar_wait_warp(stg_ready, hs & 1, guard, kErrTimeoutEpilogue)) { ok = false; break; }
+            if (t == 0) {
+              tma_reduce_add_3d(&tmDQ, stg, 0, h, qt * 128 + 64);
+              bulk_commit_group();
+              bulk_wait_group_read0();
+              mbar_arrive(stg_free);
+            }
+            ++hs;
             continue;
           } else {
             // lane t = q row t of the tile
