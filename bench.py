@@ -108,6 +108,40 @@ class ClockSampler:
                 "samples": len(sm), "power_w_max": max(power)}
 
 
+class EnergyMeter:
+    """Board energy over the timed region from NVML's cumulative energy counter (millijoules).
+
+    On this part the 1 kW board limit (sw_power_cap) sets the clock under load, so energy per step,
+    not cycles per step, decides throughput; the line reports it beside the time."""
+
+    def __init__(self, gpu_index: int):
+        self.h = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(gpu_index)
+            self.e0 = None
+        except Exception:
+            self.h = None
+
+    def start(self):
+        if self.h is not None:
+            try:
+                self.e0 = self.nvml.nvmlDeviceGetTotalEnergyConsumption(self.h)
+            except Exception:
+                self.h = None
+
+    def stop(self):
+        """Joules spent by this GPU since start(), or None."""
+        if self.h is None or self.e0 is None:
+            return None
+        try:
+            return (self.nvml.nvmlDeviceGetTotalEnergyConsumption(self.h) - self.e0) / 1e3
+        except Exception:
+            return None
+
+
 # ------------------------------------------------------------------ traffic
 
 
@@ -289,16 +323,19 @@ def main():
         gpu_index = int(vis)
     sampler = ClockSampler(gpu_index)
     sampler.start()
+    meter = EnergyMeter(gpu_index)
     time.sleep(0.4)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
+    meter.start()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     start.record(stream)
     for i in range(args.steps):
         step(evs[i])
     end.record(stream)
     torch.cuda.synchronize()
+    joules = meter.stop()
     if world > 1:
         dist.barrier()
     clocks = sampler.stop()
@@ -309,6 +346,18 @@ def main():
 
     f_fwd, f_bwd = _flops(w, pairs)
     f_step = f_fwd + f_bwd
+    # board energy, summed over the ranks' GPUs (every rank takes the collective, measured or not)
+    je = torch.tensor([joules or 0.0, 0.0 if joules is not None else 1.0], dtype=torch.float64,
+                      device=dev if world > 1 else "cpu")
+    if world > 1:
+        dist.all_reduce(je)
+    energy = None
+    if je[1].item() == 0 and je[0].item() > 0:
+        j_all = float(je[0].item())
+        energy = {"joules_per_step": round(j_all / args.steps, 2),
+                  "avg_watts_per_gpu": round(j_all / world / (start.elapsed_time(end) / 1e3), 1),
+                  "tflop_per_joule": round(f_step * world / (j_all / args.steps) / 1e12, 3),
+                  "source": "NVML total energy counter over the timed region"}
     ms_step = elapsed_ms / args.steps
     value = job_throughput(f_step, args.steps, world, elapsed_ms)
     tokens_s = world * n * args.steps / (elapsed_ms / 1e3)
@@ -390,6 +439,7 @@ def main():
                          "traffic": None if args.tokens else measured_traffic(w.name),
                          "traffic_unit": "bytes per sap_bwd_kernel launch (dram__bytes_read + dram__bytes_write)"},
             "clocks": clocks,
+            "energy": energy,
             "gpu_launches": launches_per_step * args.steps,
             "e2e": e2e,
             "cpu_baseline": cpu,

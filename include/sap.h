@@ -105,8 +105,11 @@ int sap_plan_fwd_schedule(sap_plan_t plan, const int32_t** units, int64_t* n_uni
                           const int32_t** merges, int64_t* n_merges);
 
 /* Backward schedule, host memory owned by the plan:
- *   kv_units: int32[n_kv_units][3] = (kv_tile, first_entry, n_entries), heavy-first;
- *   entries:  int32[n_items][2] = (q_tile, tag), grouped by kv tile, q-tile descending. */
+ *   entries:  int32[n_items][2] = (q_tile, tag), grouped by kv tile, q-tile descending;
+ *   kv_units: int32[n_kv_units][3] = (kv_tile, first_entry, n_entries).  A unit is the part of one
+ *             kv tile's entries whose q tiles fall in one band of 16 q tiles (q_tile / 16 equal), so a
+ *             kv tile may have several units.  Units are ordered band-major (top band first) and
+ *             heavy-first (n_entries descending, ties by kv tile) within a band. */
 int sap_plan_bwd_schedule(sap_plan_t plan, const int32_t** kv_units, int64_t* n_kv_units, const int32_t** entries);
 
 /* Fused-merge mode (enable != 0): the forward schedule gets one unit per
@@ -130,7 +133,8 @@ void sap_plan_destroy(sap_plan_t plan);
 /* Workspace bytes for a call with these head counts (which = SAP_WS_FWD for
  * sap_attn_fwd + sap_merge, SAP_WS_BWD for sap_attn_bwd).  The forward
  * workspace holds the fp32 partial outputs and LSEs of the partial slots; the
- * backward one holds the fp32 dQ accumulator and the per-row D and LSE*log2(e). */
+ * backward one holds the fp32 dQ, dK and dV accumulators and the per-row D and
+ * LSE*log2(e). */
 int sap_workspace_size(sap_plan_t plan, int32_t hq, int32_t hkv, int32_t head_dim, int32_t which, size_t* bytes);
 
 /* Forward: for every forward unit (q-tile, kv-chunk) and head, the partial
@@ -154,8 +158,9 @@ int sap_merge(sap_plan_t plan, const void* workspace, size_t ws_bytes, int32_t h
  * dV_j = sum P_ij dO_i, dS_ij = P_ij (<dO_i, V_j> - D_i), dQ_i = scale sum_j dS_ij K_j,
  * dK_j = scale sum_i dS_ij Q_i, with dK/dV summed over the q heads of each kv
  * head.  Chunk pairs need no merge here: the final LSE normalises every pair
- * and their gradients add.  dQ is accumulated in fp32 in the workspace and
- * converted to bf16 at the end. */
+ * and their gradients add.  dQ, dK and dV are accumulated in fp32 in the
+ * workspace (dQ once per (q tile, kv tile, head), dK/dV once per backward unit)
+ * and converted to bf16 at the end. */
 int sap_attn_bwd(sap_plan_t plan, const void* q, const void* k, const void* v, const void* o, const float* lse,
                  const void* dout, int32_t hq, int32_t hkv, int32_t head_dim, float softmax_scale, void* dq,
                  void* dk, void* dv, void* workspace, size_t ws_bytes, void* stream);

@@ -92,6 +92,20 @@ int make_map_f32_tile(CUtensorMap* map, void* base, int64_t rows, int32_t heads,
   return SAP_OK;
 }
 
+// fp32 [rows][heads][hd] accumulator (dK then dV, rows = 2 * n_pad), reduced into in boxes of
+// 32 features x 128 rows with 128-byte swizzle (the staging layout the drain warps write).
+int make_map_f32_sw128(CUtensorMap* map, void* base, int64_t rows, int32_t heads, int32_t hd) {
+  cuuint64_t dims[3] = {(cuuint64_t)hd, (cuuint64_t)heads, (cuuint64_t)rows};
+  cuuint64_t strides[2] = {(cuuint64_t)hd * 4, (cuuint64_t)heads * hd * 4};
+  cuuint32_t box[3] = {32, 1, 128};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
+  return SAP_OK;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
@@ -121,15 +135,16 @@ FwdWs fwd_ws(const sap_plan_s* p, int32_t hq, int32_t hd) {
   return w;
 }
 struct BwdWs {
-  size_t dq_acc = 0, dvec = 0, lse2 = 0, total = 0;
+  size_t dq_acc = 0, dkv_acc = 0, dvec = 0, lse2 = 0, total = 0;
   int64_t n_pad = 0;
 };
-BwdWs bwd_ws(const sap_plan_s* p, int32_t hq, int32_t hd) {
+BwdWs bwd_ws(const sap_plan_s* p, int32_t hq, int32_t hkv, int32_t hd) {
   BwdWs w;
   w.n_pad = round_up(p->n, 128);
-  w.dq_acc = 0;
-  w.dvec = round_up(w.n_pad * hq * hd * 4, 256);
-  w.lse2 = w.dvec + round_up(w.n_pad * hq * 4, 256);
+  w.dq_acc = 0;                                                             // [n_pad][hq][hd] fp32
+  w.dkv_acc = round_up(w.n_pad * hq * hd * 4, 1024);                        // [2][n_pad][hkv][hd] fp32
+  w.dvec = w.dkv_acc + round_up(2 * w.n_pad * hkv * hd * 4, 256);           // [hq][n_pad]
+  w.lse2 = w.dvec + round_up(w.n_pad * hq * 4, 256);                        // [hq][n_pad]
   w.total = w.lse2 + round_up(w.n_pad * hq * 4, 256);
   return w;
 }
@@ -301,7 +316,7 @@ int sap_workspace_size(sap_plan_t plan, int32_t hq, int32_t hkv, int32_t head_di
   if (which == SAP_WS_FWD)
     *bytes = fwd_ws(plan, hq, head_dim).total;
   else if (which == SAP_WS_BWD)
-    *bytes = bwd_ws(plan, hq, head_dim).total;
+    *bytes = bwd_ws(plan, hq, hkv, head_dim).total;
   else
     return SAP_ERR_INVALID_ARG;
   return SAP_OK;
@@ -391,7 +406,7 @@ int sap_attn_bwd(sap_plan_t p, const void* q, const void* k, const void* v, cons
   const void* ptrs[] = {q, k, v, o, lse, dout, dq, dk, dv};
   for (const void* ptr : ptrs)
     if (!aligned16(ptr)) return SAP_ERR_INVALID_ARG;
-  const BwdWs ws = bwd_ws(p, hq, head_dim);
+  const BwdWs ws = bwd_ws(p, hq, hkv, head_dim);
   if (!workspace || ws_bytes < ws.total || !aligned16(workspace)) return SAP_ERR_WORKSPACE;
   DeviceInfo* di = nullptr;
   if ((rc = device_info(&di))) return rc;
@@ -403,15 +418,18 @@ int sap_attn_bwd(sap_plan_t p, const void* q, const void* k, const void* v, cons
   if ((rc = make_map(&tdo, dout, p->n, hq, head_dim))) return rc;
   uint8_t* wsb = static_cast<uint8_t*>(workspace);
   float* dq_acc = reinterpret_cast<float*>(wsb + ws.dq_acc);
-  CUtensorMap tdq;
+  float* dkv_acc = reinterpret_cast<float*>(wsb + ws.dkv_acc);
+  CUtensorMap tdq, tdkv;
   if ((rc = make_map_f32_tile(&tdq, dq_acc, ws.n_pad, hq, head_dim))) return rc;
+  if ((rc = make_map_f32_sw128(&tdkv, dkv_acc, 2 * ws.n_pad, hkv, head_dim))) return rc;
   float* dvec = reinterpret_cast<float*>(wsb + ws.dvec);
   float* lse2 = reinterpret_cast<float*>(wsb + ws.lse2);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const __nv_bfloat16* ob = static_cast<const __nv_bfloat16*>(o);
   const __nv_bfloat16* dob = static_cast<const __nv_bfloat16*>(dout);
-  cudaError_t e = head_dim == 64 ? sap::launch_bwd_pre<64>(ob, dob, lse, p->n, ws.n_pad, hq, dvec, lse2, dq_acc, s)
-                                 : sap::launch_bwd_pre<128>(ob, dob, lse, p->n, ws.n_pad, hq, dvec, lse2, dq_acc, s);
+  cudaError_t e = head_dim == 64
+                      ? sap::launch_bwd_pre<64>(ob, dob, lse, p->n, ws.n_pad, hq, hkv, dvec, lse2, dq_acc, dkv_acc, s)
+                      : sap::launch_bwd_pre<128>(ob, dob, lse, p->n, ws.n_pad, hq, hkv, dvec, lse2, dq_acc, dkv_acc, s);
   if (e != cudaSuccess) return cuda_fail(e);
   const int32_t* base = static_cast<const int32_t*>(p->dev);
   sap::BwdParams bp;
@@ -429,17 +447,17 @@ int sap_attn_bwd(sap_plan_t p, const void* q, const void* k, const void* v, cons
   bp.lse2 = lse2;
   bp.dvec = dvec;
   bp.dq_acc = dq_acc;
-  bp.dk = static_cast<__nv_bfloat16*>(dk);
-  bp.dv = static_cast<__nv_bfloat16*>(dv);
   bp.err = di->err;
   const int64_t work = (int64_t)bp.n_kv_units * hkv;
   if (work > 0) {
     const int grid = (int)(work < di->sms ? work : di->sms);
-    e = head_dim == 64 ? sap::launch_bwd<64>(tq, tk, tv, tdo, tdq, bp, grid, s)
-                       : sap::launch_bwd<128>(tq, tk, tv, tdo, tdq, bp, grid, s);
+    e = head_dim == 64 ? sap::launch_bwd<64>(tq, tk, tv, tdo, tdq, tdkv, bp, grid, s)
+                       : sap::launch_bwd<128>(tq, tk, tv, tdo, tdq, tdkv, bp, grid, s);
     if (e != cudaSuccess) return cuda_fail(e);
   }
-  e = sap::launch_dq_post(dq_acc, static_cast<__nv_bfloat16*>(dq), p->n * hq * head_dim, s);
+  e = sap::launch_bwd_post(dq_acc, static_cast<__nv_bfloat16*>(dq), p->n * hq * head_dim, dkv_acc,
+                           static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv), p->n * hkv * head_dim,
+                           ws.n_pad * hkv * head_dim, s);
   if (e != cudaSuccess) return cuda_fail(e);
   return SAP_OK;
 }

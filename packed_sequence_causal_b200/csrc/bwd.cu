@@ -54,11 +54,17 @@ struct BwdCfg {
   // region stages half a dQ tile (64 q rows x 128 fp32) for the TMA reduction.
   static constexpr int OFF_DS = OFF_V + TILE;
   static constexpr int OFF_ST = OFF_DS + 128 * 128 * 2;  // stages: Q, dO, lse2, dvec
-  static constexpr int OFF_BAR = OFF_ST + NSQ * STAGE;
+  // dK/dV epilogue staging (128 rows x 64 fp32 as two 128-byte-swizzled boxes of 32 features):
+  // d = 128 shares the dQ staging buffer (same warps, same barriers); d = 64 has its own.
+  static constexpr int EPI_BYTES = 128 * 64 * 4;
+  static constexpr int OFF_EPI = (D == 128) ? OFF_DS : OFF_ST + NSQ * STAGE;
+  static constexpr int OFF_BAR = (D == 128) ? OFF_ST + NSQ * STAGE : OFF_EPI + EPI_BYTES;
   static constexpr int NBAR = 2 + 2 * NSQ + 13;
   // The dynamic shared window starts 1024-byte aligned (checked at run time),
-  // so no alignment slack is reserved: the D = 128 layout needs 231,568 bytes.
+  // so no alignment slack is reserved: the D = 128 layout needs 231,592 bytes.
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16;
+  static_assert(SMEM <= 232448, "shared memory per block");
+  static_assert(OFF_EPI % 1024 == 0 && OFF_ST % 1024 == 0 && STAGE % 1024 == 0, "128-byte swizzle alignment");
   static constexpr int THREADS = 448;
   static constexpr uint32_t COL_DK = 0, COL_DV = D, COL_R1 = 2 * D, COL_R2 = 2 * D + 128;
   static constexpr bool DQ_T = (D == 128);  // dQ^T in R2 (coalesced drain) vs dQ in its own columns
@@ -69,7 +75,8 @@ template <int D>
 __global__ void __launch_bounds__(448, 1)
     sap_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-                   const __grid_constant__ CUtensorMap tmDQ, const BwdParams p) {
+                   const __grid_constant__ CUtensorMap tmDQ, const __grid_constant__ CUtensorMap tmDKV,
+                   const BwdParams p) {
   using C = BwdCfg<D>;
   extern __shared__ __align__(1024) uint8_t smem[];
   if (smem_u32(smem) & 1023u) {  // TMA 128-byte swizzle and the descriptors need 1024-byte alignment
@@ -372,7 +379,7 @@ __global__ void __launch_bounds__(448, 1)
     const int quad = warp & 3;
     const int t = quad * 32 + lane;
     const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
-    uint32_t it = 0, unit_iter = 0, hs = 0;  // hs: half-tile stagings (d = 128)
+    uint32_t it = 0, unit_iter = 0, hs = 0;  // hs: uses of the staging buffer (dQ halves, dK/dV pieces)
     bool ok = true;
     for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
       const int u = w / p.hkv, g = w % p.hkv;
@@ -452,31 +459,48 @@ __global__ void __launch_bounds__(448, 1)
       if (!ok) break;
       if (!mbar_wait_warp(dkdv_full, unit_iter & 1, guard, kErrTimeoutEpilogue)) break;
       tc_fence_after();
-      const int64_t jrow = (int64_t)kt * 128 + t;
+      // This unit's dK (times the softmax scale left out of dS) and dV are added to the fp32
+      // accumulators, 64 features at a time: lane t holds row t, stages it into two 128-byte-
+      // swizzled boxes [128 rows][32 fp32], and thread 0 reduces both boxes with the TMA.  Rows past
+      // N hold zeros (their keys and values were loaded as zeros and all their pairs are masked).
+      uint8_t* epi = smem + C::OFF_EPI;
+      constexpr int NCH = 2 * (D / 64);
 #pragma unroll 1
-      for (int which = 0; which < 2; ++which) {
-        __nv_bfloat16* out = (which == 0 ? p.dk : p.dv) + ((size_t)jrow * p.hkv + g) * D;
-        const uint32_t col = which == 0 ? C::COL_DK : C::COL_DV;
-        const float f = which == 0 ? p.scale : 1.f;  // dK carries the softmax scale left out of dS
-#pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          float v[32];
-          tmem_ld32(lane_base + col + 32 * c, v);
-          if (jrow < p.n) {
-#pragma unroll
-            for (int e8 = 0; e8 < 32; e8 += 8) {
-              uint4 pk;
-              pk.x = pack_bf16x2(v[e8] * f, v[e8 + 1] * f);
-              pk.y = pack_bf16x2(v[e8 + 2] * f, v[e8 + 3] * f);
-              pk.z = pack_bf16x2(v[e8 + 4] * f, v[e8 + 5] * f);
-              pk.w = pack_bf16x2(v[e8 + 6] * f, v[e8 + 7] * f);
-              *reinterpret_cast<uint4*>(out + 32 * c + e8) = pk;
-            }
-          }
+      for (int m = 0; m < NCH; ++m) {
+        const int which = m / (D / 64), cb = m % (D / 64);
+        const uint32_t col = (which == 0 ? C::COL_DK : C::COL_DV) + 64 * cb;
+        const float f = which == 0 ? p.scale : 1.f;
+        if (hs > 0 && !mbar_wait_warp(stg_free, (hs - 1) & 1, guard, kErrTimeoutEpilogue)) { ok = false; break; }
+        float v0[32], v1[32];
+        tmem_ld32(lane_base + col, v0);
+        tmem_ld32(lane_base + col + 32, v1);
+        if (m == NCH - 1) {  // all of dK/dV has been read: the next unit may accumulate over it
+          tc_fence_before();
+          mbar_arrive(dkdv_free);
         }
+#pragma unroll
+        for (int c16 = 0; c16 < 8; ++c16) {
+          const uint32_t off = sw128_offset(t, c16);
+          st_shared_v4(smem_u32(epi + off), __float_as_uint(v0[4 * c16] * f), __float_as_uint(v0[4 * c16 + 1] * f),
+                       __float_as_uint(v0[4 * c16 + 2] * f), __float_as_uint(v0[4 * c16 + 3] * f));
+          st_shared_v4(smem_u32(epi + C::EPI_BYTES / 2 + off), __float_as_uint(v1[4 * c16] * f),
+                       __float_as_uint(v1[4 * c16 + 1] * f), __float_as_uint(v1[4 * c16 + 2] * f),
+                       __float_as_uint(v1[4 * c16 + 3] * f));
+        }
+        fence_async_smem();
+        mbar_arrive(stg_ready);
+        if (!mbar_wait_warp(stg_ready, hs & 1, guard, kErrTimeoutEpilogue)) { ok = false; break; }
+        if (t == 0) {
+          const int row0 = (which == 0 ? 0 : (int)p.n_pad) + kt * 128;
+          tma_reduce_add_3d(&tmDKV, epi, 64 * cb, g, row0);
+          tma_reduce_add_3d(&tmDKV, epi + C::EPI_BYTES / 2, 64 * cb + 32, g, row0);
+          bulk_commit_group();
+          bulk_wait_group_read0();
+          mbar_arrive(stg_free);
+        }
+        ++hs;
       }
-      tc_fence_before();
-      mbar_arrive(dkdv_free);
+      if (!ok) break;
       ++unit_iter;
     }
   }
@@ -493,17 +517,18 @@ __global__ void __launch_bounds__(448, 1)
 
 template <int D>
 cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
-                       const CUtensorMap& tdq, const BwdParams& p, int grid, cudaStream_t stream) {
+                       const CUtensorMap& tdq, const CUtensorMap& tdkv, const BwdParams& p, int grid,
+                       cudaStream_t stream) {
   auto kern = sap_bwd_kernel<D>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, BwdCfg<D>::SMEM);
   if (e != cudaSuccess) return e;
-  kern<<<grid, BwdCfg<D>::THREADS, BwdCfg<D>::SMEM, stream>>>(tq, tk, tv, tdo, tdq, p);
+  kern<<<grid, BwdCfg<D>::THREADS, BwdCfg<D>::SMEM, stream>>>(tq, tk, tv, tdo, tdq, tdkv, p);
   return cudaGetLastError();
 }
 
 template cudaError_t launch_bwd<64>(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
-                                    const CUtensorMap&, const BwdParams&, int, cudaStream_t);
+                                    const CUtensorMap&, const CUtensorMap&, const BwdParams&, int, cudaStream_t);
 template cudaError_t launch_bwd<128>(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
-                                     const CUtensorMap&, const BwdParams&, int, cudaStream_t);
+                                     const CUtensorMap&, const CUtensorMap&, const BwdParams&, int, cudaStream_t);
 
 }  // namespace sap

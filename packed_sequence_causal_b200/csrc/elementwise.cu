@@ -90,11 +90,12 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
   if (lane == 0) lse[(size_t)h * n + i] = lse_all;
 }
 
-// D_i = <dO_i, O_i>, LSE_i * log2(e), and a zeroed dQ accumulator row: warp = (row, head).
+// D_i = <dO_i, O_i>, LSE_i * log2(e), and zeroed accumulator rows (dQ for every head, dK and dV
+// for the kv heads): warp = (row, head).
 template <int D>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32)
     bwd_pre_kernel(const __nv_bfloat16* o, const __nv_bfloat16* dout, const float* lse, int64_t n, int64_t n_pad,
-                   int32_t hq, float* dvec, float* lse2, float* dq_acc) {
+                   int32_t hq, int32_t hkv, float* dvec, float* lse2, float* dq_acc, float* dkv_acc) {
   constexpr int E = D / 32;
   const int64_t wid = (int64_t)blockIdx.x * kWarpsPerBlock + threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
@@ -102,6 +103,11 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
   const int64_t i = wid / hq;
   const int h = (int)(wid % hq);
   Vec<E>::store_zero(dq_acc + (size_t)wid * D + lane * E);
+  if (h < hkv) {
+    const size_t kv_row = ((size_t)i * hkv + h) * D + lane * E;
+    Vec<E>::store_zero(dkv_acc + kv_row);
+    Vec<E>::store_zero(dkv_acc + (size_t)n_pad * hkv * D + kv_row);
+  }
   float dsum = 0.f;
   if (i < n) {
     float a[E], b[E];
@@ -118,12 +124,24 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
   }
 }
 
-__global__ void dq_post_kernel(const float* dq_acc, __nv_bfloat16* dq, int64_t count4) {
-  const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (t >= count4) return;
+// fp32 accumulators -> bf16, four values per thread: dQ, then dK, then dV.
+__global__ void bwd_post_kernel(const float* dq_acc, __nv_bfloat16* dq, int64_t q4, const float* dkv_acc,
+                                __nv_bfloat16* dk, __nv_bfloat16* dv, int64_t kv4, int64_t dv_offset) {
+  int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const float* src;
+  __nv_bfloat16* dst;
+  if (t < q4) {
+    src = dq_acc + 4 * t, dst = dq + 4 * t;
+  } else if ((t -= q4) < kv4) {
+    src = dkv_acc + 4 * t, dst = dk + 4 * t;
+  } else if ((t -= kv4) < kv4) {
+    src = dkv_acc + dv_offset + 4 * t, dst = dv + 4 * t;
+  } else {
+    return;
+  }
   float v[4];
-  Vec<4>::load(dq_acc + 4 * t, v);
-  Vec<4>::store_bf16(dq + 4 * t, v);
+  Vec<4>::load(src, v);
+  Vec<4>::store_bf16(dst, v);
 }
 
 }  // namespace
@@ -141,19 +159,23 @@ cudaError_t launch_merge(const int32_t* merges, int64_t n_merges, int32_t hq, in
 
 template <int D>
 cudaError_t launch_bwd_pre(const __nv_bfloat16* o, const __nv_bfloat16* dout, const float* lse, int64_t n,
-                           int64_t n_pad, int32_t hq, float* dvec, float* lse2, float* dq_acc, cudaStream_t stream) {
+                           int64_t n_pad, int32_t hq, int32_t hkv, float* dvec, float* lse2, float* dq_acc,
+                           float* dkv_acc, cudaStream_t stream) {
   const int64_t warps = n_pad * hq;
   if (warps == 0) return cudaSuccess;
   const int64_t blocks = (warps + kWarpsPerBlock - 1) / kWarpsPerBlock;
-  bwd_pre_kernel<D><<<(unsigned)blocks, kWarpsPerBlock * 32, 0, stream>>>(o, dout, lse, n, n_pad, hq, dvec, lse2,
-                                                                          dq_acc);
+  bwd_pre_kernel<D><<<(unsigned)blocks, kWarpsPerBlock * 32, 0, stream>>>(o, dout, lse, n, n_pad, hq, hkv, dvec,
+                                                                          lse2, dq_acc, dkv_acc);
   return cudaGetLastError();
 }
 
-cudaError_t launch_dq_post(const float* dq_acc, __nv_bfloat16* dq, int64_t count, cudaStream_t stream) {
-  const int64_t c4 = count / 4;
-  if (c4 == 0) return cudaSuccess;
-  dq_post_kernel<<<(unsigned)((c4 + 255) / 256), 256, 0, stream>>>(dq_acc, dq, c4);
+cudaError_t launch_bwd_post(const float* dq_acc, __nv_bfloat16* dq, int64_t count_q, const float* dkv_acc,
+                            __nv_bfloat16* dk, __nv_bfloat16* dv, int64_t count_kv, int64_t dv_offset,
+                            cudaStream_t stream) {
+  const int64_t total4 = count_q / 4 + 2 * (count_kv / 4);
+  if (total4 == 0) return cudaSuccess;
+  bwd_post_kernel<<<(unsigned)((total4 + 255) / 256), 256, 0, stream>>>(dq_acc, dq, count_q / 4, dkv_acc, dk, dv,
+                                                                        count_kv / 4, dv_offset);
   return cudaGetLastError();
 }
 
@@ -162,8 +184,8 @@ template cudaError_t launch_merge<64>(const int32_t*, int64_t, int32_t, int64_t,
 template cudaError_t launch_merge<128>(const int32_t*, int64_t, int32_t, int64_t, const float*, const float*,
                                        __nv_bfloat16*, float*, cudaStream_t);
 template cudaError_t launch_bwd_pre<64>(const __nv_bfloat16*, const __nv_bfloat16*, const float*, int64_t, int64_t,
-                                        int32_t, float*, float*, float*, cudaStream_t);
+                                        int32_t, int32_t, float*, float*, float*, float*, cudaStream_t);
 template cudaError_t launch_bwd_pre<128>(const __nv_bfloat16*, const __nv_bfloat16*, const float*, int64_t, int64_t,
-                                         int32_t, float*, float*, float*, cudaStream_t);
+                                         int32_t, int32_t, float*, float*, float*, float*, cudaStream_t);
 
 }  // namespace sap

@@ -25,7 +25,7 @@ struct FwdParams {
 };
 
 struct BwdParams {
-  const int32_t* kv_units;    // [n_kv_units][3] (kv_tile, first_entry, n_entries), heavy-first
+  const int32_t* kv_units;    // [n_kv_units][3] (kv_tile, first_entry, n_entries), band-major
   const int32_t* entries;     // [n_items][2] (q_tile, tag)
   const int32_t* tok_hi;      // [N] last token of each token's document
   int32_t n_kv_units;
@@ -35,9 +35,7 @@ struct BwdParams {
   float scale;                // softmax_scale
   const float* lse2;          // [hq][n_pad] LSE * log2(e) (+inf past N)
   const float* dvec;          // [hq][n_pad] D_i = <dO_i, O_i> (0 past N)
-  float* dq_acc;              // [n_pad][hq][D] fp32 dQ accumulator
-  __nv_bfloat16* dk;          // [N][hkv][D]
-  __nv_bfloat16* dv;          // [N][hkv][D]
+  float* dq_acc;              // [n_pad][hq][D] fp32 dQ accumulator (d = 64: atomics; d = 128: the tdq map)
   int* err;
 };
 
@@ -47,7 +45,8 @@ cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
 
 template <int D>
 cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
-                       const CUtensorMap& tdq, const BwdParams& p, int grid, cudaStream_t stream);
+                       const CUtensorMap& tdq, const CUtensorMap& tdkv, const BwdParams& p, int grid,
+                       cudaStream_t stream);
 
 template <int D>
 cudaError_t launch_merge(const int32_t* merges, int64_t n_merges, int32_t hq, int64_t n, const float* o_part,
@@ -55,8 +54,13 @@ cudaError_t launch_merge(const int32_t* merges, int64_t n_merges, int32_t hq, in
 
 template <int D>
 cudaError_t launch_bwd_pre(const __nv_bfloat16* o, const __nv_bfloat16* dout, const float* lse, int64_t n,
-                           int64_t n_pad, int32_t hq, float* dvec, float* lse2, float* dq_acc, cudaStream_t stream);
+                           int64_t n_pad, int32_t hq, int32_t hkv, float* dvec, float* lse2, float* dq_acc,
+                           float* dkv_acc, cudaStream_t stream);
 
-cudaError_t launch_dq_post(const float* dq_acc, __nv_bfloat16* dq, int64_t count, cudaStream_t stream);
+// fp32 accumulators -> bf16: dq (count_q values), dk and dv (count_kv values each; the dV
+// accumulator starts dv_offset values after the dK one).
+cudaError_t launch_bwd_post(const float* dq_acc, __nv_bfloat16* dq, int64_t count_q, const float* dkv_acc,
+                            __nv_bfloat16* dk, __nv_bfloat16* dv, int64_t count_kv, int64_t dv_offset,
+                            cudaStream_t stream);
 
 }  // namespace sap

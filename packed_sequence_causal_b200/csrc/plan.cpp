@@ -135,10 +135,12 @@ int sap_plan_build(const int32_t* cu, int32_t num_docs, int64_t n, int32_t num_c
 
   sap_plan_build_fwd_schedule(p, false);
 
-  // backward: items grouped by kv tile, q-tile descending within a kv tile.
-  // The backward kernel walks each list in this order, so the persistent CTAs
-  // (which start their heavy kv tiles together) sweep the q tiles from the
-  // top down roughly in step and share Q, dO and dQ rows in L2.
+  // backward: items grouped by kv tile, q-tile descending within a kv tile, and each kv tile's
+  // list cut into bands of kBwdBandTiles q tiles.  A unit is one (kv tile, band) piece; units are
+  // ordered band-major from the top band down, heavy-first within a band.  The persistent CTAs take
+  // units in this order, so at any time they all work on Q, dO and dQ rows of about one band (a few
+  // tens of MB at 32 heads) and those rows stay in L2; the price is one fp32 dK/dV reduction per unit
+  // instead of one bf16 store per kv tile.
   const int64_t ntk = (n + block_n - 1) / block_n;
   std::vector<int64_t> cnt((size_t)ntk + 1, 0);
   for (const auto& it : p->items) cnt[(size_t)it.kv_tile + 1]++;
@@ -152,13 +154,25 @@ int sap_plan_build(const int32_t* cu, int32_t num_docs, int64_t n, int32_t num_c
       p->kv_entries[2 * w + 1] = it.tag;
     }
   }
-  std::vector<int32_t> kvs;
-  for (int64_t t = 0; t < ntk; ++t)
-    if (cnt[t + 1] > cnt[t]) kvs.push_back((int32_t)t);
-  std::stable_sort(kvs.begin(), kvs.end(),
-                   [&](int32_t x, int32_t y) { return cnt[x + 1] - cnt[x] > cnt[y + 1] - cnt[y]; });
+  struct Unit {
+    int32_t band, kv_tile, first, count;
+  };
+  std::vector<Unit> units;
+  for (int64_t t = 0; t < ntk; ++t) {
+    int64_t e = cnt[t];
+    while (e < cnt[t + 1]) {
+      const int32_t band = p->kv_entries[2 * e] / kBwdBandTiles;
+      int64_t f = e + 1;
+      while (f < cnt[t + 1] && p->kv_entries[2 * f] / kBwdBandTiles == band) ++f;
+      units.push_back(Unit{band, (int32_t)t, (int32_t)e, (int32_t)(f - e)});
+      e = f;
+    }
+  }
+  std::stable_sort(units.begin(), units.end(), [](const Unit& a, const Unit& b) {
+    return a.band != b.band ? a.band > b.band : a.count > b.count;
+  });
   p->kv_units.clear();
-  for (int32_t t : kvs)
-    p->kv_units.insert(p->kv_units.end(), {t, (int32_t)cnt[t], (int32_t)(cnt[t + 1] - cnt[t])});
+  p->kv_units.reserve(units.size() * 3);
+  for (const Unit& u : units) p->kv_units.insert(p->kv_units.end(), {u.kv_tile, u.first, u.count});
   return SAP_OK;
 }

@@ -8,6 +8,9 @@
 
 #include "sap.h"
 
+// Backward units cover at most this many q tiles of one kv tile's list (one "band").
+constexpr int32_t kBwdBandTiles = 16;
+
 struct sap_plan_s {
   // inputs
   int64_t n = 0;
@@ -28,7 +31,7 @@ struct sap_plan_s {
   bool fused_merge = false;  // forward units span all kv chunks of a q-tile (no partials)
 
   // backward schedule
-  std::vector<int32_t> kv_units;    // [V][3] (kv_tile, first_entry, n_entries), heavy-first
+  std::vector<int32_t> kv_units;    // [V][3] (kv_tile, first_entry, n_entries): band-major, heavy-first in a band
   std::vector<int32_t> kv_entries;  // [items][2] (q_tile, tag)
 
   // per-token document bounds: first token of the document, last token of the document

@@ -53,18 +53,32 @@ def _check_schedules(plan, items, n, nchunks, bm, bn):
     for a, b in zip(order[:-1], order[1:]):
         if units[a, 2] == units[b, 2]:
             assert a < b
-    # backward: every item once, grouped by kv tile, q-tile descending, heavy-first
+    # backward: every item once; each unit is the part of one kv tile's q-descending list that
+    # falls in one band of 16 q tiles; units band-major (top band first), heavy-first within a
+    # band, ties by kv tile
     kv_units, entries = sap.sap_plan_bwd_schedule(plan)
+    band = 16
     seen = set()
-    prev_cnt = None
+    covered = np.zeros(len(entries), dtype=np.int64)
+    prev = None
     for kt, e0, ne in kv_units:
+        assert ne > 0
         grp = entries[e0:e0 + ne]
         assert np.all(np.diff(grp[:, 0]) < 0)
+        assert len(set((grp[:, 0] // band).tolist())) == 1
+        covered[e0:e0 + ne] += 1
         for qt, tag in grp:
             seen.add((int(qt), int(kt), int(tag)))
-        if prev_cnt is not None:
-            assert ne <= prev_cnt
-        prev_cnt = ne
+        key = (int(grp[0, 0]) // band, int(ne), int(kt))
+        if prev is not None:
+            assert key[0] < prev[0] or (key[0] == prev[0] and (key[1] < prev[1] or
+                                                               (key[1] == prev[1] and key[2] > prev[2])))
+        prev = key
+    assert np.all(covered == 1)
+    assert len(seen) == len(entries)
+    # units of one kv tile do not share a band (each band piece is maximal)
+    pieces = {(int(kt), int(entries[e0, 0]) // band) for kt, e0, _ in kv_units}
+    assert len(pieces) == len(kv_units)
     assert seen == {(int(a), int(b), int(t)) for a, b, _, _, t in items}
 
 
