@@ -365,38 +365,81 @@ def main():
     # per-call device times from the events recorded on the launching stream
     t_fwd, t_merge, t_bwd = (sum(e[c].elapsed_time(e[c + 1]) for e in evs) / args.steps for c in range(3))
 
-    # end to end through the public API: pinned host inputs -> device, the path, results -> pinned host
+    # end to end through the public API: every step copies its inputs from pinned host memory to
+    # the device and reads all of its results back to pinned host memory inside the timed region.
+    # Two device sets of inputs and results let step s+1's inputs arrive and step s's results
+    # leave on two copy streams while the GPU computes (the prefetch a training loop does); the
+    # region opens before the first input copy and closes after the last result has landed.
     e2e = None
     if not args.no_e2e:
-        hq_in = [t.cpu().pin_memory() for t in (q, k, v, do)]
+        h_in = [t.cpu().pin_memory() for t in (q, k, v, do)]
         h_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (o, lse, dq, dk, dv)]
-        dev_in = (q, k, v, do)
-        h2d = sum(t.numel() * t.element_size() for t in hq_in)
+        d_in = [[torch.empty_like(t) for t in (q, k, v, do)] for _ in range(2)]
+        d_out = [[torch.empty_like(t) for t in (o, lse, dq, dk, dv)] for _ in range(2)]
+        s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        h2d = sum(t.numel() * t.element_size() for t in h_in)
         d2h = sum(t.numel() * t.element_size() for t in h_out)
 
-        def e2e_step():
-            for dst, src in zip(dev_in, hq_in):
-                dst.copy_(src, non_blocking=True)
-            step()
-            for dst, src in zip(h_out, (o, lse, dq, dk, dv)):
-                dst.copy_(src, non_blocking=True)
+        def e2e_run(steps, start_ev=None, end_ev=None):
+            ev = lambda: torch.cuda.Event()  # noqa: E731
+            in_ready, in_free = [ev() for _ in range(steps)], [ev() for _ in range(steps)]
+            out_ready, out_free = [ev() for _ in range(steps)], [ev() for _ in range(steps)]
+            if start_ev is not None:
+                start_ev.record(stream)
+            s_in.wait_stream(stream)
+            s_out.wait_stream(stream)
 
-        for _ in range(2):
-            e2e_step()
+            def copy_in(i):
+                with torch.cuda.stream(s_in):
+                    if i >= 2:
+                        s_in.wait_event(in_free[i - 2])   # step i-2 no longer reads this set
+                    for dst, src in zip(d_in[i % 2], h_in):
+                        dst.copy_(src, non_blocking=True)
+                    in_ready[i].record(s_in)
+
+            copy_in(0)
+            for i in range(steps):
+                if i + 1 < steps:
+                    copy_in(i + 1)
+                stream.wait_event(in_ready[i])
+                if i >= 2:
+                    stream.wait_event(out_free[i - 2])    # step i-2's results have left this set
+                qi, ki, vi, doi = d_in[i % 2]
+                oi, lsei, dqi, dki, dvi = d_out[i % 2]
+                sap.sap_attn_fwd(plan, qi, ki, vi, scale, oi, lsei, ws_f, stream)
+                sap.sap_merge(plan, ws_f, hq, d, oi, lsei, stream)
+                sap.sap_attn_bwd(plan, qi, ki, vi, oi, lsei, doi, scale, dqi, dki, dvi, ws_b, stream)
+                in_free[i].record(stream)
+                out_ready[i].record(stream)
+                with torch.cuda.stream(s_out):
+                    s_out.wait_event(out_ready[i])
+                    for dst, src in zip(h_out, d_out[i % 2]):
+                        dst.copy_(src, non_blocking=True)
+                    out_free[i].record(s_out)
+            stream.wait_stream(s_in)
+            stream.wait_stream(s_out)
+            if end_ev is not None:
+                end_ev.record(stream)
+
+        e2e_run(2)
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
         s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        s2.record(stream)
-        for _ in range(args.steps):
-            e2e_step()
-        e2.record(stream)
+        e2e_run(args.steps, s2, e2)
         torch.cuda.synchronize()
         e2e_ms = max_over_ranks(s2.elapsed_time(e2), dist if world > 1 else None, dev)
+        status = sap.sap_device_status()
+        if status != 0:
+            raise RuntimeError(f"device error word {status} after the end-to-end steps")
+        if not torch.equal(h_out[0], o.cpu()):  # the forward is deterministic; the gradients' fp32 sums are not
+            raise RuntimeError("end-to-end O differs from the device-resident run on the same inputs")
         e2e = {"value": round(job_throughput(f_step, args.steps, world, e2e_ms), 2), "unit": "TFLOP/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": round(e2e_ms / args.steps, 3),
-               "tokens_per_s": round(world * n * args.steps / (e2e_ms / 1e3), 1)}
+               "tokens_per_s": round(world * n * args.steps / (e2e_ms / 1e3), 1),
+               "overlap": "double-buffered: step s+1's inputs in and step s's results out on two copy "
+                          "streams while step s+1 computes"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
