@@ -10,7 +10,7 @@ The five named workloads follow the configurations of the SAP/HSAP setting
 tiny MHA case, and the attention shapes of Llama-3.2-1B, Llama-3.1-8B, a
 512K hybrid-context batch and Llama-2-13B with many short documents.
 
-Recipe (also listed in the design doc):
+Recipe:
   * doc lengths come from ``numpy.random.default_rng(seed)``;
   * log-uniform L = floor(exp(U(ln lo, ln hi))) clamped to [lo, hi]; docs are
     appended until their sum reaches N and the last one is truncated to fit;
