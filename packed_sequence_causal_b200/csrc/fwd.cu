@@ -599,13 +599,24 @@ __global__ void __launch_bounds__(320, 1)
         }
         const float base = (m == -INFINITY) ? 0.f : m;
         float rs4[4] = {0.f, 0.f, 0.f, 0.f};  // row sum as 4 independent chains
+        // The exponentials re-read S from TMEM 64 columns at a time: sv is dead after the row max,
+        // which keeps the softmax warps inside the 168 registers that 10 warps per CTA allow.
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           uint32_t pk[32];
+          float sh[64];
+          tmem_ld32(lane_base + colS + 64 * half, sh);
+          tmem_ld32(lane_base + colS + 64 * half + 32, sh + 32);
+          if (tag != 0) {
+            const int c_lo = row_lo - kt * 128 - 64 * half, c_hi = row_hi - kt * 128 - 64 * half;
+#pragma unroll
+            for (int c = 0; c < 64; ++c)
+              if (c < c_lo || c > c_hi) sh[c] = -INFINITY;
+          }
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
-            const float p0 = ex2(fmaf(sv[64 * half + 2 * e], sl2, -base));
-            const float p1 = ex2(fmaf(sv[64 * half + 2 * e + 1], sl2, -base));
+            const float p0 = ex2(fmaf(sh[2 * e], sl2, -base));
+            const float p1 = ex2(fmaf(sh[2 * e + 1], sl2, -base));
             rs4[e & 3] += p0 + p1;
             pk[e] = pack_bf16x2(p0, p1);
           }

@@ -167,6 +167,15 @@ def test_long_document_elementwise():
 
 
 @pytest.mark.parametrize("d", [64, 128])
+def test_documents_across_backward_bands(d):
+    """Backward units cover one band of 16 q tiles (2048 tokens) of a kv tile's
+    list, so a kv tile of a long document sums dK/dV over several units.  Here
+    documents start and end inside bands and span up to four of them (N = 10240,
+    GQA 2, P = 5): every element against the full oracle."""
+    _fwd_bwd_full([5000, 1100, 3, 2900, 1237], 4, 2, d, 5, seed=22)
+
+
+@pytest.mark.parametrize("d", [64, 128])
 def test_fused_merge_mode(d):
     """Fused-merge schedule (one pass over all kv chunks of a q-tile): same result as the oracle,
     and within rounding of the chunked path."""
