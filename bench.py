@@ -476,7 +476,7 @@ def main():
                            "fwd_tflops": round(f_fwd / (t_fwd / 1e3) / 1e12, 1),
                            "bwd_tflops": round(f_bwd / (t_bwd / 1e3) / 1e12, 1),
                            "plan_host_ms": round(1e3 * t_plan, 2)},
-            "roofline": {"bound": "tensor", "kernel": "sap_attn_bwd (bwd_pre + sap_bwd_kernel + dq_post)",
+            "roofline": {"bound": "tensor", "kernel": "sap_attn_bwd (bwd_pre + sap_bwd_kernel + bwd_post)",
                          "achieved": round(achieved, 1), "peak": sustained, "unit": "TFLOP/s",
                          "frac": round(achieved / sustained, 4), "frac_of_burst_peak": round(achieved / burst, 4),
                          "traffic": None if args.tokens else measured_traffic(w.name),
