@@ -81,8 +81,9 @@ typedef struct {
  * chunking, lists the non-empty tiles in canonical order (q-tile ascending,
  * then kv-tile ascending; bit-exact with the tile-list definition above), and
  * derives the work schedule: forward units = (q-tile, kv-chunk) groups of
- * items, partial slots for q-tiles that see more than one kv-chunk, the
- * per-kv-tile lists for the backward pass, and heavy-first launch orders.
+ * items, partial slots for q-tiles that see more than one kv-chunk and a
+ * heavy-first launch order; backward units = per-kv-tile q lists cut into bands
+ * of 16 q tiles, in band-major order (sap_plan_bwd_schedule).
  * P = num_chunks; with P = 1 any N >= 0 is accepted (a partial last tile is
  * masked).  On success *out owns the plan. */
 int sap_plan(const int32_t* cu_seqlens_host, int32_t num_docs, int64_t total_tokens, int32_t num_chunks,

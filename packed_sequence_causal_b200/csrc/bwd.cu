@@ -1,9 +1,10 @@
-// Backward kernel: dK, dV (and dQ by fp32 reduction) for one kv tile and one
-// kv head per work item, looping over the q heads of its GQA group and the
-// q tiles that attend to the kv tile (the per-kv-tile lists of the planner).
+// Backward kernel: dK, dV (and dQ by fp32 reduction) for one backward unit and one
+// kv head per work item.  A unit is the part of one kv tile's q-tile list (the
+// planner's per-kv-tile lists) that falls in one band of 16 q tiles; the work
+// item loops over those q tiles and the q heads of the kv head's GQA group.
 // With the final, merged LSE every (q-tile, kv-tile) pair is normalised
-// already, so the pairs of different chunks are independent and their
-// gradients simply add.
+// already, so the pairs of different chunks (and of different bands) are
+// independent and their gradients simply add.
 //
 // Persistent CTA, warp-specialised (448 threads), transposed so that a TMEM
 // lane is a key/value row:
@@ -17,17 +18,21 @@
 //                  S^T_{j+1}          (issued here: R1 is free once dV_j has read P^T_j)
 //                  dK    += dS^T_j Q_j  (A = dS^T from shared memory) -> dK
 //                  dQ_j               (D=128: dQ^T = K^T dS^T -> R2; D=64: dQ = dS K -> DQ)
+//                and releases the Q/dO ring slot once dK_j and dQ_j have read it.
 //   warps 2..9   two warpgroups, one per half of the 128 q columns; thread t
 //                owns kv row j = kt*128 + t.  P^T = exp2(S^T c - LSE2_i) on the
 //                pairs of its document with i >= j (all pairs for FULL tiles),
 //                written back to TMEM as packed bf16 over its own S columns;
 //                dS^T = P^T (dP^T - D_i) (the softmax scale is applied to dK and dQ
-//                as they are drained) written to a 128-byte swizzled
-//                shared tile as bf16 (read as a K-major operand by dK and as an
-//                MN-major operand by dQ).
-//   warps 10..13 drain dQ from TMEM into the fp32 accumulator (global
-//                reductions, one 128-byte row per warp instruction for D=128),
-//                and write dK, dV (bf16) at the end of a work item.
+//                as they are drained) written to a 128-byte swizzled shared tile
+//                as bf16 (read as a K-major operand by dK and as an MN-major
+//                operand by dQ): for D = 128 over the ring slot's dO tile once dV_j
+//                has read it, for D = 64 into a buffer of its own.
+//   warps 10..13 drain dQ from TMEM into the fp32 accumulator (D = 128: staged
+//                64 q rows at a time in a dedicated buffer and added by TMA bulk
+//                reductions; D = 64: vector global reductions), and at the end of
+//                a work item add its dK and dV into fp32 accumulators the same way
+//                (the conversion to bf16 is a separate elementwise kernel).
 //
 // TMEM columns: dK [0,D), dV [D,2D), R1 = S^T/P^T [2D, 2D+128),
 // R2 = dP^T [2D+128, 2D+256); dQ shares R2 for D = 128 (dP^T is consumed
