@@ -286,6 +286,12 @@ def main():
     pairs = stats["unmasked_pairs"]
     n_items = len(sap.sap_plan_items(plan))
     _, _, merges = sap.sap_plan_fwd_schedule(plan)
+    # merge kernel: algorithmic bytes per call = per (row, head) of a merged q tile, its k fp32
+    # partials (O and LSE) read and bf16 O + fp32 LSE written
+    merge_bytes = 0
+    for qt, _, k in np.asarray(merges).reshape(-1, 3).tolist():
+        rows = min(128, n - qt * 128)
+        merge_bytes += rows * hq * (k * (4 * d + 4) + 2 * d + 4)
     q, k, v, do = b.q, b.k, b.v, b.do
     o = torch.empty_like(q)
     lse = torch.empty((hq, n), dtype=torch.float32, device=dev)
@@ -472,6 +478,10 @@ def main():
             "pct_bf16_peak": round(100 * value / world / burst, 2),
             "pct_bf16_peak_sustained": round(100 * value / world / sustained, 2),
             "peak_source": peak_src,
+            "hbm": {"merge_kernel": {"bytes": int(merge_bytes), "ms": round(t_merge, 3),
+                                     "gbs": round(merge_bytes / (t_merge / 1e3) / 1e9, 1) if t_merge > 0 else None,
+                                     "frac_of_measured": round(merge_bytes / (t_merge / 1e3) / 1e9 / hbm, 3)
+                                     if t_merge > 0 else None, "peak_gbs": hbm}},
             "kernels_ms": {"fwd": round(t_fwd, 3), "merge": round(t_merge, 3), "bwd": round(t_bwd, 3),
                            "fwd_tflops": round(f_fwd / (t_fwd / 1e3) / 1e12, 1),
                            "bwd_tflops": round(f_bwd / (t_bwd / 1e3) / 1e12, 1),
