@@ -350,7 +350,10 @@ __global__ void __launch_bounds__(192, 1)
 // share every K/V load.  P is written back into TMEM (packed bf16 over the S
 // columns) and read from there by the PV MMA, and the MMA thread interleaves
 // the tiles -- S0, S1, PV0, S0', PV1, S1', ... -- so that while one softmax
-// warpgroup exponentiates its tile the tensor core works on the other.
+// warpgroup exponentiates its tile the tensor core works on the other.  Each PV
+// is issued in two halves (kv rows 0..63, then 64..127): the softmax signals
+// p_half once the first half of P is in TMEM, so the first half of PV runs while
+// the second half of P is being computed.
 //
 // Threads: warp 0 TMA, warp 1 MMA, warps 2..5 softmax of tile 0 (head 2p),
 // warps 6..9 softmax of tile 1 (head 2p+1).
@@ -366,7 +369,7 @@ struct Fwd2Cfg {
   static constexpr int OFF_K = 2 * QBYTES;
   static constexpr int OFF_V = OFF_K + NS * KVBYTES;
   static constexpr int OFF_BAR = OFF_V + NS * KVBYTES;
-  static constexpr int NBAR = 2 + 4 * NS + 2 + 2 + 2;
+  static constexpr int NBAR = 2 + 4 * NS + 2 + 2 + 2 + 2;
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16;
   static constexpr int THREADS = 320;
   static constexpr uint32_t COL_O = 256;
@@ -391,7 +394,8 @@ __global__ void __launch_bounds__(320, 1)
   uint64_t* v_empty = v_full + C::NS;
   uint64_t* s_full = v_empty + C::NS;  // [2], one per tile
   uint64_t* p_full = s_full + 2;       // [2]
-  uint64_t* o_done = p_full + 2;
+  uint64_t* p_half = p_full + 2;       // [2] first half of P (kv rows 0..63) is in TMEM
+  uint64_t* o_done = p_half + 2;
   uint64_t* mma_drain = o_done + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBAR);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -411,6 +415,7 @@ __global__ void __launch_bounds__(320, 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(s_full + b, 1);
       mbar_init(p_full + b, 128);
+      mbar_init(p_half + b, 128);
     }
     mbar_init(o_done, 1);
     mbar_init(mma_drain, 1);
@@ -490,10 +495,10 @@ __global__ void __launch_bounds__(320, 1)
         }
         tc_commit(s_full + tile);
       };
-      auto issue_pv = [&](int tile, uint32_t it, bool first) {  // O_tile += P_tile V_it, P from TMEM
+      auto issue_pv = [&](int tile, uint32_t it, bool first, int part) {  // O_tile += P_tile V_it (half), P from TMEM
         const int s = it % C::NS;
 #pragma unroll
-        for (int kk = 0; kk < 128 / 16; ++kk)
+        for (int kk = 4 * part; kk < 4 * part + 4; ++kk)
           mma_bf16_tmem_a(tmem + C::COL_O + D * tile, tmem + 128 * tile + kk * 8,
                           sdesc_sw128(sV + s * C::KVBYTES + kk * 2048, C::BOX, 1024), idesc_pv,
                           (first && kk == 0) ? 0u : 1u);
@@ -510,9 +515,12 @@ __global__ void __launch_bounds__(320, 1)
         for (int j = 0; j < ic; ++j, ++tile_iter) {
           const uint32_t it = kv_iter + j;
           if (!mbar_wait(v_full + it % C::NS, (it / C::NS) & 1, guard, kErrTimeoutMma)) { ok = false; break; }
+          if (!mbar_wait(p_half + 0, tile_iter & 1, guard, kErrTimeoutMma)) { ok = false; break; }
+          tc_fence_after();
+          issue_pv(0, it, j == 0, 0);
           if (!mbar_wait(p_full + 0, tile_iter & 1, guard, kErrTimeoutMma)) { ok = false; break; }
           tc_fence_after();
-          issue_pv(0, it, j == 0);
+          issue_pv(0, it, j == 0, 1);
           const bool more = j + 1 < ic;
           if (more) {
             if (!mbar_wait(k_full + (it + 1) % C::NS, ((it + 1) / C::NS) & 1, guard, kErrTimeoutMma)) {
@@ -522,9 +530,12 @@ __global__ void __launch_bounds__(320, 1)
             tc_fence_after();
             issue_s(0, it + 1);  // rewrites S0/P0 only after PV0 (issued above) has read P0
           }
+          if (!mbar_wait(p_half + 1, tile_iter & 1, guard, kErrTimeoutMma)) { ok = false; break; }
+          tc_fence_after();
+          issue_pv(1, it, j == 0, 0);
           if (!mbar_wait(p_full + 1, tile_iter & 1, guard, kErrTimeoutMma)) { ok = false; break; }
           tc_fence_after();
-          issue_pv(1, it, j == 0);
+          issue_pv(1, it, j == 0, 1);
           tc_commit(v_empty + it % C::NS);
           if (more) {
             issue_s(1, it + 1);
@@ -621,6 +632,10 @@ __global__ void __launch_bounds__(320, 1)
             pk[e] = pack_bf16x2(p0, p1);
           }
           tmem_st32_u(lane_base + colS + 32 * half, pk);  // P over the S columns already read
+          if (half == 0) {  // PV over kv rows 0..63 may start while the second half is computed
+            tc_fence_before();
+            mbar_arrive(p_half + tile);
+          }
         }
         l += (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
         tc_fence_before();
@@ -665,7 +680,7 @@ __global__ void __launch_bounds__(320, 1)
         }
         p.lse_part[((size_t)slot * p.hq + h) * 128 + r] = lse_val;
       }
-      // The next unit's first PV into O waits for this warpgroup's next p_full.
+      // The next unit's first PV into O waits for this warpgroup's next p_half and p_full.
       tc_fence_before();
     }
   }
