@@ -11,14 +11,18 @@
 //   warp 0       TMA producer: K, V per work item; per iteration Q, dO and the
 //                128 LSE*log2(e) and D values of the q tile, through an
 //                NSQ-stage ring.
-//   warp 1       TMEM owner and tcgen05.mma issuer (one thread), per iteration j
-//                  S^T_j  = K Q_j^T   (M=128 kv, N=128 q, K=D)        -> R1
-//                  dP^T_j = V dO_j^T  (M=128 kv, N=128 q, K=D)        -> R2
+//   warp 1       TMEM owner and tcgen05.mma issuer (one thread); S^T_j = K Q_j^T
+//                (M=128 kv, N=128 q, K=D) -> R1 is issued one iteration ahead, then
+//                per iteration j
 //                  dV    += P^T_j dO_j  (A = P^T from TMEM R1)         -> dV
-//                  S^T_{j+1}          (issued here: R1 is free once dV_j has read P^T_j)
-//                  dK    += dS^T_j Q_j  (A = dS^T from shared memory) -> dK
+//                  dP^T_j = V dO_j^T  (M=128 kv, N=128 q, K=D)        -> R2
+//                  S^T_{j+1}          (R1 is free once dV_j has read P^T_j)
 //                  dQ_j               (D=128: dQ^T = K^T dS^T -> R2; D=64: dQ = dS K -> DQ)
-//                and releases the Q/dO ring slot once dK_j and dQ_j have read it.
+//                  dK    += dS^T_j Q_j  (A = dS^T from shared memory) -> dK
+//                dV goes first because P^T_j is ready long before the previous dQ^T
+//                has left R2 (which dP^T_j needs at D = 128), and dQ before dK so
+//                that its drain overlaps dK; the Q/dO ring slot is released once dK_j
+//                and dQ_j have read it.
 //   warps 2..9   two warpgroups, one per half of the 128 q columns; thread t
 //                owns kv row j = kt*128 + t.  P^T = exp2(S^T c - LSE2_i) on the
 //                pairs of its document with i >= j (all pairs for FULL tiles),
@@ -226,16 +230,8 @@ __global__ void __launch_bounds__(448, 1)
         if (!issue_s(it)) break;
         for (int j = 0; j < n_it; ++j, ++it) {
           const uint32_t sQ = stage_q(it), sDO = sQ + C::TILE;
-          // dP^T_j -> R2 once the previous dQ (D = 128: same columns) has been drained
-          if (C::DQ_T && it > 0 && !mbar_wait(dq_free, (it - 1) & 1, guard, kErrTimeoutMma)) { ok = false; break; }
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t ko = (kk / 4) * C::BOX + (kk % 4) * 32;
-            mma_bf16(R2, sdesc_sw128(sV + ko, 16, 1024), sdesc_sw128(sDO + ko, 16, 1024), id_sq, kk > 0);
-          }
-          tc_commit(dp_full);
-          // dV += P^T_j dO_j, P^T in TMEM (packed bf16 over the S^T columns of each half)
+          // dV += P^T_j dO_j first (P^T in TMEM, packed bf16 over the S^T columns of each half):
+          // P^T_j is usually ready well before the previous dQ has been drained.
           if (!mbar_wait(p_ready, it & 1, guard, kErrTimeoutMma)) { ok = false; break; }
           if (j == 0 && unit_iter > 0 && !mbar_wait(dkdv_free, (unit_iter - 1) & 1, guard, kErrTimeoutMma)) {
             ok = false;
@@ -247,18 +243,21 @@ __global__ void __launch_bounds__(448, 1)
             mma_bf16_tmem_a(tmem + C::COL_DV, R1 + (kk / 4) * 64 + (kk % 4) * 8,
                             sdesc_sw128(sDO + kk * 2048, C::BOX, 1024), id_kv, (j > 0 || kk > 0) ? 1u : 0u);
           if (C::DQ_T) tc_commit(dv_done);
+          // dP^T_j -> R2 once the previous dQ (D = 128: same columns) has been drained
+          if (C::DQ_T && it > 0 && !mbar_wait(dq_free, (it - 1) & 1, guard, kErrTimeoutMma)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t ko = (kk / 4) * C::BOX + (kk % 4) * 32;
+            mma_bf16(R2, sdesc_sw128(sV + ko, 16, 1024), sdesc_sw128(sDO + ko, 16, 1024), id_sq, kk > 0);
+          }
+          tc_commit(dp_full);
           const uint32_t sDSj = C::DQ_T ? sDO : sDS;  // d = 128: dS^T_j over dO_j
           // S^T_{j+1}: R1 is rewritten only after dV_j (issued above) has read P^T_j
           if (j + 1 < n_it && !issue_s(it + 1)) { ok = false; break; }
-          // dK += dS^T_j Q_j ; dQ_j
+          // dQ_j and dK += dS^T_j Q_j
           if (!mbar_wait(ds_ready, it & 1, guard, kErrTimeoutMma)) { ok = false; break; }
           tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < 128 / 16; ++kk) {
-            const uint64_t a = sdesc_sw128(sDSj + (kk / 4) * C::BOX + (kk % 4) * 32, 16, 1024);
-            mma_bf16(tmem + C::COL_DK, a, sdesc_sw128(sQ + kk * 2048, C::BOX, 1024), id_kv,
-                     (j > 0 || kk > 0) ? 1u : 0u);
-          }
           if (!C::DQ_T && it > 0 && !mbar_wait(dq_free, (it - 1) & 1, guard, kErrTimeoutMma)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll
@@ -270,6 +269,12 @@ __global__ void __launch_bounds__(448, 1)
             mma_bf16(tmem + C::COL_DQ, C::DQ_T ? kd : sd, C::DQ_T ? sd : kd, id_dq, kk > 0);
           }
           tc_commit(dq_full);
+#pragma unroll
+          for (int kk = 0; kk < 128 / 16; ++kk) {
+            const uint64_t a = sdesc_sw128(sDSj + (kk / 4) * C::BOX + (kk % 4) * 32, 16, 1024);
+            mma_bf16(tmem + C::COL_DK, a, sdesc_sw128(sQ + kk * 2048, C::BOX, 1024), id_kv,
+                     (j > 0 || kk > 0) ? 1u : 0u);
+          }
           if (!C::DQ_T) tc_commit(ds_free);
           tc_commit(q_empty + it % C::NSQ);
         }
