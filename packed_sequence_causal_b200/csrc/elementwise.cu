@@ -78,12 +78,26 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
     float sum = 0.f;
     for (int b = 0; b < ns; ++b) sum += __expf(lse_part[((size_t)(s0 + b) * hq + h) * 128 + r] - mx);
     lse_all = mx + __logf(sum);
-    for (int b = 0; b < ns; ++b) {
-      const float wgt = __expf(lse_part[((size_t)(s0 + b) * hq + h) * 128 + r] - lse_all);
-      float v[E];
-      Vec<E>::load(o_part + (((size_t)(s0 + b) * hq + h) * 128 + r) * D + lane * E, v);
+    // up to four partials' rows are loaded before they are accumulated (in order), so that
+    // several 4*D-byte loads per warp are in flight
+    for (int b0 = 0; b0 < ns; b0 += 4) {
+      float v[4][E], wgt[4];
 #pragma unroll
-      for (int e = 0; e < E; ++e) acc[e] = fmaf(wgt, v[e], acc[e]);
+      for (int u = 0; u < 4; ++u) {
+        if (b0 + u < ns) {
+          const size_t row = ((size_t)(s0 + b0 + u) * hq + h) * 128 + r;
+          wgt[u] = lse_part[row];
+          Vec<E>::load(o_part + row * D + lane * E, v[u]);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (b0 + u < ns) {
+          const float w = __expf(wgt[u] - lse_all);
+#pragma unroll
+          for (int e = 0; e < E; ++e) acc[e] = fmaf(w, v[u][e], acc[e]);
+        }
+      }
     }
   }
   Vec<E>::store_bf16(o + ((size_t)i * hq + h) * D + lane * E, acc);
