@@ -420,7 +420,10 @@ int sap_attn_bwd(sap_plan_t p, const void* q, const void* k, const void* v, cons
   float* dq_acc = reinterpret_cast<float*>(wsb + ws.dq_acc);
   float* dkv_acc = reinterpret_cast<float*>(wsb + ws.dkv_acc);
   CUtensorMap tdq, tdkv;
-  if ((rc = make_map_f32_tile(&tdq, dq_acc, ws.n_pad, hq, head_dim))) return rc;
+  // d = 128 stages dQ^T as 64-row [q][d] tiles; d = 64 stages dQ rows as 128-byte-swizzled boxes
+  if ((rc = head_dim == 128 ? make_map_f32_tile(&tdq, dq_acc, ws.n_pad, hq, head_dim)
+                            : make_map_f32_sw128(&tdq, dq_acc, ws.n_pad, hq, head_dim)))
+    return rc;
   if ((rc = make_map_f32_sw128(&tdkv, dkv_acc, 2 * ws.n_pad, hkv, head_dim))) return rc;
   float* dvec = reinterpret_cast<float*>(wsb + ws.dvec);
   float* lse2 = reinterpret_cast<float*>(wsb + ws.lse2);

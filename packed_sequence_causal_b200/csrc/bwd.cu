@@ -449,21 +449,38 @@ __global__ void __launch_bounds__(448, 1)
             ++hs;
             continue;
           } else {
-            // lane t = q row t of the tile
-            float* dst = p.dq_acc + (((size_t)qt * 128 + t) * p.hq + h) * D;
-#pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
-              float v[32];
-              tmem_ld32(lane_base + C::COL_DQ + 32 * c, v);
+            // Lane t holds q row t of dQ (D = 64 features).  The tile is staged, times the softmax
+            // scale, as two 128-byte-swizzled boxes [128 rows][32 fp32] in the epilogue buffer (the
+            // same layout and barriers as the dK/dV epilogue) and added by two TMA bulk reductions.
+            uint8_t* epi = smem + C::OFF_EPI;
+            if (hs > 0 && !mbar_wait_warp(stg_free, (hs - 1) & 1, guard, kErrTimeoutEpilogue)) { ok = false; break; }
+            float v0[32], v1[32];
+            tmem_ld32(lane_base + C::COL_DQ, v0);
+            tmem_ld32(lane_base + C::COL_DQ + 32, v1);
+            tc_fence_before();
+            mbar_arrive(dq_free);  // all of dQ is in registers: the next dQ may overwrite its columns
 #pragma unroll
-              for (int e4 = 0; e4 < 32; e4 += 4)
-                atomicAdd(reinterpret_cast<float4*>(dst + 32 * c + e4),
-                          make_float4(v[e4] * p.scale, v[e4 + 1] * p.scale, v[e4 + 2] * p.scale,
-                                      v[e4 + 3] * p.scale));
+            for (int c16 = 0; c16 < 8; ++c16) {
+              const uint32_t off = sw128_offset(t, c16);
+              st_shared_v4(smem_u32(epi + off), __float_as_uint(v0[4 * c16] * p.scale),
+                           __float_as_uint(v0[4 * c16 + 1] * p.scale), __float_as_uint(v0[4 * c16 + 2] * p.scale),
+                           __float_as_uint(v0[4 * c16 + 3] * p.scale));
+              st_shared_v4(smem_u32(epi + C::EPI_BYTES / 2 + off), __float_as_uint(v1[4 * c16] * p.scale),
+                           __float_as_uint(v1[4 * c16 + 1] * p.scale), __float_as_uint(v1[4 * c16 + 2] * p.scale),
+                           __float_as_uint(v1[4 * c16 + 3] * p.scale));
             }
+            fence_async_smem();
+            mbar_arrive(stg_ready);
+            if (!mbar_wait_warp(stg_ready, hs & 1, guard, kErrTimeoutEpilogue)) { ok = false; break; }
+            if (t == 0) {
+              tma_reduce_add_3d(&tmDQ, epi, 0, h, qt * 128);
+              tma_reduce_add_3d(&tmDQ, epi + C::EPI_BYTES / 2, 32, h, qt * 128);
+              bulk_commit_group();
+              bulk_wait_group_read0();
+              mbar_arrive(stg_free);
+            }
+            ++hs;
           }
-          tc_fence_before();
-          mbar_arrive(dq_free);
         }
       }
       if (!ok) break;
