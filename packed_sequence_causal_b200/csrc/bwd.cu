@@ -64,7 +64,8 @@ struct BwdCfg {
   static constexpr int OFF_DS = OFF_V + TILE;
   static constexpr int OFF_ST = OFF_DS + 128 * 128 * 2;  // stages: Q, dO, lse2, dvec
   // dK/dV epilogue staging (128 rows x 64 fp32 as two 128-byte-swizzled boxes of 32 features):
-  // d = 128 shares the dQ staging buffer (same warps, same barriers); d = 64 has its own.
+  // d = 128 shares the dQ staging buffer; d = 64 has its own, which also stages dQ (d = 64 dQ is
+  // [q][d] in TMEM, the same row-per-lane shape).  Same warps and barriers in both cases.
   static constexpr int EPI_BYTES = 128 * 64 * 4;
   static constexpr int OFF_EPI = (D == 128) ? OFF_DS : OFF_ST + NSQ * STAGE;
   static constexpr int OFF_BAR = (D == 128) ? OFF_ST + NSQ * STAGE : OFF_EPI + EPI_BYTES;
