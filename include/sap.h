@@ -100,7 +100,8 @@ int sap_plan_stats(sap_plan_t plan, int64_t* unmasked_pairs, int64_t* n_partial_
 /* Forward schedule, host memory owned by the plan:
  *   units: int32[n_units][4] = (q_tile, item_begin, item_count, slot), slot = -1
  *          when the unit writes O/LSE directly, else its partial slot;
- *   order: int32[n_units], heavy-first (item_count descending, ties by index);
+ *   order: int32[n_units], heavy-first (item_count descending; ties by the kv chunk
+ *          of the unit's items, then by index, so that concurrent units share K/V tiles);
  *   merges: int32[n_merges][3] = (q_tile, first_slot, n_slots). */
 int sap_plan_fwd_schedule(sap_plan_t plan, const int32_t** units, int64_t* n_units, const int32_t** order,
                           const int32_t** merges, int64_t* n_merges);

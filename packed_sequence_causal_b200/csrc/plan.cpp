@@ -57,8 +57,13 @@ void sap_plan_build_fwd_schedule(sap_plan_s* p, bool fused) {
   const size_t nu = p->fwd_units.size() / 4;
   p->fwd_order.resize(nu);
   std::iota(p->fwd_order.begin(), p->fwd_order.end(), 0);
-  std::stable_sort(p->fwd_order.begin(), p->fwd_order.end(),
-                   [&](int32_t x, int32_t y) { return p->fwd_units[4 * x + 2] > p->fwd_units[4 * y + 2]; });
+  // heavy-first; among units of equal size, kv chunk first, so that the CTAs running at the same
+  // time stream the K/V tiles of one kv chunk (which then stay in L2) rather than of several
+  auto chunk_of = [&](int32_t u) { return p->items[p->fwd_units[4 * u + 1]].kv_chunk; };
+  std::stable_sort(p->fwd_order.begin(), p->fwd_order.end(), [&](int32_t x, int32_t y) {
+    const int32_t cx = p->fwd_units[4 * x + 2], cy = p->fwd_units[4 * y + 2];
+    return cx != cy ? cx > cy : chunk_of(x) < chunk_of(y);
+  });
 }
 
 int sap_plan_build(const int32_t* cu, int32_t num_docs, int64_t n, int32_t num_chunks, int32_t block_m,

@@ -46,13 +46,15 @@ def _check_schedules(plan, items, n, nchunks, bm, bn):
             mi += 1
     assert mi == len(merges)
     assert sap.sap_plan_stats(plan)["n_partial_slots"] == next_slot
-    # heavy-first order: a permutation, non-increasing item counts, stable on ties
+    # heavy-first order: a permutation, non-increasing item counts; among equal counts the kv chunk
+    # of the unit's items ascending, then the unit index
     assert sorted(order.tolist()) == list(range(len(units)))
     counts = units[order, 2]
     assert np.all(np.diff(counts) <= 0)
+    chunk = {u: items[units[u, 1]][3] for u in range(len(units))}
     for a, b in zip(order[:-1], order[1:]):
         if units[a, 2] == units[b, 2]:
-            assert a < b
+            assert (chunk[a], a) < (chunk[b], b)
     # backward: every item once; each unit is the part of one kv tile's q-descending list that
     # falls in one band of 16 q tiles; units band-major (top band first), heavy-first within a
     # band, ties by kv tile
