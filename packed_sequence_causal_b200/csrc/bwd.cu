@@ -108,8 +108,8 @@ __global__ void __launch_bounds__(448, 1)
   uint64_t* dkdv_full = dq_free + 1;
   uint64_t* dkdv_free = dkdv_full + 1;
   uint64_t* mma_drain = dkdv_free + 1;
-  uint64_t* stg_ready = mma_drain + 1;  // half dQ tile staged in shared memory (d = 128)
-  uint64_t* stg_free = stg_ready + 1;   // its reduction has read the staging buffer (d = 128)
+  uint64_t* stg_ready = mma_drain + 1;  // the staging buffer holds a dQ or dK/dV piece
+  uint64_t* stg_free = stg_ready + 1;   // its reduction has read the staging buffer
   uint64_t* dv_done = stg_free + 1;     // dV has read dO: dS^T may go over it (d = 128)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBAR);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
