@@ -1,8 +1,8 @@
 """ctypes front end of the fp64 CPU oracle (``oracle.c``).
 
 TEST INFRASTRUCTURE ONLY.  The tests, the smoke check and the benchmark's
-CPU-baseline leg use it; the CUDA library never imports it, and it imports
-nothing from the CUDA side.  Inputs are widened exactly from bf16 to float64.
+CPU-baseline leg and reference arm use it; the CUDA library never imports it,
+and it imports nothing from the CUDA side.  Inputs are widened exactly from bf16 to float64.
 """
 from __future__ import annotations
 

@@ -1,8 +1,8 @@
 /*
  * oracle.c -- plain, slow, fp64 CPU oracle for packed causal attention with
  * sequence-aware chunking.  TEST INFRASTRUCTURE ONLY: the tests, the smoke
- * check and the CPU-baseline leg of the benchmark call it; the CUDA library
- * never does, and the two share no code.
+ * check and the benchmark's CPU-baseline leg and reference arm call it; the
+ * CUDA library never does, and the two share no code.
  *
  * What it computes (SAP/HSAP page, abstract: packing documents into one
  * sequence must not let attention cross documents; "partial attention
