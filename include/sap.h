@@ -27,8 +27,10 @@
  *
  * Ownership: the caller owns every device buffer (inputs, outputs and the
  * workspace).  The library owns only a plan: its host arrays and their device
- * copy, released by sap_plan_destroy.  Device pointers must be 16-byte
- * aligned.
+ * copy, released by sap_plan_destroy.  One exception: the library keeps a
+ * 16 MiB device array of its own on every device that loads it, the scratch
+ * of sap_attn_fwd_static_scratch (see that declaration).  Device pointers,
+ * workspaces included, must be 16-byte aligned.
  *
  * Streams: every device call is asynchronous on the given cudaStream_t
  * (passed as void*, NULL = the legacy default stream).
@@ -68,10 +70,13 @@ enum { SAP_WS_FWD = 0, SAP_WS_BWD = 1 };
 typedef struct sap_plan_s* sap_plan_t;
 
 /* One non-empty (q-tile, kv-tile) pair of the packed causal mask.
- *   tag FULL   : no pair of the block_m x block_n box is masked;
- *   tag CAUSAL : the diagonal box (same token range) inside one document;
- *   tag MASKED : anything else (document boundaries inside the box, or a
- *                partial last tile).
+ *   tag FULL   : no pair of the block_m x block_n box is masked (never a partial
+ *                last tile: its missing rows count as masked);
+ *   tag CAUSAL : a diagonal box (same token range) whose real rows all lie in one
+ *                document, a partial last tile included; inside it the mask is
+ *                exactly j <= i;
+ *   tag MASKED : anything else (a document boundary inside the box, or an
+ *                off-diagonal box of a partial last tile).
  * q_chunk = q_tile*block_m / C and kv_chunk = kv_tile*block_n / C, C = N / P. */
 typedef struct {
   int32_t q_tile, kv_tile, q_chunk, kv_chunk, tag;

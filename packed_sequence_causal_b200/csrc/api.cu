@@ -333,7 +333,8 @@ int sap_attn_fwd(sap_plan_t p, const void* q, const void* k, const void* v, int3
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
     return SAP_ERR_INVALID_ARG;
   const FwdWs ws = fwd_ws(p, hq, head_dim);
-  if (ws.total > 0 && p->n_slots > 0 && (!workspace || ws_bytes < ws.total)) return SAP_ERR_WORKSPACE;
+  if (ws.total > 0 && p->n_slots > 0 && (!workspace || ws_bytes < ws.total || !aligned16(workspace)))
+    return SAP_ERR_WORKSPACE;
   DeviceInfo* di = nullptr;
   if ((rc = device_info(&di))) return rc;
   if ((rc = sap_plan_upload(p, stream))) return rc;
@@ -378,7 +379,7 @@ int sap_merge(sap_plan_t p, const void* workspace, size_t ws_bytes, int32_t hq, 
   if (p->n == 0 || n_merges == 0) return SAP_OK;
   if (!o || !lse || !aligned16(o)) return SAP_ERR_INVALID_ARG;
   const FwdWs ws = fwd_ws(p, hq, head_dim);
-  if (!workspace || ws_bytes < ws.total) return SAP_ERR_WORKSPACE;
+  if (!workspace || ws_bytes < ws.total || !aligned16(workspace)) return SAP_ERR_WORKSPACE;
   if ((rc = sap_plan_upload(p, stream))) return rc;
   const int32_t* base = static_cast<const int32_t*>(p->dev);
   const uint8_t* wsb = static_cast<const uint8_t*>(workspace);

@@ -32,11 +32,12 @@
 //                as bf16 (read as a K-major operand by dK and as an MN-major
 //                operand by dQ): for D = 128 over the ring slot's dO tile once dV_j
 //                has read it, for D = 64 into a buffer of its own.
-//   warps 10..13 drain dQ from TMEM into the fp32 accumulator (D = 128: staged
-//                64 q rows at a time in a dedicated buffer and added by TMA bulk
-//                reductions; D = 64: vector global reductions), and at the end of
-//                a work item add its dK and dV into fp32 accumulators the same way
-//                (the conversion to bf16 is a separate elementwise kernel).
+//   warps 10..13 drain dQ from TMEM into the fp32 accumulator by TMA bulk
+//                reductions (D = 128: dQ^T staged 64 q rows at a time in a dedicated
+//                buffer; D = 64: dQ staged as two 128-byte-swizzled boxes of 32
+//                features), and at the end of a work item add its dK and dV into
+//                fp32 accumulators the same way (the conversion to bf16 is a
+//                separate elementwise kernel).
 //
 // TMEM columns: dK [0,D), dV [D,2D), R1 = S^T/P^T [2D, 2D+128),
 // R2 = dP^T [2D+128, 2D+256); dQ shares R2 for D = 128 (dP^T is consumed

@@ -1,7 +1,8 @@
 // Memory-bound kernels of the path: the exact LSE merge of partial outputs,
-// the backward pre-pass (D_i and LSE in the log2 domain, zeroed dQ
-// accumulator) and the fp32 -> bf16 conversion of dQ.  One warp per
-// (row, head) keeps every global access coalesced along the head dimension.
+// the backward pre-pass (D_i and LSE in the log2 domain, zeroed dQ, dK and dV
+// accumulators) and the fp32 -> bf16 conversion of the dQ, dK and dV
+// accumulators.  One warp per (row, head) keeps every global access coalesced
+// along the head dimension.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 

@@ -35,7 +35,7 @@ struct BwdParams {
   float scale;                // softmax_scale
   const float* lse2;          // [hq][n_pad] LSE * log2(e) (+inf past N)
   const float* dvec;          // [hq][n_pad] D_i = <dO_i, O_i> (0 past N)
-  float* dq_acc;              // [n_pad][hq][D] fp32 dQ accumulator (d = 64: atomics; d = 128: the tdq map)
+  float* dq_acc;              // [n_pad][hq][D] fp32 dQ accumulator (reduced into through the tdq map)
   int* err;
 };
 

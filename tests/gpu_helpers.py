@@ -8,10 +8,16 @@ by up to 2^-9 |ref|; 2^-8 leaves room for the fp32 sums), i.e. every element
 satisfies
     |out - ref| <= 2e-2 + 2^-8 |ref|
 and mean |out - ref| <= 2e-3; for LSE, max-abs 1e-3.
+
+Every comparison also records the plain max-abs and mean-abs error (and the
+largest |ref|), so that the distance from the literal max-abs 2e-2 bound is
+visible: tests/conftest.py writes the records to the JSON file named by the
+SAP_PARITY_REPORT environment variable at the end of the session.
 """
 from __future__ import annotations
 
 import math
+import os
 
 import numpy as np
 import torch
@@ -24,27 +30,93 @@ MEAN_ATOL = 2e-3
 LSE_ATOL = 1e-3
 BF16_HALF_ULP = 2.0 ** -8
 
+# one record per comparison: test id, tensor, plain max-abs / mean-abs error, max |ref|, elements
+PARITY_RECORDS: list = []
 
-def assert_close(out, ref, what: str):
-    out = out.detach().double().cpu().numpy() if hasattr(out, "detach") else np.asarray(out, dtype=np.float64)
+
+def _record(what: str, err: np.ndarray, ref: np.ndarray, **extra):
+    rec = {"test": os.environ.get("PYTEST_CURRENT_TEST", "").split(" ")[0], "what": what,
+           "max_abs": float(err.max()) if err.size else 0.0, "mean_abs": float(err.mean()) if err.size else 0.0,
+           "max_ref": float(np.abs(ref).max()) if ref.size else 0.0, "elements": int(err.size)}
+    rec.update(extra)
+    PARITY_RECORDS.append(rec)
+
+
+def _as_f64(out):
+    return out.detach().double().cpu().numpy() if hasattr(out, "detach") else np.asarray(out, dtype=np.float64)
+
+
+def assert_close(out, ref, what: str, extra_bound=None, mean_extra: float = 0.0):
+    """Element bound |out - ref| <= 2e-2 + 2^-8 |ref| (+ extra_bound, an array of the same shape, where a
+    test states a larger, derived rounding term) and mean |out - ref| <= 2e-3 (+ mean_extra)."""
+    out = _as_f64(out)
     ref = np.asarray(ref, dtype=np.float64)
     assert out.shape == ref.shape, (what, out.shape, ref.shape)
     assert np.all(np.isfinite(out)), f"{what}: non-finite output"
     err = np.abs(out - ref)
-    excess = err - (ATOL + BF16_HALF_ULP * np.abs(ref))
+    bound = ATOL + BF16_HALF_ULP * np.abs(ref)
+    if extra_bound is not None:
+        bound = bound + extra_bound
+    _record(what, err, ref, **({"max_extra_bound": float(np.max(extra_bound))} if extra_bound is not None else {}))
+    excess = err - bound
     worst = int(np.argmax(excess)) if excess.size else 0
     assert excess.size == 0 or excess.max() <= 0, (
         f"{what}: |err| {err.flat[worst]:.4g} at {np.unravel_index(worst, err.shape)} "
-        f"(ref {ref.flat[worst]:.4g}, out {out.flat[worst]:.4g})")
-    assert err.size == 0 or err.mean() <= MEAN_ATOL, f"{what}: mean |err| {err.mean():.4g}"
+        f"(ref {ref.flat[worst]:.4g}, out {out.flat[worst]:.4g}, bound {bound.flat[worst]:.4g})")
+    assert err.size == 0 or err.mean() <= MEAN_ATOL + mean_extra, f"{what}: mean |err| {err.mean():.4g}"
 
 
 def assert_lse(out, ref, what="lse"):
-    out = out.detach().double().cpu().numpy() if hasattr(out, "detach") else np.asarray(out)
+    out = _as_f64(out)
     ref = np.asarray(ref, dtype=np.float64)
     assert np.all(np.isfinite(out)), f"{what}: non-finite"
     err = np.abs(out - ref)
+    _record(what, err, ref)
     assert err.size == 0 or err.max() <= LSE_ATOL, f"{what}: max |err| {err.max():.4g}"
+
+
+def bwd_rounding_bound(q, k, v, do, cu, scale: float, o_ref, lse_ref, k_sigma: float = 6.0):
+    """Bound of the backward's rounding error that grows with the logit spread, per element of dQ and
+    dK, from the inputs and the oracle's fp64 O and LSE only: k_sigma standard deviations of the
+    first-order error model below.
+
+    Each rounding to bf16 (8 significant bits, round to nearest) leaves an error uniform in
+    +-2^-9 |x|, standard deviation u|x| with u = 2^-9 / sqrt(3); different roundings are independent.
+      * The forward rounds P to bf16 before the PV product and O to bf16 on output, so
+        sd(dO_ic) = u sqrt(O_ic^2 + sum_j P_ij^2 V_jc^2).
+      * The backward takes D_i = <dO_i, O_i> from that bf16 O (the FlashAttention convention):
+        sd(dD_i) = sqrt(sum_c dO_ic^2 sd(dO_ic)^2).  This one error is shared by every key of row i:
+        dS_ij = P_ij (dP_ij - D_i) moves by -P_ij dD_i, so dQ_ic moves by -scale dD_i sum_j P_ij K_jc
+        and dK_jc by -scale sum_i P_ij dD_i Q_ic (independent over i and over the group's heads).
+      * dS is rounded to bf16 before the dQ and dK products: independent errors of sd u |dS_ij|.
+    At the default scale (logit standard deviation 1) these terms stay near 1e-3; with a peaky
+    softmax (logit spread ~4x) P_ij and |dS_ij| concentrate on few keys and they reach ~1e-2.
+    Returns (dq_extra [N,hq,d], dk_extra [N,hkv,d]) as float64 arrays."""
+    qd, kd, vd, dod = (torch.as_tensor(oracle.widen(t)[0]) for t in (q, k, v, do))
+    o = torch.as_tensor(np.asarray(o_ref, dtype=np.float64))
+    lse = torch.as_tensor(np.asarray(lse_ref, dtype=np.float64))
+    n, hq, d = qd.shape
+    hkv = kd.shape[1]
+    G = hq // hkv
+    u = 2.0 ** -9 / math.sqrt(3.0)
+    var_q = torch.zeros_like(qd)
+    var_k = torch.zeros_like(kd)
+    for s0, e0 in zip(np.asarray(cu)[:-1].tolist(), np.asarray(cu)[1:].tolist()):
+        if e0 <= s0:
+            continue
+        L = e0 - s0
+        causal = torch.tril(torch.ones(L, L, dtype=torch.bool))
+        for h in range(hq):
+            g = h // G
+            Q, K, V, dO, O = qd[s0:e0, h], kd[s0:e0, g], vd[s0:e0, g], dod[s0:e0, h], o[s0:e0, h]
+            P = torch.where(causal, torch.exp(scale * (Q @ K.T) - lse[h, s0:e0, None]),
+                            torch.zeros((), dtype=torch.float64))
+            dS = P * (dO @ V.T - (dO * O).sum(1)[:, None])
+            var_o = u * u * (O * O + (P * P) @ (V * V))              # [L, d]
+            var_d = (dO * dO * var_o).sum(1)                          # [L]
+            var_q[s0:e0, h] += scale ** 2 * (var_d[:, None] * (P @ K) ** 2 + u * u * ((dS * dS) @ (K * K)))
+            var_k[s0:e0, g] += scale ** 2 * (((P * P) * var_d[:, None]).T @ (Q * Q) + u * u * ((dS * dS).T @ (Q * Q)))
+    return (k_sigma * var_q.sqrt()).numpy(), (k_sigma * var_k.sqrt()).numpy()
 
 
 class Run:
@@ -132,13 +204,12 @@ def doc_sum_identities(dk, dv, do, q, scale: float, cu, hq: int, hkv: int, what:
     in exact arithmetic; sum_j P_ij is 1 only in exact arithmetic), so its
     natural scale is that of a random walk over the document's rows and heads:
     sqrt(sum dO^2) for dV and softmax_scale * sqrt(sum Q^2) for dK (per
-    element).  Tolerance: 0.1 + 4e-3 * that scale.  Measured deviations of the
+    element).  Tolerance: 0.1 + 2e-3 * that scale.  Measured deviations of the
     kernel's per-document sums: at most 3e-4 of the dV scale against the full
     oracle on a 16K-token batch with an 8K-token document, and 1.4e-3 of it
-    for the 256K-token document of the 512K batch, whose individual dK/dV rows
-    (its first keys included) are all within the element bound against an
-    independent fp64 computation; a dropped near-diagonal tile moves a sum by
-    O(1).
+    for the 256K-token document of the 512K batch; a dropped near-diagonal
+    tile moves a sum by O(1).  The largest deviation per tensor, as a fraction
+    of its scale, is recorded with the parity records.
     """
     G = hq // hkv
     cu_t = torch.as_tensor(np.asarray(cu, dtype=np.int64), device=dk.device)
@@ -158,7 +229,12 @@ def doc_sum_identities(dk, dv, do, q, scale: float, cu, hq: int, hkv: int, what:
     scale_v = torch.sqrt(seg_sum((dog ** 2).sum(2)))
     qg = q.double().reshape(q.shape[0], hkv, G, q.shape[2])
     scale_k = scale * torch.sqrt(seg_sum((qg ** 2).sum(2)))
-    tol_k = 0.1 + 4e-3 * scale_k
-    tol_v = 0.1 + 4e-3 * scale_v
+    tol_k = 0.1 + 2e-3 * scale_k
+    tol_v = 0.1 + 2e-3 * scale_v
+    PARITY_RECORDS.append({"test": os.environ.get("PYTEST_CURRENT_TEST", "").split(" ")[0], "what": what,
+                           "sum_dK_over_scale": float((sk.abs() / scale_k.clamp_min(1e-30)).max().item()),
+                           "sum_dV_dev_over_scale": float(((sv - ref_v).abs() / scale_v.clamp_min(1e-30)).max().item()),
+                           "sum_dK_max": float(sk.abs().max().item()),
+                           "sum_dV_dev_max": float((sv - ref_v).abs().max().item())})
     assert torch.all(sk.abs() <= tol_k), f"{what}: sum dK per doc {sk.abs().max().item():.4g}"
     assert torch.all((sv - ref_v).abs() <= tol_v), f"{what}: sum dV per doc {(sv - ref_v).abs().max().item():.4g}"

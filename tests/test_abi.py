@@ -39,3 +39,19 @@ def test_null_arguments_rejected_without_gpu():
     assert lib.sap_plan(None, 0, 0, 1, 128, 128, None) == -1
     assert lib.sap_plan_items(None, None, None) == -1
     assert lib.sap_workspace_size(None, 1, 1, 64, 0, None) == -1
+
+
+def test_misaligned_workspace_rejected_without_gpu():
+    """A workspace that is not 16-byte aligned is refused (SAP_ERR_WORKSPACE) by the forward and the
+    merge before any device work: the kernels store and load the partials as 16-byte vectors.  The
+    pointers are never dereferenced; the checks run on the host before the first CUDA call."""
+    lib = sap.load_library()
+    plan = sap.sap_plan([0, 512], 512, 2)  # q tiles 2 and 3 see both chunks: partial slots exist
+    assert sap.sap_plan_stats(plan)["n_partial_slots"] > 0
+    need = sap.sap_workspace_size(plan, 2, 1, 64, sap.SAP_WS_FWD)
+    fake = ctypes.c_void_p(1 << 20)  # 16-byte aligned, never dereferenced
+    bad_ws = ctypes.c_void_p((1 << 21) + 8)
+    st = lib.sap_attn_fwd(plan.handle, fake, fake, fake, 2, 1, 64, 0.125, fake, fake, bad_ws, need + 64, None)
+    assert st == -4
+    st = lib.sap_merge(plan.handle, bad_ws, need + 64, 2, 64, fake, fake, None)
+    assert st == -4

@@ -12,7 +12,7 @@ import torch
 import oracle
 import packed_sequence_causal_b200 as sap
 import workloads
-from gpu_helpers import Run, assert_close, assert_lse
+from gpu_helpers import Run, assert_close, assert_lse, bwd_rounding_bound
 
 pytestmark = pytest.mark.gpu
 
@@ -117,16 +117,29 @@ def test_custom_scale():
     _fwd_bwd_full([400, 112], 2, 1, 128, 2, seed=10, scale=0.1)
 
 
-@pytest.mark.parametrize("scale", [0.37, 1.0 / math.sqrt(8.0)])
-def test_large_scores_forward(scale):
-    """Logits ~4x the usual spread: exercises the lazy O rescaling of the forward.
+@pytest.mark.parametrize("lens,hq,hkv,nchunks,seed,scale", [
+    ([400, 112], 2, 1, 2, 10, 0.37),
+    ([256, 384], 2, 2, 1, 11, 1.0 / math.sqrt(8.0)),
+])
+def test_large_scores(lens, hq, hkv, nchunks, seed, scale):
+    """Logits with ~4x the usual spread (scale 0.37 or 1/sqrt(8) on d = 128): exercises the lazy O
+    rescaling of the forward, and the backward where the softmax is peaky.
 
-    Only the forward is held to the parity bound here: with such peaky softmax
-    the backward's bf16 operands (dS, P) and the D_i = <dO_i, O_i> taken from
-    the bf16 O put dQ/dK errors at ~0.06 -- the same size as a reference bf16
-    tensor-core backward shows on the same input."""
-    _fwd_bwd_full([400, 112] if scale == 0.37 else [256, 384], 2, 1 if scale == 0.37 else 2, 128,
-                  2 if scale == 0.37 else 1, seed=10 if scale == 0.37 else 11, scale=scale, bwd=False)
+    O and LSE are held to the usual bounds.  dQ and dK get, on top of them, the first-order rounding
+    term of bwd_rounding_bound (D_i from the bf16 O, dS rounded to bf16), which grows with the logit
+    spread; dV keeps the usual bound."""
+    b = workloads.custom_batch(lens, hq, hkv, 128, seed=seed, with_do=True)
+    r = Run(b, nchunks, scale)
+    o, lse = r.fwd()
+    ro, rl = oracle.attn_fwd(b.q, b.k, b.v, b.cu_seqlens, r.scale)
+    assert_close(o, ro, "O (large scores)")
+    assert_lse(lse, rl, "LSE (large scores)")
+    dq, dk, dv = r.bwd()
+    rdq, rdk, rdv = oracle.attn_bwd(b.q, b.k, b.v, b.do, b.cu_seqlens, r.scale)
+    eq, ek = bwd_rounding_bound(b.q, b.k, b.v, b.do, b.cu_seqlens, r.scale, ro, rl)
+    assert_close(dq, rdq, "dQ (large scores)", extra_bound=eq, mean_extra=float(eq.mean()))
+    assert_close(dk, rdk, "dK (large scores)", extra_bound=ek, mean_extra=float(ek.mean()))
+    assert_close(dv, rdv, "dV (large scores)")
 
 
 def test_empty_batch_is_a_no_op():

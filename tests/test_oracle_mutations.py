@@ -87,6 +87,28 @@ def _tiles_match_brute_force(mod):
     return bool(np.all(covered[mask]))
 
 
+def _tags_match_brute_force(mod):
+    """Every tag against the dense mask, in both directions: FULL iff the box is fully unmasked,
+    CAUSAL iff (otherwise) it is a diagonal box holding exactly the pattern j <= i."""
+    cu = workloads.cu_seqlens_from_lengths([20, 5, 39, 16, 21])
+    n, bm = 101, 16
+    items = mod.tile_list(cu, n, 1, bm, bm)
+    doc = np.repeat(np.arange(len(cu) - 1), np.diff(cu))
+    i, j = np.arange(n)[:, None], np.arange(n)[None, :]
+    mask = (doc[:, None] == doc[None, :]) & (j <= i)
+    for qt, kt, _, _, tag in items:
+        box = np.zeros((bm, bm), dtype=bool)
+        sub = mask[qt * bm:(qt + 1) * bm, kt * bm:(kt + 1) * bm]
+        box[: sub.shape[0], : sub.shape[1]] = sub
+        ii = np.arange(bm)[:, None] + qt * bm
+        jj = np.arange(bm)[None, :] + kt * bm
+        causal = qt == kt and np.array_equal(box, (jj <= ii) & (ii < n))
+        want = 0 if box.all() else (1 if causal else 2)
+        if tag != want:
+            return False
+    return True
+
+
 MUTATIONS = [
     ("no_diagonal", "int64_t hi = i < kv_hi - 1 ? i : kv_hi - 1;",
      "int64_t hi = (i - 1) < kv_hi - 1 ? (i - 1) : kv_hi - 1;", _fwd_matches_library),
@@ -98,12 +120,14 @@ MUTATIONS = [
     ("merge_weight", "double w = exp(lse_parts[((size_t)b * hq + h) * n + i] - l_all);",
      "double w = exp(lse_parts[((size_t)b * hq + h) * n + i] - m);", _chunked_equals_plain),
     ("full_tag", "if (all)\n        tag = 0;", "if (any)\n        tag = 0;", _tiles_match_brute_force),
+    ("causal_tag_dropped", "        tag = 1;\n", "        tag = 2;\n", _tags_match_brute_force),
 ]
 
 
 def test_unmutated_oracle_passes_every_check():
     import oracle
-    for check in (_fwd_matches_library, _bwd_matches_autograd, _chunked_equals_plain, _tiles_match_brute_force):
+    for check in (_fwd_matches_library, _bwd_matches_autograd, _chunked_equals_plain, _tiles_match_brute_force,
+                  _tags_match_brute_force):
         assert check(oracle), check.__name__
 
 

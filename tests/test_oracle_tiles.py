@@ -4,7 +4,8 @@ The tile list is checked against brute force on every (i, j) pair: each
 unmasked pair of the packed causal mask lies in exactly one emitted item, no
 emitted item is empty, and each tag says what the kernels rely on (FULL: no
 pair of the box is masked; CAUSAL: inside the box the mask is exactly j <= i;
-MASKED: neither).  The interval-based and exhaustive evaluations must agree.
+MASKED: neither), in both directions: a diagonal box that holds exactly the
+causal pattern is tagged CAUSAL, not MASKED.  The interval-based and exhaustive evaluations must agree.
 """
 import numpy as np
 import pytest
@@ -38,16 +39,20 @@ def _check_against_mask(cu, n, nchunks, bm, bn):
         assert box.any()
         covered[i0:i0 + bm, j0:j0 + bn] += 1
         assert qc == i0 // chunk and kc == j0 // chunk
+        ii = np.arange(bm)[:, None] + i0
+        jj = np.arange(bn)[None, :] + j0
+        causal_box = qt * bm == kt * bn and bm == bn and np.array_equal(box, (jj <= ii) & (ii < n))
         if tag == oracle.TAG_FULL:
             assert box.all()
         elif tag == oracle.TAG_CAUSAL:
             assert qt == kt and bm == bn
-            ii = np.arange(bm)[:, None] + i0
-            jj = np.arange(bn)[None, :] + j0
-            causal = (jj <= ii) & (ii < n)
-            assert np.array_equal(box, causal)
+            assert causal_box
         else:
             assert tag == oracle.TAG_MASKED and not box.all()
+        # converse: a box that is not fully unmasked but holds exactly the causal pattern of its
+        # diagonal (one document covers every real row of the tile) must be tagged CAUSAL
+        if causal_box and not box.all():
+            assert tag == oracle.TAG_CAUSAL, (qt, kt, tag)
     assert np.all(covered[mask] == 1)
     assert int(mask.sum()) == oracle.unmasked_pairs(cu)
     ex = oracle.tile_list(cu, n, nchunks, bm, bn, exhaustive=True)
@@ -96,3 +101,17 @@ def test_tile_list_tiny_workload():
     b = workloads.make_batch("tiny", 0)
     items = _check_against_mask(b.cu_seqlens, 1024, 2, 128, 128)
     assert len(items) == 21
+
+
+def test_tile_list_diagonal_tiles_of_one_document_are_causal():
+    """One document over five 16-token tiles: every diagonal tile is CAUSAL and every tile below
+    the diagonal FULL.  With N = 100 (ragged last tile, two documents) the partial last diagonal
+    tile lies inside the second document and is CAUSAL too."""
+    items = _check_against_mask(workloads.cu_seqlens_from_lengths([80]), 80, 1, 16, 16)
+    for qt, kt, _, _, tag in items:
+        assert tag == (oracle.TAG_CAUSAL if qt == kt else oracle.TAG_FULL)
+    assert len(items) == 15
+    items = _check_against_mask(workloads.cu_seqlens_from_lengths([33, 67]), 100, 1, 16, 16)
+    tags = {(int(qt), int(kt)): int(tag) for qt, kt, _, _, tag in items}
+    assert tags[(6, 6)] == oracle.TAG_CAUSAL
+    assert tags[(2, 2)] == oracle.TAG_MASKED  # tokens 32 | 33..47: a document boundary inside the tile
