@@ -41,6 +41,10 @@ def lib():
         L.oracle_max_threads.restype = ctypes.c_int
         L.oracle_tile_list.restype = i64
         L.oracle_tile_list.argtypes = [P, i32, i64, i32, i32, i32, ctypes.c_int, P, i64]
+        L.oracle_tile_list_bounds.restype = i64
+        L.oracle_tile_list_bounds.argtypes = [P, i32, i64, P, i32, i32, i32, ctypes.c_int, P, i64]
+        L.oracle_balanced_bounds.restype = ctypes.c_int
+        L.oracle_balanced_bounds.argtypes = [P, i32, i64, i32, i32, P]
         L.oracle_attn_fwd.restype = ctypes.c_int
         L.oracle_attn_fwd.argtypes = [P, P, P, i64, i32, i32, i32, P, i32, dbl, i64, i64, P, P, ctypes.c_int]
         L.oracle_merge.restype = ctypes.c_int
@@ -86,15 +90,36 @@ def max_threads() -> int:
     return int(lib().oracle_max_threads())
 
 
-def tile_list(cu_seqlens, n: int, nchunks: int, bm: int = 128, bn: int = 128, exhaustive: bool = False) -> np.ndarray:
-    """Canonical non-empty tile list, int32 [items, 5] = (q_tile, kv_tile, q_chunk, kv_chunk, tag)."""
+def tile_list(cu_seqlens, n: int, nchunks: int, bm: int = 128, bn: int = 128, exhaustive: bool = False,
+              bounds=None) -> np.ndarray:
+    """Canonical non-empty tile list, int32 [items, 5] = (q_tile, kv_tile, q_chunk, kv_chunk, tag).
+
+    Chunks: nchunks equal parts, or the explicit token bounds ``bounds`` (nchunks + 1 entries)."""
     cu = _cu(cu_seqlens)
-    cnt = _check(lib().oracle_tile_list(_ptr(cu), len(cu) - 1, n, nchunks, bm, bn, int(exhaustive), None, 0),
-                 "tile_list")
+    if bounds is None:
+        def call(out, cap):
+            return lib().oracle_tile_list(_ptr(cu), len(cu) - 1, n, nchunks, bm, bn, int(exhaustive), out, cap)
+    else:
+        b = np.ascontiguousarray(np.asarray(bounds, dtype=np.int64))
+        if len(b) != nchunks + 1:
+            raise ValueError("bounds needs nchunks + 1 entries")
+
+        def call(out, cap):
+            return lib().oracle_tile_list_bounds(_ptr(cu), len(cu) - 1, n, _ptr(b), nchunks, bm, bn,
+                                                 int(exhaustive), out, cap)
+    cnt = _check(call(None, 0), "tile_list")
     out = np.zeros((max(cnt, 1), 5), dtype=np.int32)
-    cnt2 = lib().oracle_tile_list(_ptr(cu), len(cu) - 1, n, nchunks, bm, bn, int(exhaustive), _ptr(out), cnt)
+    cnt2 = call(_ptr(out), cnt)
     assert cnt2 == cnt
     return out[:cnt]
+
+
+def balanced_bounds(cu_seqlens, n: int, nchunks: int, block: int = 128) -> np.ndarray:
+    """Balanced contiguous chunk bounds (int64, nchunks + 1 token offsets): see oracle_balanced_bounds."""
+    cu = _cu(cu_seqlens)
+    out = np.zeros(nchunks + 1, dtype=np.int64)
+    _check(lib().oracle_balanced_bounds(_ptr(cu), len(cu) - 1, n, nchunks, block, _ptr(out)), "balanced_bounds")
+    return out
 
 
 def attn_fwd(q, k, v, cu_seqlens, scale: float, kv_range=None, nthreads: int = 0):
@@ -122,15 +147,21 @@ def merge(o_parts, lse_parts):
     return o, lse
 
 
-def attn_fwd_chunked(q, k, v, cu_seqlens, scale: float, nchunks: int, nthreads: int = 0):
-    """Partials per kv chunk (each over all query rows), then the exact merge.
+def attn_fwd_chunked(q, k, v, cu_seqlens, scale: float, nchunks: int, nthreads: int = 0, bounds=None):
+    """Partials per kv chunk (each over all query rows), then the exact merge.  Chunks: nchunks equal
+    parts, or the explicit token bounds ``bounds``.
 
     Returns (O, LSE, o_parts, lse_parts)."""
     n = q.shape[0]
-    if nchunks < 1 or (nchunks > 1 and n % nchunks):
-        raise ValueError("N must split into equal chunks")
-    c = n // nchunks if nchunks > 1 else n
-    parts = [attn_fwd(q, k, v, cu_seqlens, scale, (b * c, (b + 1) * c), nthreads) for b in range(nchunks)]
+    if bounds is None:
+        if nchunks < 1 or (nchunks > 1 and n % nchunks):
+            raise ValueError("N must split into equal chunks")
+        c = n // nchunks if nchunks > 1 else n
+        bounds = [b * c for b in range(nchunks)] + [n]
+    bounds = [int(x) for x in bounds]
+    if len(bounds) != nchunks + 1 or bounds[0] != 0 or bounds[-1] != n:
+        raise ValueError("bounds must run from 0 to N in nchunks parts")
+    parts = [attn_fwd(q, k, v, cu_seqlens, scale, (bounds[b], bounds[b + 1]), nthreads) for b in range(nchunks)]
     op = np.stack([p[0] for p in parts])
     lp = np.stack([p[1] for p in parts])
     o, lse = merge(op, lp)

@@ -31,7 +31,9 @@
  *   CAUSAL (1) the diagonal tile (same row and column range) of one document,
  *   MASKED (2) anything else,
  * in canonical order (q-tile ascending, then kv-tile ascending), with
- * q_chunk = qt*BM / C and kv_chunk = kt*BN / C, C = N / P.
+ * q_chunk / kv_chunk the chunk holding the tile's first row / key, chunks being
+ * P equal parts of the sequence or explicit contiguous bounds.
+ * Balanced chunk bounds: see oracle_balanced_bounds.
  *
  * Layouts: Q, O, dO, dQ are [N][hq][d]; K, V, dK, dV are [N][hkv][d]; LSE is
  * [hq][N].  All floating point is double.
@@ -86,17 +88,47 @@ static void token_docs(const int32_t* cu, int32_t ndocs, int64_t n, int32_t* doc
 
 /* ---------------------------------------------------------------- tile list */
 
-static int tile_geometry(int64_t n, int32_t nchunks, int32_t bm, int32_t bn, int64_t* chunk) {
-  if (bm <= 0 || bn <= 0 || nchunks < 1) return ORACLE_ERR_ARG;
-  if (nchunks == 1) {
-    *chunk = n > 0 ? n : 1;
-    return ORACLE_OK;
+/*
+ * Chunks are contiguous token ranges [bounds[c], bounds[c+1]): bounds[0] = 0,
+ * bounds[nchunks] = n, strictly increasing (except the single empty chunk of
+ * an empty batch), interior bounds multiples of both tile sizes.  Equal chunks
+ * are bounds[c] = c * n / nchunks.
+ */
+static int check_bounds(int64_t n, const int64_t* bounds, int32_t nchunks, int32_t bm, int32_t bn) {
+  if (bm <= 0 || bn <= 0 || nchunks < 1 || bounds == NULL) return ORACLE_ERR_ARG;
+  if (bounds[0] != 0 || bounds[nchunks] != n) return ORACLE_ERR_CHUNKS;
+  for (int32_t c = 0; c < nchunks; ++c) {
+    if (bounds[c + 1] <= bounds[c] && !(nchunks == 1 && n == 0)) return ORACLE_ERR_CHUNKS;
+    if (c > 0 && (bounds[c] % bm != 0 || bounds[c] % bn != 0)) return ORACLE_ERR_CHUNKS;
   }
-  if (n % nchunks != 0) return ORACLE_ERR_CHUNKS;
-  int64_t c = n / nchunks;
-  if (c % bm != 0 || c % bn != 0) return ORACLE_ERR_CHUNKS;
-  *chunk = c;
   return ORACLE_OK;
+}
+
+/* The chunk holding token t: the c with bounds[c] <= t < bounds[c+1]. */
+static int32_t chunk_of_token(const int64_t* bounds, int32_t nchunks, int64_t t) {
+  int32_t c = 0;
+  while (c + 1 < nchunks && bounds[c + 1] <= t) ++c;
+  return c;
+}
+
+int64_t oracle_tile_list_bounds(const int32_t* cu, int32_t ndocs, int64_t n, const int64_t* bounds, int32_t nchunks,
+                                int32_t bm, int32_t bn, int exhaustive, int32_t* out, int64_t cap);
+
+/*
+ * Equal chunks: bounds[c] = c * n / nchunks, which needs n % nchunks == 0 and
+ * a chunk length that is a multiple of both tile sizes (one chunk: any n).
+ */
+int64_t oracle_tile_list(const int32_t* cu, int32_t ndocs, int64_t n, int32_t nchunks, int32_t bm, int32_t bn,
+                         int exhaustive, int32_t* out, int64_t cap) {
+  if (bm <= 0 || bn <= 0 || nchunks < 1) return ORACLE_ERR_ARG;
+  if (nchunks > 1 && n % nchunks != 0) return ORACLE_ERR_CHUNKS;
+  int64_t* bounds = (int64_t*)malloc(sizeof(int64_t) * ((size_t)nchunks + 1));
+  if (!bounds) return ORACLE_ERR_NOMEM;
+  for (int32_t c = 0; c <= nchunks; ++c) bounds[c] = (int64_t)c * (n / nchunks);
+  bounds[nchunks] = n;
+  int64_t r = oracle_tile_list_bounds(cu, ndocs, n, bounds, nchunks, bm, bn, exhaustive, out, cap);
+  free(bounds);
+  return r;
 }
 
 /*
@@ -106,12 +138,11 @@ static int tile_geometry(int64_t n, int32_t nchunks, int32_t bm, int32_t bn, int
  * the first cap items are written and ORACLE_ERR_CAPACITY is not raised: the
  * caller compares the count to cap).
  */
-int64_t oracle_tile_list(const int32_t* cu, int32_t ndocs, int64_t n, int32_t nchunks, int32_t bm, int32_t bn,
-                         int exhaustive, int32_t* out, int64_t cap) {
+int64_t oracle_tile_list_bounds(const int32_t* cu, int32_t ndocs, int64_t n, const int64_t* bounds, int32_t nchunks,
+                                int32_t bm, int32_t bn, int exhaustive, int32_t* out, int64_t cap) {
   int rc = check_seqlens(cu, ndocs, n);
   if (rc) return rc;
-  int64_t chunk;
-  rc = tile_geometry(n, nchunks, bm, bn, &chunk);
+  rc = check_bounds(n, bounds, nchunks, bm, bn);
   if (rc) return rc;
   if (n == 0) return 0;
   int32_t* doc_of = (int32_t*)malloc(sizeof(int32_t) * (size_t)n);
@@ -159,8 +190,8 @@ int64_t oracle_tile_list(const int32_t* cu, int32_t ndocs, int64_t n, int32_t nc
         int32_t* it = out + 5 * count;
         it[0] = (int32_t)qt;
         it[1] = (int32_t)kt;
-        it[2] = (int32_t)(i0 / chunk);
-        it[3] = (int32_t)(j0 / chunk);
+        it[2] = chunk_of_token(bounds, nchunks, i0);
+        it[3] = chunk_of_token(bounds, nchunks, j0);
         it[4] = tag;
       }
       ++count;
@@ -169,6 +200,88 @@ int64_t oracle_tile_list(const int32_t* cu, int32_t ndocs, int64_t n, int32_t nc
   free(doc_of);
   free(start_of);
   return count;
+}
+
+/* ------------------------------------------------------------ balanced cut */
+
+/*
+ * Balanced chunk bounds (the load-balancing scheduler of the HSAP method
+ * details, read as: cut the sequence into nchunks contiguous, tile-aligned,
+ * non-empty parts whose largest work is as small as possible).  Work of a q
+ * tile = the number of items (non-empty tiles) in its row of the tile list.
+ * Definition:
+ *   M* = min over all cuts of max over chunks of the chunk's summed work;
+ *   among the cuts reaching M*, the one with the lexicographically largest
+ *   bound vector.
+ * M* comes from the textbook dynamic program best[k][t] = min over s of
+ * max(best[k-1][s], work(s..t)) over cuts of tiles [0, t) into k parts; the
+ * bounds are then chosen left to right, each the largest tile index b after
+ * the previous bound such that the chunk's work is <= M* and tiles [b, T) can
+ * still be cut into the remaining number of parts with work <= M* (a second
+ * table, over suffixes).  out_bounds: nchunks + 1 entries, in tokens.
+ */
+int oracle_balanced_bounds(const int32_t* cu, int32_t ndocs, int64_t n, int32_t nchunks, int32_t block,
+                           int64_t* out_bounds) {
+  int rc = check_seqlens(cu, ndocs, n);
+  if (rc) return rc;
+  if (block <= 0 || nchunks < 1 || out_bounds == NULL) return ORACLE_ERR_ARG;
+  if (n == 0) {
+    if (nchunks != 1) return ORACLE_ERR_CHUNKS;
+    out_bounds[0] = out_bounds[1] = 0;
+    return ORACLE_OK;
+  }
+  int64_t T = (n + block - 1) / block;
+  if (nchunks > T) return ORACLE_ERR_CHUNKS;
+  int64_t cnt = oracle_tile_list(cu, ndocs, n, 1, block, block, 0, NULL, 0);
+  if (cnt < 0) return (int)cnt;
+  int32_t* items = (int32_t*)malloc(sizeof(int32_t) * 5 * (size_t)(cnt > 0 ? cnt : 1));
+  int64_t* pre = (int64_t*)calloc((size_t)T + 1, sizeof(int64_t));   /* pre[t] = work of tiles [0, t) */
+  int64_t K = nchunks, W = T + 1;
+  int64_t* best = (int64_t*)malloc(sizeof(int64_t) * (size_t)((K + 1) * W));
+  int64_t* suf = (int64_t*)malloc(sizeof(int64_t) * (size_t)((K + 1) * W));
+  if (!items || !pre || !best || !suf) {
+    free(items), free(pre), free(best), free(suf);
+    return ORACLE_ERR_NOMEM;
+  }
+  oracle_tile_list(cu, ndocs, n, 1, block, block, 0, items, cnt);
+  for (int64_t e = 0; e < cnt; ++e) pre[items[5 * e] + 1] += 1;
+  for (int64_t t = 0; t < T; ++t) pre[t + 1] += pre[t];
+  const int64_t INF = INT64_MAX;
+  /* best[k][t]: tiles [0, t) in k non-empty parts; suf[m][s]: tiles [s, T) in m non-empty parts */
+  for (int64_t i = 0; i < (K + 1) * W; ++i) best[i] = suf[i] = INF;
+  best[0 * W + 0] = 0;
+  suf[0 * W + T] = 0;
+  for (int64_t k = 1; k <= K; ++k)
+    for (int64_t t = k; t <= T; ++t)
+      for (int64_t s = k - 1; s < t; ++s) {
+        int64_t a = best[(k - 1) * W + s];
+        if (a == INF) continue;
+        int64_t w = pre[t] - pre[s];
+        int64_t v = a > w ? a : w;
+        if (v < best[k * W + t]) best[k * W + t] = v;
+      }
+  for (int64_t m = 1; m <= K; ++m)
+    for (int64_t s = T - m; s >= 0; --s)
+      for (int64_t e = s + 1; e <= T - (m - 1); ++e) {
+        int64_t a = suf[(m - 1) * W + e];
+        if (a == INF) continue;
+        int64_t w = pre[e] - pre[s];
+        int64_t v = a > w ? a : w;
+        if (v < suf[m * W + s]) suf[m * W + s] = v;
+      }
+  int64_t mstar = best[K * W + T];
+  out_bounds[0] = 0;
+  int64_t prev = 0;
+  for (int64_t k = 1; k < K; ++k) {
+    int64_t chosen = -1;
+    for (int64_t b = prev + 1; b <= T - (K - k); ++b)
+      if (pre[b] - pre[prev] <= mstar && suf[(K - k) * W + b] <= mstar) chosen = b;
+    out_bounds[k] = chosen * block;
+    prev = chosen;
+  }
+  out_bounds[K] = n;
+  free(items), free(pre), free(best), free(suf);
+  return ORACLE_OK;
 }
 
 /* ------------------------------------------------------------------ forward */
