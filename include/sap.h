@@ -94,6 +94,64 @@ typedef struct {
 int sap_plan(const int32_t* cu_seqlens_host, int32_t num_docs, int64_t total_tokens, int32_t num_chunks,
              int32_t block_m, int32_t block_n, sap_plan_t* out);
 
+/* Plan over explicit contiguous chunks: chunk c is tokens [chunk_bounds[c], chunk_bounds[c+1]),
+ * with chunk_bounds[0] = 0, chunk_bounds[num_chunks] = N, strictly increasing, and every
+ * interior bound a multiple of block_m and block_n (otherwise SAP_ERR_BAD_CHUNKS).  Equal chunks
+ * (sap_plan) are the special case chunk_bounds[c] = c N / P.  The items, tags and schedules are
+ * those of sap_plan with q_chunk / kv_chunk the chunk that holds the tile's first token.
+ * (HSAP page, method details: the sequence is cut into parts per device; the load-balancing
+ * scheduler chooses the cut -- see sap_balanced_chunks.)  chunk_bounds is read, not kept. */
+int sap_plan_chunks(const int32_t* cu_seqlens_host, int32_t num_docs, int64_t total_tokens,
+                    const int64_t* chunk_bounds, int32_t num_chunks, int32_t block_m, int32_t block_n,
+                    sap_plan_t* out);
+
+/* Balanced chunk bounds (HSAP page, method details: the load-balancing scheduler; explainer page,
+ * challenges: uneven document lengths leave devices idle).  The cost of a q tile of `block`
+ * tokens is the number of kv tiles it touches (its items: one block x block tile of work per
+ * head in each pass).  Writes num_chunks + 1 bounds into chunk_bounds (caller-owned): contiguous,
+ * interior bounds multiples of block, every chunk non-empty, minimising the largest summed cost
+ * of a chunk; among the cuts that reach that minimum, the lexicographically largest bounds (each
+ * chunk takes as many tiles as fit, leaving at least one tile per later chunk).  Errors:
+ * SAP_ERR_BAD_SEQLENS, SAP_ERR_BAD_CHUNKS (num_chunks < 1 or more chunks than tiles). */
+int sap_balanced_chunks(const int32_t* cu_seqlens_host, int32_t num_docs, int64_t total_tokens, int32_t num_chunks,
+                        int32_t block, int64_t* chunk_bounds);
+
+/* The chunk bounds of a plan (num_chunks + 1 entries; host memory owned by the plan). */
+int sap_plan_chunk_bounds(sap_plan_t plan, const int64_t** bounds, int32_t* num_chunks);
+
+/* Per q chunk c (caller-owned arrays of num_chunks entries, either may be NULL): the plan's items
+ * whose q tile lies in chunk c, and the unmasked (i, j) pairs of its query rows (per head).  The
+ * work of device c under sequence parallelism; a rank plan reports its own chunk only. */
+int sap_plan_chunk_stats(sap_plan_t plan, int64_t* items_per_chunk, int64_t* pairs_per_chunk);
+
+/* Rank plan for sequence parallelism (HSAP page, abstract and method details: each device computes
+ * the partial attention of its own part of the sequence, and only the key/value data of documents
+ * that reach into that part crosses devices).  From a full plan, the plan of the device that owns
+ * q chunk `chunk`: the items whose q tile lies in the chunk, with the same tags and global tile
+ * indices, and their forward / backward schedules.  Its device calls take WINDOWED buffers:
+ *   query side  Q, O, dO, dQ : rows [q_begin, q_end) = the chunk;  LSE [hq][q_end - q_begin];
+ *   key side    K, V, dK, dV : rows [kv_begin, q_end),
+ * where span_begin = first token of the document holding token q_begin (the earliest key any
+ * query of the chunk may see) and kv_begin = span_begin rounded down to a kv tile
+ * (sap_plan_window).  K/V rows [kv_begin, span_begin) are never attended to but are read as whole
+ * tiles: they must hold finite values (zeros will do).  Rows [span_begin, q_begin) are the other
+ * devices' keys and values (sap_plan_rank_spans lists who sends which).  dK/dV rows below q_begin
+ * are this device's partial sums for other devices' tokens (see sap_attn_bwd_kv_add).  The rank
+ * plan is independent of the full plan (destroy both). */
+int sap_plan_rank(sap_plan_t plan, int32_t chunk, sap_plan_t* out);
+
+/* Buffer window of a plan: [q_begin, q_end) query rows, [kv_begin, q_end) key/value rows, and
+ * span_begin (see sap_plan_rank).  A full plan reports 0, N, 0, 0. */
+int sap_plan_window(sap_plan_t plan, int64_t* q_begin, int64_t* q_end, int64_t* kv_begin, int64_t* span_begin);
+
+/* Exchange list of the device owning q chunk `chunk` (full plans only): for every earlier chunk b
+ * that holds keys of a document reaching into `chunk`, one entry (b, lo, hi) = the token range
+ * [lo, hi) of chunk b that this device needs; *n_spans entries are written into spans (caller-owned,
+ * 3 * num_chunks int64).  These are exactly the chunk pairs of the plan's chunk-pair table with
+ * q_chunk = chunk and kv_chunk < chunk, cut to the document-spanning part -- the sequence-aware
+ * transfer of the HSAP abstract, instead of a ring that passes every chunk. */
+int sap_plan_rank_spans(sap_plan_t plan, int32_t chunk, int64_t* spans, int32_t* n_spans);
+
 /* Canonical item list; host memory owned by the plan. */
 int sap_plan_items(sap_plan_t plan, const sap_item_t** items, int64_t* n_items);
 
@@ -171,6 +229,25 @@ int sap_merge(sap_plan_t plan, const void* workspace, size_t ws_bytes, int32_t h
 int sap_attn_bwd(sap_plan_t plan, const void* q, const void* k, const void* v, const void* o, const float* lse,
                  const void* dout, int32_t hq, int32_t hkv, int32_t head_dim, float softmax_scale, void* dq,
                  void* dk, void* dv, void* workspace, size_t ws_bytes, void* stream);
+
+/* Byte offsets, inside the backward workspace, of the fp32 dK and dV accumulators that
+ * sap_attn_bwd leaves behind: [rows][hkv][head_dim] each, row r = token kv_begin + r of the plan's
+ * window (row stride hkv * head_dim floats).  Under sequence parallelism the rows below q_begin
+ * hold this device's partial dK/dV for other devices' tokens: sent to their owners and added
+ * there with sap_attn_bwd_kv_add. */
+int sap_workspace_kv_offsets(sap_plan_t plan, int32_t hq, int32_t hkv, int32_t head_dim, size_t* dk_offset,
+                             size_t* dv_offset);
+
+/* Adds received fp32 partial gradients into the dK/dV accumulators that the last sap_attn_bwd with
+ * this plan and workspace left behind, and rewrites the bf16 dK/dV of those rows:
+ *   acc[t] += part[t - row_begin]; dk[t] = bf16(acc_dK[t]); dv[t] = bf16(acc_dV[t])
+ * for tokens t in [row_begin, row_begin + rows), which must lie in the plan's key/value window
+ * (SAP_ERR_INVALID_ARG otherwise).  dk_part, dv_part: fp32 [rows][hkv][head_dim], 16-byte
+ * aligned; dk, dv: the bf16 window buffers sap_attn_bwd wrote.  Several calls add up (the chunk
+ * pair gradients of the backward add, as on one device); calls on one stream are ordered. */
+int sap_attn_bwd_kv_add(sap_plan_t plan, void* workspace, size_t ws_bytes, int32_t hq, int32_t hkv, int32_t head_dim,
+                        const float* dk_part, const float* dv_part, int64_t row_begin, int64_t rows, void* dk,
+                        void* dv, void* stream);
 
 /* Forward + merge (the same kernels as sap_attn_fwd followed by sap_merge)
  * without any device allocation: the partial outputs and LSEs live in a

@@ -18,18 +18,27 @@ from ._capi import (  # noqa: F401
     library_path,
     load_library,
     sap_attn_bwd,
+    sap_attn_bwd_kv_add,
     sap_attn_fwd,
     sap_attn_fwd_static_scratch,
     sap_device_status,
     sap_error_string,
+    sap_balanced_chunks,
     sap_merge,
     sap_plan,
     sap_plan_bwd_schedule,
+    sap_plan_chunk_bounds,
+    sap_plan_chunk_stats,
+    sap_plan_chunks,
     sap_plan_destroy,
     sap_plan_fwd_schedule,
     sap_plan_items,
+    sap_plan_rank,
+    sap_plan_rank_spans,
     sap_plan_set_fused_merge,
     sap_plan_stats,
     sap_plan_upload,
+    sap_plan_window,
+    sap_workspace_kv_offsets,
     sap_workspace_size,
 )

@@ -43,6 +43,24 @@ def load_library():
     PP = ctypes.POINTER(ctypes.c_void_p)
     L.sap_plan.restype = ctypes.c_int
     L.sap_plan.argtypes = [P, i32, i64, i32, i32, i32, PP]
+    L.sap_plan_chunks.restype = ctypes.c_int
+    L.sap_plan_chunks.argtypes = [P, i32, i64, P, i32, i32, i32, PP]
+    L.sap_balanced_chunks.restype = ctypes.c_int
+    L.sap_balanced_chunks.argtypes = [P, i32, i64, i32, i32, P]
+    L.sap_plan_chunk_bounds.restype = ctypes.c_int
+    L.sap_plan_chunk_bounds.argtypes = [P, PP, ctypes.POINTER(i32)]
+    L.sap_plan_chunk_stats.restype = ctypes.c_int
+    L.sap_plan_chunk_stats.argtypes = [P, P, P]
+    L.sap_plan_rank.restype = ctypes.c_int
+    L.sap_plan_rank.argtypes = [P, i32, PP]
+    L.sap_plan_window.restype = ctypes.c_int
+    L.sap_plan_window.argtypes = [P] + [ctypes.POINTER(i64)] * 4
+    L.sap_plan_rank_spans.restype = ctypes.c_int
+    L.sap_plan_rank_spans.argtypes = [P, i32, P, ctypes.POINTER(i32)]
+    L.sap_workspace_kv_offsets.restype = ctypes.c_int
+    L.sap_workspace_kv_offsets.argtypes = [P, i32, i32, i32, ctypes.POINTER(sz), ctypes.POINTER(sz)]
+    L.sap_attn_bwd_kv_add.restype = ctypes.c_int
+    L.sap_attn_bwd_kv_add.argtypes = [P, P, sz, i32, i32, i32, P, P, i64, i64, P, P, P]
     L.sap_plan_items.restype = ctypes.c_int
     L.sap_plan_items.argtypes = [P, PP, ctypes.POINTER(i64)]
     L.sap_plan_stats.restype = ctypes.c_int
@@ -109,6 +127,69 @@ def sap_plan(cu_seqlens, total_tokens: int, num_chunks: int, block_m: int = 128,
     _check(L.sap_plan(cu.ctypes.data_as(ctypes.c_void_p), len(cu) - 1, int(total_tokens), int(num_chunks),
                       int(block_m), int(block_n), ctypes.byref(h)), "sap_plan")
     return Plan(h.value, int(total_tokens), int(num_chunks), int(block_m), int(block_n))
+
+
+def sap_plan_chunks(cu_seqlens, total_tokens: int, chunk_bounds, block_m: int = 128, block_n: int = 128) -> Plan:
+    """Plan over explicit contiguous chunks [bounds[c], bounds[c+1])."""
+    L = load_library()
+    cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int32))
+    b = np.ascontiguousarray(np.asarray(chunk_bounds, dtype=np.int64))
+    h = ctypes.c_void_p()
+    _check(L.sap_plan_chunks(cu.ctypes.data_as(ctypes.c_void_p), len(cu) - 1, int(total_tokens),
+                             b.ctypes.data_as(ctypes.c_void_p), len(b) - 1, int(block_m), int(block_n),
+                             ctypes.byref(h)), "sap_plan_chunks")
+    return Plan(h.value, int(total_tokens), len(b) - 1, int(block_m), int(block_n))
+
+
+def sap_balanced_chunks(cu_seqlens, total_tokens: int, num_chunks: int, block: int = 128) -> np.ndarray:
+    """Balanced contiguous chunk bounds (int64, num_chunks + 1 entries)."""
+    cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int32))
+    out = np.zeros(int(num_chunks) + 1, dtype=np.int64)
+    _check(load_library().sap_balanced_chunks(cu.ctypes.data_as(ctypes.c_void_p), len(cu) - 1, int(total_tokens),
+                                              int(num_chunks), int(block), out.ctypes.data_as(ctypes.c_void_p)),
+           "sap_balanced_chunks")
+    return out
+
+
+def sap_plan_chunk_bounds(plan: Plan) -> np.ndarray:
+    p, n = ctypes.c_void_p(), ctypes.c_int32()
+    _check(load_library().sap_plan_chunk_bounds(plan.handle, ctypes.byref(p), ctypes.byref(n)),
+           "sap_plan_chunk_bounds")
+    return np.ctypeslib.as_array(ctypes.cast(p, ctypes.POINTER(ctypes.c_int64)), shape=(n.value + 1,)).copy()
+
+
+def sap_plan_chunk_stats(plan: Plan) -> dict:
+    """Per q chunk: items and unmasked pairs (int64 arrays of num_chunks entries)."""
+    nc = len(sap_plan_chunk_bounds(plan)) - 1
+    items = np.zeros(nc, dtype=np.int64)
+    pairs = np.zeros(nc, dtype=np.int64)
+    _check(load_library().sap_plan_chunk_stats(plan.handle, items.ctypes.data_as(ctypes.c_void_p),
+                                               pairs.ctypes.data_as(ctypes.c_void_p)), "sap_plan_chunk_stats")
+    return {"items": items, "pairs": pairs}
+
+
+def sap_plan_rank(plan: Plan, chunk: int) -> Plan:
+    """Rank plan of q chunk `chunk` (windowed buffers, see sap_plan_window)."""
+    h = ctypes.c_void_p()
+    _check(load_library().sap_plan_rank(plan.handle, int(chunk), ctypes.byref(h)), "sap_plan_rank")
+    return Plan(h.value, plan.n, plan.num_chunks, plan.block_m, plan.block_n)
+
+
+def sap_plan_window(plan: Plan) -> dict:
+    """q_begin, q_end, kv_begin, span_begin of the plan's buffer window (global token indices)."""
+    v = [ctypes.c_int64() for _ in range(4)]
+    _check(load_library().sap_plan_window(plan.handle, *[ctypes.byref(x) for x in v]), "sap_plan_window")
+    return dict(zip(("q_begin", "q_end", "kv_begin", "span_begin"), (x.value for x in v)))
+
+
+def sap_plan_rank_spans(plan: Plan, chunk: int) -> np.ndarray:
+    """Token ranges the owner of `chunk` receives: int64 [n, 3] = (source chunk, lo, hi)."""
+    nc = plan.num_chunks
+    out = np.zeros((max(nc, 1), 3), dtype=np.int64)
+    n = ctypes.c_int32()
+    _check(load_library().sap_plan_rank_spans(plan.handle, int(chunk), out.ctypes.data_as(ctypes.c_void_p),
+                                              ctypes.byref(n)), "sap_plan_rank_spans")
+    return out[: n.value].copy()
 
 
 def sap_plan_destroy(plan: Plan):
@@ -219,6 +300,27 @@ def sap_attn_bwd(plan: Plan, q, k, v, o, lse, dout, softmax_scale: float, dq, dk
     _check(load_library().sap_attn_bwd(plan.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), hq,
                                        hkv, d, float(softmax_scale), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace),
                                        _nbytes(workspace), ctypes.c_void_p(_stream_ptr(stream))), "sap_attn_bwd")
+
+
+def sap_workspace_kv_offsets(plan: Plan, hq: int, hkv: int, head_dim: int):
+    """(dk_offset, dv_offset): byte offsets of the fp32 dK / dV accumulators in the backward workspace."""
+    a, b = ctypes.c_size_t(), ctypes.c_size_t()
+    _check(load_library().sap_workspace_kv_offsets(plan.handle, hq, hkv, head_dim, ctypes.byref(a), ctypes.byref(b)),
+           "sap_workspace_kv_offsets")
+    return a.value, b.value
+
+
+def sap_attn_bwd_kv_add(plan: Plan, workspace, hq: int, dk_part, dv_part, row_begin: int, dk, dv, stream=None):
+    """Add fp32 dK/dV partials for tokens [row_begin, row_begin + rows) into the backward's accumulators
+    and rewrite those rows of the bf16 dk, dv."""
+    import torch
+    for t, nme in ((dk_part, "dk_part"), (dv_part, "dv_part")):
+        if t.dtype != torch.float32 or t.dim() != 3 or not t.is_contiguous() or not t.is_cuda:
+            raise ValueError(f"{nme} must be a contiguous CUDA fp32 tensor [rows, hkv, head_dim]")
+    rows, hkv, d = dk_part.shape
+    _check(load_library().sap_attn_bwd_kv_add(plan.handle, _ptr(workspace), _nbytes(workspace), hq, hkv, d,
+                                              _ptr(dk_part), _ptr(dv_part), int(row_begin), int(rows), _ptr(dk),
+                                              _ptr(dv), ctypes.c_void_p(_stream_ptr(stream))), "sap_attn_bwd_kv_add")
 
 
 def sap_attn_fwd_static_scratch(plan: Plan, q, k, v, softmax_scale: float, o, lse, stream=None):

@@ -136,17 +136,37 @@ FwdWs fwd_ws(const sap_plan_s* p, int32_t hq, int32_t hd) {
 }
 struct BwdWs {
   size_t dq_acc = 0, dkv_acc = 0, dvec = 0, lse2 = 0, total = 0;
-  int64_t n_pad = 0;
+  int64_t n_pad = 0, n_pad_kv = 0;  // query-side and key/value-side window rows, rounded up to 128
 };
 BwdWs bwd_ws(const sap_plan_s* p, int32_t hq, int32_t hkv, int32_t hd) {
   BwdWs w;
-  w.n_pad = round_up(p->n, 128);
+  w.n_pad = round_up(p->q_rows(), 128);
+  w.n_pad_kv = round_up(p->kv_rows(), 128);
   w.dq_acc = 0;                                                             // [n_pad][hq][hd] fp32
-  w.dkv_acc = round_up(w.n_pad * hq * hd * 4, 1024);                        // [2][n_pad][hkv][hd] fp32
-  w.dvec = w.dkv_acc + round_up(2 * w.n_pad * hkv * hd * 4, 256);           // [hq][n_pad]
+  w.dkv_acc = round_up(w.n_pad * hq * hd * 4, 1024);                        // [2][n_pad_kv][hkv][hd] fp32
+  w.dvec = w.dkv_acc + round_up(2 * w.n_pad_kv * hkv * hd * 4, 256);        // [hq][n_pad]
   w.lse2 = w.dvec + round_up(w.n_pad * hq * 4, 256);                        // [hq][n_pad]
   w.total = w.lse2 + round_up(w.n_pad * hq * 4, 256);
   return w;
+}
+
+// Forward parameters of a plan's window (everything but the buffers and the error word).
+sap::FwdParams fwd_params(const sap_plan_s* p, int32_t hq, int32_t hkv, float softmax_scale) {
+  const int32_t* base = static_cast<const int32_t*>(p->dev);
+  sap::FwdParams fp{};
+  fp.items = base + p->off_items;
+  fp.units = base + p->off_units;
+  fp.order = base + p->off_order;
+  fp.tok_lo = base + p->off_tok_lo;
+  fp.n_units = (int32_t)(p->fwd_units.size() / 4);
+  fp.hq = hq;
+  fp.group = hq / hkv;
+  fp.q0 = p->q_begin;
+  fp.kv0 = p->kv_begin;
+  fp.q_end = p->q_end;
+  fp.lse_ld = p->q_rows();
+  fp.scale_log2 = softmax_scale * 1.4426950408889634f;
+  return fp;
 }
 
 // Scratch for sap_attn_fwd_static_scratch: the forward's partial outputs and
@@ -186,7 +206,7 @@ int sap_plan(const int32_t* cu_seqlens_host, int32_t num_docs, int64_t total_tok
   if (!p) return SAP_ERR_NOMEM;
   int rc;
   try {
-    rc = sap_plan_build(cu_seqlens_host, num_docs, total_tokens, num_chunks, block_m, block_n, p);
+    rc = sap_plan_build(cu_seqlens_host, num_docs, total_tokens, num_chunks, nullptr, block_m, block_n, p);
   } catch (const std::bad_alloc&) {
     rc = SAP_ERR_NOMEM;
   }
@@ -195,6 +215,108 @@ int sap_plan(const int32_t* cu_seqlens_host, int32_t num_docs, int64_t total_tok
     return rc;
   }
   *out = p;
+  return SAP_OK;
+}
+
+int sap_plan_chunks(const int32_t* cu_seqlens_host, int32_t num_docs, int64_t total_tokens,
+                    const int64_t* chunk_bounds, int32_t num_chunks, int32_t block_m, int32_t block_n,
+                    sap_plan_t* out) {
+  if (!out || !chunk_bounds) return SAP_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (num_chunks < 1) return SAP_ERR_BAD_CHUNKS;
+  sap_plan_s* p = new (std::nothrow) sap_plan_s();
+  if (!p) return SAP_ERR_NOMEM;
+  int rc;
+  try {
+    rc = sap_plan_build(cu_seqlens_host, num_docs, total_tokens, num_chunks, chunk_bounds, block_m, block_n, p);
+  } catch (const std::bad_alloc&) {
+    rc = SAP_ERR_NOMEM;
+  }
+  if (rc != SAP_OK) {
+    delete p;
+    return rc;
+  }
+  *out = p;
+  return SAP_OK;
+}
+
+int sap_balanced_chunks(const int32_t* cu_seqlens_host, int32_t num_docs, int64_t total_tokens, int32_t num_chunks,
+                        int32_t block, int64_t* chunk_bounds) {
+  try {
+    return sap_balanced_bounds(cu_seqlens_host, num_docs, total_tokens, num_chunks, block, chunk_bounds);
+  } catch (const std::bad_alloc&) {
+    return SAP_ERR_NOMEM;
+  }
+}
+
+int sap_plan_rank(sap_plan_t plan, int32_t chunk, sap_plan_t* out) {
+  if (!out) return SAP_ERR_INVALID_ARG;
+  *out = nullptr;
+  sap_plan_s* r = new (std::nothrow) sap_plan_s();
+  if (!r) return SAP_ERR_NOMEM;
+  int rc;
+  try {
+    rc = sap_plan_build_rank(plan, chunk, r);
+  } catch (const std::bad_alloc&) {
+    rc = SAP_ERR_NOMEM;
+  }
+  if (rc != SAP_OK) {
+    delete r;
+    return rc;
+  }
+  *out = r;
+  return SAP_OK;
+}
+
+int sap_plan_window(sap_plan_t plan, int64_t* q_begin, int64_t* q_end, int64_t* kv_begin, int64_t* span_begin) {
+  if (!plan) return SAP_ERR_INVALID_ARG;
+  if (q_begin) *q_begin = plan->q_begin;
+  if (q_end) *q_end = plan->q_end;
+  if (kv_begin) *kv_begin = plan->kv_begin;
+  if (span_begin) *span_begin = plan->span_begin;
+  return SAP_OK;
+}
+
+int sap_plan_chunk_bounds(sap_plan_t plan, const int64_t** bounds, int32_t* num_chunks) {
+  if (!plan) return SAP_ERR_INVALID_ARG;
+  if (bounds) *bounds = plan->bounds.data();
+  if (num_chunks) *num_chunks = plan->num_chunks;
+  return SAP_OK;
+}
+
+int sap_plan_chunk_stats(sap_plan_t plan, int64_t* items_per_chunk, int64_t* pairs_per_chunk) {
+  if (!plan) return SAP_ERR_INVALID_ARG;
+  const int32_t P = plan->num_chunks;
+  if (items_per_chunk) {
+    for (int32_t c = 0; c < P; ++c) items_per_chunk[c] = 0;
+    for (const auto& it : plan->items) items_per_chunk[it.q_chunk]++;
+  }
+  if (pairs_per_chunk) {
+    for (int32_t c = 0; c < P; ++c) {
+      pairs_per_chunk[c] = 0;
+      const int64_t a = plan->bounds[c] > plan->q_begin ? plan->bounds[c] : plan->q_begin;
+      const int64_t b = plan->bounds[c + 1] < plan->q_end ? plan->bounds[c + 1] : plan->q_end;
+      for (int64_t i = a; i < b; ++i) pairs_per_chunk[c] += i - plan->tok_lo[i] + 1;
+    }
+  }
+  return SAP_OK;
+}
+
+int sap_plan_rank_spans(sap_plan_t plan, int32_t chunk, int64_t* spans, int32_t* n_spans) {
+  if (!plan || !spans || !n_spans || plan->rank_chunk >= 0 || chunk < 0 || chunk >= plan->num_chunks)
+    return SAP_ERR_INVALID_ARG;
+  const int64_t q0 = plan->bounds[chunk];
+  const int64_t s0 = q0 < plan->n ? plan->tok_lo[q0] : q0;
+  int32_t k = 0;
+  for (int32_t b = 0; b < chunk; ++b) {
+    const int64_t lo = s0 > plan->bounds[b] ? s0 : plan->bounds[b];
+    const int64_t hi = q0 < plan->bounds[b + 1] ? q0 : plan->bounds[b + 1];
+    if (lo < hi) {
+      spans[3 * k] = b, spans[3 * k + 1] = lo, spans[3 * k + 2] = hi;
+      ++k;
+    }
+  }
+  *n_spans = k;
   return SAP_OK;
 }
 
@@ -309,6 +431,17 @@ void sap_plan_destroy(sap_plan_t plan) {
   delete plan;
 }
 
+int sap_workspace_kv_offsets(sap_plan_t plan, int32_t hq, int32_t hkv, int32_t head_dim, size_t* dk_offset,
+                             size_t* dv_offset) {
+  if (!plan) return SAP_ERR_INVALID_ARG;
+  int rc = check_heads(hq, hkv, head_dim);
+  if (rc) return rc;
+  const BwdWs ws = bwd_ws(plan, hq, hkv, head_dim);
+  if (dk_offset) *dk_offset = ws.dkv_acc;
+  if (dv_offset) *dv_offset = ws.dkv_acc + (size_t)ws.n_pad_kv * hkv * head_dim * 4;
+  return SAP_OK;
+}
+
 int sap_workspace_size(sap_plan_t plan, int32_t hq, int32_t hkv, int32_t head_dim, int32_t which, size_t* bytes) {
   if (!plan || !bytes) return SAP_ERR_INVALID_ARG;
   int rc = check_heads(hq, hkv, head_dim);
@@ -328,7 +461,7 @@ int sap_attn_fwd(sap_plan_t p, const void* q, const void* k, const void* v, int3
   int rc = check_kernel_plan(p);
   if (rc) return rc;
   if ((rc = check_heads(hq, hkv, head_dim))) return rc;
-  if (p->n == 0) return SAP_OK;
+  if (p->q_rows() == 0) return SAP_OK;
   if (!q || !k || !v || !o || !lse) return SAP_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
     return SAP_ERR_INVALID_ARG;
@@ -339,20 +472,10 @@ int sap_attn_fwd(sap_plan_t p, const void* q, const void* k, const void* v, int3
   if ((rc = device_info(&di))) return rc;
   if ((rc = sap_plan_upload(p, stream))) return rc;
   CUtensorMap tq, tk, tv;
-  if ((rc = make_map(&tq, q, p->n, hq, head_dim))) return rc;
-  if ((rc = make_map(&tk, k, p->n, hkv, head_dim))) return rc;
-  if ((rc = make_map(&tv, v, p->n, hkv, head_dim))) return rc;
-  const int32_t* base = static_cast<const int32_t*>(p->dev);
-  sap::FwdParams fp;
-  fp.items = base + p->off_items;
-  fp.units = base + p->off_units;
-  fp.order = base + p->off_order;
-  fp.tok_lo = base + p->off_tok_lo;
-  fp.n_units = (int32_t)(p->fwd_units.size() / 4);
-  fp.hq = hq;
-  fp.group = hq / hkv;
-  fp.n = p->n;
-  fp.scale_log2 = softmax_scale * 1.4426950408889634f;
+  if ((rc = make_map(&tq, q, p->q_rows(), hq, head_dim))) return rc;
+  if ((rc = make_map(&tk, k, p->kv_rows(), hkv, head_dim))) return rc;
+  if ((rc = make_map(&tv, v, p->kv_rows(), hkv, head_dim))) return rc;
+  sap::FwdParams fp = fwd_params(p, hq, hkv, softmax_scale);
   fp.o = static_cast<__nv_bfloat16*>(o);
   fp.lse = lse;
   uint8_t* wsb = static_cast<uint8_t*>(workspace);
@@ -376,7 +499,7 @@ int sap_merge(sap_plan_t p, const void* workspace, size_t ws_bytes, int32_t hq, 
   if (hq <= 0) return SAP_ERR_INVALID_ARG;
   if (head_dim != 64 && head_dim != 128) return SAP_ERR_UNSUPPORTED;
   const int64_t n_merges = (int64_t)p->merges.size() / 3;
-  if (p->n == 0 || n_merges == 0) return SAP_OK;
+  if (p->q_rows() == 0 || n_merges == 0) return SAP_OK;
   if (!o || !lse || !aligned16(o)) return SAP_ERR_INVALID_ARG;
   const FwdWs ws = fwd_ws(p, hq, head_dim);
   if (!workspace || ws_bytes < ws.total || !aligned16(workspace)) return SAP_ERR_WORKSPACE;
@@ -387,11 +510,10 @@ int sap_merge(sap_plan_t p, const void* workspace, size_t ws_bytes, int32_t hq, 
   const float* lp = reinterpret_cast<const float*>(wsb + ws.lse_part);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e =
-      head_dim == 64
-          ? sap::launch_merge<64>(base + p->off_merges, n_merges, hq, p->n, op, lp, static_cast<__nv_bfloat16*>(o),
-                                  lse, s)
-          : sap::launch_merge<128>(base + p->off_merges, n_merges, hq, p->n, op, lp,
-                                   static_cast<__nv_bfloat16*>(o), lse, s);
+      head_dim == 64 ? sap::launch_merge<64>(base + p->off_merges, n_merges, hq, p->q_begin, p->q_end, op, lp,
+                                             static_cast<__nv_bfloat16*>(o), lse, s)
+                     : sap::launch_merge<128>(base + p->off_merges, n_merges, hq, p->q_begin, p->q_end, op, lp,
+                                              static_cast<__nv_bfloat16*>(o), lse, s);
   if (e != cudaSuccess) return cuda_fail(e);
   return SAP_OK;
 }
@@ -402,7 +524,7 @@ int sap_attn_bwd(sap_plan_t p, const void* q, const void* k, const void* v, cons
   int rc = check_kernel_plan(p);
   if (rc) return rc;
   if ((rc = check_heads(hq, hkv, head_dim))) return rc;
-  if (p->n == 0) return SAP_OK;
+  if (p->q_rows() == 0) return SAP_OK;
   if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return SAP_ERR_INVALID_ARG;
   const void* ptrs[] = {q, k, v, o, lse, dout, dq, dk, dv};
   for (const void* ptr : ptrs)
@@ -413,10 +535,10 @@ int sap_attn_bwd(sap_plan_t p, const void* q, const void* k, const void* v, cons
   if ((rc = device_info(&di))) return rc;
   if ((rc = sap_plan_upload(p, stream))) return rc;
   CUtensorMap tq, tk, tv, tdo;
-  if ((rc = make_map(&tq, q, p->n, hq, head_dim))) return rc;
-  if ((rc = make_map(&tk, k, p->n, hkv, head_dim))) return rc;
-  if ((rc = make_map(&tv, v, p->n, hkv, head_dim))) return rc;
-  if ((rc = make_map(&tdo, dout, p->n, hq, head_dim))) return rc;
+  if ((rc = make_map(&tq, q, p->q_rows(), hq, head_dim))) return rc;
+  if ((rc = make_map(&tk, k, p->kv_rows(), hkv, head_dim))) return rc;
+  if ((rc = make_map(&tv, v, p->kv_rows(), hkv, head_dim))) return rc;
+  if ((rc = make_map(&tdo, dout, p->q_rows(), hq, head_dim))) return rc;
   uint8_t* wsb = static_cast<uint8_t*>(workspace);
   float* dq_acc = reinterpret_cast<float*>(wsb + ws.dq_acc);
   float* dkv_acc = reinterpret_cast<float*>(wsb + ws.dkv_acc);
@@ -425,15 +547,16 @@ int sap_attn_bwd(sap_plan_t p, const void* q, const void* k, const void* v, cons
   if ((rc = head_dim == 128 ? make_map_f32_tile(&tdq, dq_acc, ws.n_pad, hq, head_dim)
                             : make_map_f32_sw128(&tdq, dq_acc, ws.n_pad, hq, head_dim)))
     return rc;
-  if ((rc = make_map_f32_sw128(&tdkv, dkv_acc, 2 * ws.n_pad, hkv, head_dim))) return rc;
+  if ((rc = make_map_f32_sw128(&tdkv, dkv_acc, 2 * ws.n_pad_kv, hkv, head_dim))) return rc;
   float* dvec = reinterpret_cast<float*>(wsb + ws.dvec);
   float* lse2 = reinterpret_cast<float*>(wsb + ws.lse2);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const __nv_bfloat16* ob = static_cast<const __nv_bfloat16*>(o);
   const __nv_bfloat16* dob = static_cast<const __nv_bfloat16*>(dout);
-  cudaError_t e = head_dim == 64
-                      ? sap::launch_bwd_pre<64>(ob, dob, lse, p->n, ws.n_pad, hq, hkv, dvec, lse2, dq_acc, dkv_acc, s)
-                      : sap::launch_bwd_pre<128>(ob, dob, lse, p->n, ws.n_pad, hq, hkv, dvec, lse2, dq_acc, dkv_acc, s);
+  cudaError_t e = head_dim == 64 ? sap::launch_bwd_pre<64>(ob, dob, lse, p->q_rows(), ws.n_pad, ws.n_pad_kv, hq, hkv,
+                                                           dvec, lse2, dq_acc, dkv_acc, s)
+                                 : sap::launch_bwd_pre<128>(ob, dob, lse, p->q_rows(), ws.n_pad, ws.n_pad_kv, hq, hkv,
+                                                            dvec, lse2, dq_acc, dkv_acc, s);
   if (e != cudaSuccess) return cuda_fail(e);
   const int32_t* base = static_cast<const int32_t*>(p->dev);
   sap::BwdParams bp;
@@ -444,8 +567,11 @@ int sap_attn_bwd(sap_plan_t p, const void* q, const void* k, const void* v, cons
   bp.hq = hq;
   bp.hkv = hkv;
   bp.group = hq / hkv;
-  bp.n = p->n;
+  bp.q0 = p->q_begin;
+  bp.kv0 = p->kv_begin;
+  bp.q_end = p->q_end;
   bp.n_pad = ws.n_pad;
+  bp.n_pad_kv = ws.n_pad_kv;
   bp.scale_log2 = softmax_scale * 1.4426950408889634f;
   bp.scale = softmax_scale;
   bp.lse2 = lse2;
@@ -459,9 +585,31 @@ int sap_attn_bwd(sap_plan_t p, const void* q, const void* k, const void* v, cons
                        : sap::launch_bwd<128>(tq, tk, tv, tdo, tdq, tdkv, bp, grid, s);
     if (e != cudaSuccess) return cuda_fail(e);
   }
-  e = sap::launch_bwd_post(dq_acc, static_cast<__nv_bfloat16*>(dq), p->n * hq * head_dim, dkv_acc,
-                           static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv), p->n * hkv * head_dim,
-                           ws.n_pad * hkv * head_dim, s);
+  e = sap::launch_bwd_post(dq_acc, static_cast<__nv_bfloat16*>(dq), p->q_rows() * hq * head_dim, dkv_acc,
+                           static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv),
+                           p->kv_rows() * hkv * head_dim, ws.n_pad_kv * hkv * head_dim, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return SAP_OK;
+}
+
+int sap_attn_bwd_kv_add(sap_plan_t p, void* workspace, size_t ws_bytes, int32_t hq, int32_t hkv, int32_t head_dim,
+                        const float* dk_part, const float* dv_part, int64_t row_begin, int64_t rows, void* dk,
+                        void* dv, void* stream) {
+  if (!p) return SAP_ERR_INVALID_ARG;
+  int rc = check_heads(hq, hkv, head_dim);
+  if (rc) return rc;
+  if (rows == 0) return SAP_OK;
+  if (rows < 0 || row_begin < p->kv_begin || row_begin + rows > p->q_end) return SAP_ERR_INVALID_ARG;
+  if (!dk_part || !dv_part || !dk || !dv || !aligned16(dk_part) || !aligned16(dv_part) || !aligned16(dk) ||
+      !aligned16(dv))
+    return SAP_ERR_INVALID_ARG;
+  const BwdWs ws = bwd_ws(p, hq, hkv, head_dim);
+  if (!workspace || ws_bytes < ws.total || !aligned16(workspace)) return SAP_ERR_WORKSPACE;
+  float* dkv_acc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + ws.dkv_acc);
+  const int64_t row_elems = (int64_t)hkv * head_dim;
+  cudaError_t e = sap::launch_kv_add(dkv_acc, ws.n_pad_kv * row_elems, dk_part, dv_part, row_begin - p->kv_begin,
+                                     rows, row_elems, static_cast<__nv_bfloat16*>(dk),
+                                     static_cast<__nv_bfloat16*>(dv), static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e);
   return SAP_OK;
 }
@@ -504,7 +652,7 @@ int sap_attn_fwd_static_scratch(sap_plan_t p, const void* q, const void* k, cons
   int rc = check_kernel_plan(p);
   if (rc) return rc;
   if ((rc = check_heads(hq, hkv, head_dim))) return rc;
-  if (p->n == 0) return SAP_OK;
+  if (p->q_rows() == 0) return SAP_OK;
   if (!q || !k || !v || !o || !lse) return SAP_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
     return SAP_ERR_INVALID_ARG;
@@ -520,21 +668,12 @@ int sap_attn_fwd_static_scratch(sap_plan_t p, const void* q, const void* k, cons
   void* scratch = nullptr;
   if ((rc = static_scratch_address(&scratch))) return rc;
   CUtensorMap tq, tk, tv;
-  if ((rc = make_map(&tq, q, p->n, hq, head_dim))) return rc;
-  if ((rc = make_map(&tk, k, p->n, hkv, head_dim))) return rc;
-  if ((rc = make_map(&tv, v, p->n, hkv, head_dim))) return rc;
+  if ((rc = make_map(&tq, q, p->q_rows(), hq, head_dim))) return rc;
+  if ((rc = make_map(&tk, k, p->kv_rows(), hkv, head_dim))) return rc;
+  if ((rc = make_map(&tv, v, p->kv_rows(), hkv, head_dim))) return rc;
   const int32_t* base = static_cast<const int32_t*>(p->dev);
   uint8_t* wsb = static_cast<uint8_t*>(scratch);
-  sap::FwdParams fp;
-  fp.items = base + p->off_items;
-  fp.units = base + p->off_units;
-  fp.order = base + p->off_order;
-  fp.tok_lo = base + p->off_tok_lo;
-  fp.n_units = (int32_t)(p->fwd_units.size() / 4);
-  fp.hq = hq;
-  fp.group = hq / hkv;
-  fp.n = p->n;
-  fp.scale_log2 = softmax_scale * 1.4426950408889634f;
+  sap::FwdParams fp = fwd_params(p, hq, hkv, softmax_scale);
   fp.o = static_cast<__nv_bfloat16*>(o);
   fp.lse = lse;
   // Every (slot, head, row) partial that the merge reads is written by this
@@ -552,10 +691,10 @@ int sap_attn_fwd_static_scratch(sap_plan_t p, const void* q, const void* k, cons
   if (e != cudaSuccess) return cuda_fail(e);
   const int64_t n_merges = (int64_t)p->merges.size() / 3;
   if (n_merges > 0) {
-    e = head_dim == 64 ? sap::launch_merge<64>(base + p->off_merges, n_merges, hq, p->n, fp.o_part, fp.lse_part,
-                                               fp.o, lse, s)
-                       : sap::launch_merge<128>(base + p->off_merges, n_merges, hq, p->n, fp.o_part, fp.lse_part,
-                                                fp.o, lse, s);
+    e = head_dim == 64 ? sap::launch_merge<64>(base + p->off_merges, n_merges, hq, p->q_begin, p->q_end, fp.o_part,
+                                               fp.lse_part, fp.o, lse, s)
+                       : sap::launch_merge<128>(base + p->off_merges, n_merges, hq, p->q_begin, p->q_end,
+                                                fp.o_part, fp.lse_part, fp.o, lse, s);
     if (e != cudaSuccess) return cuda_fail(e);
   }
   return SAP_OK;

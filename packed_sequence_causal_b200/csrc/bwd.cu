@@ -168,13 +168,14 @@ __global__ void __launch_bounds__(448, 1)
         if (!mbar_wait(kv_empty, (unit_iter & 1) ^ 1, guard, kErrTimeoutLoad)) break;
         mbar_arrive_expect_tx(kv_full, 2 * C::TILE);
         for (int b = 0; b < D / 64; ++b) {
-          tma_load_3d(smem + C::OFF_K + b * C::BOX, &tmK, kv_full, 64 * b, g, kt * 128);
-          tma_load_3d(smem + C::OFF_V + b * C::BOX, &tmV, kv_full, 64 * b, g, kt * 128);
+          tma_load_3d(smem + C::OFF_K + b * C::BOX, &tmK, kv_full, 64 * b, g, kt * 128 - (int)p.kv0);
+          tma_load_3d(smem + C::OFF_V + b * C::BOX, &tmV, kv_full, 64 * b, g, kt * 128 - (int)p.kv0);
         }
         // entries are walked q-tile outer, head inner; the next q tile is fetched one entry ahead
         int qt_next = p.entries[2 * e0];
         for (int e = 0; e < ne && ok; ++e) {
           const int qt = qt_next;
+          const int qrow = qt * 128 - (int)p.q0;  // first row of the q tile in the query-side buffers
           if (e + 1 < ne) qt_next = p.entries[2 * (e0 + e + 1)];
           for (int hh = 0; hh < G; ++hh) {
             const int h = g * G + hh;
@@ -184,11 +185,11 @@ __global__ void __launch_bounds__(448, 1)
             uint8_t* st = smem + C::OFF_ST + s * C::STAGE;
             mbar_arrive_expect_tx(q_full + s, C::STAGE);
             for (int b = 0; b < D / 64; ++b) {
-              tma_load_3d(st + b * C::BOX, &tmQ, q_full + s, 64 * b, h, qt * 128);
-              tma_load_3d(st + C::TILE + b * C::BOX, &tmDO, q_full + s, 64 * b, h, qt * 128);
+              tma_load_3d(st + b * C::BOX, &tmQ, q_full + s, 64 * b, h, qrow);
+              tma_load_3d(st + C::TILE + b * C::BOX, &tmDO, q_full + s, 64 * b, h, qrow);
             }
-            bulk_load(st + 2 * C::TILE, p.lse2 + (size_t)h * p.n_pad + (size_t)qt * 128, C::VEC, q_full + s);
-            bulk_load(st + 2 * C::TILE + C::VEC, p.dvec + (size_t)h * p.n_pad + (size_t)qt * 128, C::VEC,
+            bulk_load(st + 2 * C::TILE, p.lse2 + (size_t)h * p.n_pad + (size_t)qrow, C::VEC, q_full + s);
+            bulk_load(st + 2 * C::TILE + C::VEC, p.dvec + (size_t)h * p.n_pad + (size_t)qrow, C::VEC,
                       q_full + s);
             ++q_iter;
           }
@@ -302,7 +303,7 @@ __global__ void __launch_bounds__(448, 1)
       const int u = w / p.hkv;
       const int kt = p.kv_units[3 * u], e0 = p.kv_units[3 * u + 1], ne = p.kv_units[3 * u + 2];
       const int64_t jrow = (int64_t)kt * 128 + t;
-      const bool real_row = jrow < p.n;
+      const bool real_row = jrow < p.q_end;
       const int j_lo = real_row ? (int)jrow : 1;  // queries i with j <= i <= last token of the document
       const int j_hi = real_row ? p.tok_hi[jrow] : 0;
       int qt_next = p.entries[2 * e0], tag_next = p.entries[2 * e0 + 1];
@@ -427,7 +428,7 @@ __global__ void __launch_bounds__(448, 1)
             mbar_arrive(dq_free);  // all of dQ^T is in registers or staged: R2 may take the next dP^T
             if (!mbar_wait_warp(stg_ready, hs & 1, guard, kErrTimeoutEpilogue)) { ok = false; break; }
             if (t == 0) {
-              tma_reduce_add_3d(&tmDQ, stg, 0, h, qt * 128);
+              tma_reduce_add_3d(&tmDQ, stg, 0, h, qt * 128 - (int)p.q0);
               bulk_commit_group();
               bulk_wait_group_read0();
               mbar_arrive(stg_free);
@@ -443,7 +444,7 @@ __global__ void __launch_bounds__(448, 1)
             mbar_arrive(stg_ready);
             if (!mbar_wait_warp(stg_ready, hs & 1, guard, kErrTimeoutEpilogue)) { ok = false; break; }
             if (t == 0) {
-              tma_reduce_add_3d(&tmDQ, stg, 0, h, qt * 128 + 64);
+              tma_reduce_add_3d(&tmDQ, stg, 0, h, qt * 128 - (int)p.q0 + 64);
               bulk_commit_group();
               bulk_wait_group_read0();
               mbar_arrive(stg_free);
@@ -475,8 +476,8 @@ __global__ void __launch_bounds__(448, 1)
             mbar_arrive(stg_ready);
             if (!mbar_wait_warp(stg_ready, hs & 1, guard, kErrTimeoutEpilogue)) { ok = false; break; }
             if (t == 0) {
-              tma_reduce_add_3d(&tmDQ, epi, 0, h, qt * 128);
-              tma_reduce_add_3d(&tmDQ, epi + C::EPI_BYTES / 2, 32, h, qt * 128);
+              tma_reduce_add_3d(&tmDQ, epi, 0, h, qt * 128 - (int)p.q0);
+              tma_reduce_add_3d(&tmDQ, epi + C::EPI_BYTES / 2, 32, h, qt * 128 - (int)p.q0);
               bulk_commit_group();
               bulk_wait_group_read0();
               mbar_arrive(stg_free);
@@ -520,7 +521,7 @@ __global__ void __launch_bounds__(448, 1)
         mbar_arrive(stg_ready);
         if (!mbar_wait_warp(stg_ready, hs & 1, guard, kErrTimeoutEpilogue)) { ok = false; break; }
         if (t == 0) {
-          const int row0 = (which == 0 ? 0 : (int)p.n_pad) + kt * 128;
+          const int row0 = (which == 0 ? 0 : (int)p.n_pad_kv) + kt * 128 - (int)p.kv0;
           tma_reduce_add_3d(&tmDKV, epi, 64 * cb, g, row0);
           tma_reduce_add_3d(&tmDKV, epi + C::EPI_BYTES / 2, 64 * cb + 32, g, row0);
           bulk_commit_group();

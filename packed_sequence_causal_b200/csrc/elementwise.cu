@@ -55,11 +55,12 @@ struct Vec<4> {
   }
 };
 
-// Merge of the partials of one q-tile: warp = (merge entry, head, row).
+// Merge of the partials of one q-tile: warp = (merge entry, head, row).  O and LSE hold the
+// query rows [q0, q_end) (global token indices); LSE's row stride is q_end - q0.
 template <int D>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32)
-    merge_kernel(const int32_t* merges, int64_t n_merges, int32_t hq, int64_t n, const float* o_part,
-                 const float* lse_part, __nv_bfloat16* o, float* lse) {
+    merge_kernel(const int32_t* merges, int64_t n_merges, int32_t hq, int64_t q0, int64_t q_end,
+                 const float* o_part, const float* lse_part, __nv_bfloat16* o, float* lse) {
   constexpr int E = D / 32;
   const int64_t wid = (int64_t)blockIdx.x * kWarpsPerBlock + threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
@@ -67,8 +68,9 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
   const int64_t mi = wid / (hq * 128);
   const int h = (int)((wid / 128) % hq), r = (int)(wid % 128);
   const int qt = merges[3 * mi], s0 = merges[3 * mi + 1], ns = merges[3 * mi + 2];
-  const int64_t i = (int64_t)qt * 128 + r;
-  if (i >= n) return;
+  const int64_t gi = (int64_t)qt * 128 + r;
+  if (gi >= q_end) return;
+  const int64_t i = gi - q0, n = q_end - q0;  // row in the window, window rows
   float mx = -INFINITY;
   for (int b = 0; b < ns; ++b) mx = fmaxf(mx, lse_part[((size_t)(s0 + b) * hq + h) * 128 + r]);
   float acc[E];
@@ -105,24 +107,26 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
   if (lane == 0) lse[(size_t)h * n + i] = lse_all;
 }
 
-// D_i = <dO_i, O_i>, LSE_i * log2(e), and zeroed accumulator rows (dQ for every head, dK and dV
-// for the kv heads): warp = (row, head).
+// D_i = <dO_i, O_i>, LSE_i * log2(e), and zeroed accumulator rows (dQ for every head of the n_pad
+// query rows, dK and dV for the kv heads of the n_pad_kv key/value rows): warp = (row, head), over
+// max(n_pad, n_pad_kv) rows.
 template <int D>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32)
     bwd_pre_kernel(const __nv_bfloat16* o, const __nv_bfloat16* dout, const float* lse, int64_t n, int64_t n_pad,
-                   int32_t hq, int32_t hkv, float* dvec, float* lse2, float* dq_acc, float* dkv_acc) {
+                   int64_t n_pad_kv, int32_t hq, int32_t hkv, float* dvec, float* lse2, float* dq_acc,
+                   float* dkv_acc) {
   constexpr int E = D / 32;
   const int64_t wid = (int64_t)blockIdx.x * kWarpsPerBlock + threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
-  if (wid >= n_pad * hq) return;
   const int64_t i = wid / hq;
   const int h = (int)(wid % hq);
-  Vec<E>::store_zero(dq_acc + (size_t)wid * D + lane * E);
-  if (h < hkv) {
+  if (i < n_pad_kv && h < hkv) {
     const size_t kv_row = ((size_t)i * hkv + h) * D + lane * E;
     Vec<E>::store_zero(dkv_acc + kv_row);
-    Vec<E>::store_zero(dkv_acc + (size_t)n_pad * hkv * D + kv_row);
+    Vec<E>::store_zero(dkv_acc + (size_t)n_pad_kv * hkv * D + kv_row);
   }
+  if (i >= n_pad) return;
+  Vec<E>::store_zero(dq_acc + (size_t)wid * D + lane * E);
   float dsum = 0.f;
   if (i < n) {
     float a[E], b[E];
@@ -159,28 +163,63 @@ __global__ void bwd_post_kernel(const float* dq_acc, __nv_bfloat16* dq, int64_t 
   Vec<4>::store_bf16(dst, v);
 }
 
+// Received fp32 dK/dV partials added into rows of the fp32 accumulators, and those rows
+// rewritten as bf16: four values per thread, dK then dV.
+__global__ void kv_add_kernel(float* dkv_acc, int64_t dv_offset, const float* dk_part, const float* dv_part,
+                              int64_t base, int64_t count4, __nv_bfloat16* dk, __nv_bfloat16* dv) {
+  int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  float* acc;
+  const float* part;
+  __nv_bfloat16* dst;
+  if (t < count4) {
+    acc = dkv_acc + base + 4 * t, part = dk_part + 4 * t, dst = dk + base + 4 * t;
+  } else if ((t -= count4) < count4) {
+    acc = dkv_acc + dv_offset + base + 4 * t, part = dv_part + 4 * t, dst = dv + base + 4 * t;
+  } else {
+    return;
+  }
+  float a[4], b[4];
+  Vec<4>::load(acc, a);
+  Vec<4>::load(part, b);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) a[e] += b[e];
+  *reinterpret_cast<float4*>(acc) = make_float4(a[0], a[1], a[2], a[3]);
+  Vec<4>::store_bf16(dst, a);
+}
+
 }  // namespace
 
 template <int D>
-cudaError_t launch_merge(const int32_t* merges, int64_t n_merges, int32_t hq, int64_t n, const float* o_part,
-                         const float* lse_part, __nv_bfloat16* o, float* lse, cudaStream_t stream) {
+cudaError_t launch_merge(const int32_t* merges, int64_t n_merges, int32_t hq, int64_t q0, int64_t q_end,
+                         const float* o_part, const float* lse_part, __nv_bfloat16* o, float* lse,
+                         cudaStream_t stream) {
   const int64_t warps = n_merges * hq * 128;
   if (warps == 0) return cudaSuccess;
   const int64_t blocks = (warps + kWarpsPerBlock - 1) / kWarpsPerBlock;
-  merge_kernel<D><<<(unsigned)blocks, kWarpsPerBlock * 32, 0, stream>>>(merges, n_merges, hq, n, o_part, lse_part, o,
-                                                                        lse);
+  merge_kernel<D><<<(unsigned)blocks, kWarpsPerBlock * 32, 0, stream>>>(merges, n_merges, hq, q0, q_end, o_part,
+                                                                        lse_part, o, lse);
   return cudaGetLastError();
 }
 
 template <int D>
 cudaError_t launch_bwd_pre(const __nv_bfloat16* o, const __nv_bfloat16* dout, const float* lse, int64_t n,
-                           int64_t n_pad, int32_t hq, int32_t hkv, float* dvec, float* lse2, float* dq_acc,
-                           float* dkv_acc, cudaStream_t stream) {
-  const int64_t warps = n_pad * hq;
+                           int64_t n_pad, int64_t n_pad_kv, int32_t hq, int32_t hkv, float* dvec, float* lse2,
+                           float* dq_acc, float* dkv_acc, cudaStream_t stream) {
+  const int64_t warps = (n_pad > n_pad_kv ? n_pad : n_pad_kv) * hq;
   if (warps == 0) return cudaSuccess;
   const int64_t blocks = (warps + kWarpsPerBlock - 1) / kWarpsPerBlock;
-  bwd_pre_kernel<D><<<(unsigned)blocks, kWarpsPerBlock * 32, 0, stream>>>(o, dout, lse, n, n_pad, hq, hkv, dvec,
-                                                                          lse2, dq_acc, dkv_acc);
+  bwd_pre_kernel<D><<<(unsigned)blocks, kWarpsPerBlock * 32, 0, stream>>>(o, dout, lse, n, n_pad, n_pad_kv, hq, hkv,
+                                                                          dvec, lse2, dq_acc, dkv_acc);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_kv_add(float* dkv_acc, int64_t dv_offset, const float* dk_part, const float* dv_part,
+                          int64_t row0, int64_t rows, int64_t row_elems, __nv_bfloat16* dk, __nv_bfloat16* dv,
+                          cudaStream_t stream) {
+  const int64_t count4 = rows * row_elems / 4;
+  if (count4 == 0) return cudaSuccess;
+  kv_add_kernel<<<(unsigned)((2 * count4 + 255) / 256), 256, 0, stream>>>(dkv_acc, dv_offset, dk_part, dv_part,
+                                                                          row0 * row_elems, count4, dk, dv);
   return cudaGetLastError();
 }
 
@@ -194,13 +233,13 @@ cudaError_t launch_bwd_post(const float* dq_acc, __nv_bfloat16* dq, int64_t coun
   return cudaGetLastError();
 }
 
-template cudaError_t launch_merge<64>(const int32_t*, int64_t, int32_t, int64_t, const float*, const float*,
-                                      __nv_bfloat16*, float*, cudaStream_t);
-template cudaError_t launch_merge<128>(const int32_t*, int64_t, int32_t, int64_t, const float*, const float*,
-                                       __nv_bfloat16*, float*, cudaStream_t);
+template cudaError_t launch_merge<64>(const int32_t*, int64_t, int32_t, int64_t, int64_t, const float*,
+                                      const float*, __nv_bfloat16*, float*, cudaStream_t);
+template cudaError_t launch_merge<128>(const int32_t*, int64_t, int32_t, int64_t, int64_t, const float*,
+                                       const float*, __nv_bfloat16*, float*, cudaStream_t);
 template cudaError_t launch_bwd_pre<64>(const __nv_bfloat16*, const __nv_bfloat16*, const float*, int64_t, int64_t,
-                                        int32_t, int32_t, float*, float*, float*, float*, cudaStream_t);
+                                        int64_t, int32_t, int32_t, float*, float*, float*, float*, cudaStream_t);
 template cudaError_t launch_bwd_pre<128>(const __nv_bfloat16*, const __nv_bfloat16*, const float*, int64_t, int64_t,
-                                         int32_t, int32_t, float*, float*, float*, float*, cudaStream_t);
+                                         int64_t, int32_t, int32_t, float*, float*, float*, float*, cudaStream_t);
 
 }  // namespace sap

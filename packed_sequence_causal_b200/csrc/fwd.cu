@@ -116,7 +116,8 @@ __global__ void __launch_bounds__(192, 1)
         const int qt = p.units[4 * u], ib = p.units[4 * u + 1], ic = p.units[4 * u + 2];
         if (!mbar_wait(q_empty, (unit_iter & 1) ^ 1, guard, kErrTimeoutLoad)) break;
         mbar_arrive_expect_tx(q_full, C::QBYTES);
-        for (int b = 0; b < D / 64; ++b) tma_load_3d(smem + C::OFF_Q + b * C::BOX, &tmQ, q_full, 64 * b, h, qt * 128);
+        for (int b = 0; b < D / 64; ++b)
+          tma_load_3d(smem + C::OFF_Q + b * C::BOX, &tmQ, q_full, 64 * b, h, qt * 128 - (int)p.q0);
         for (int t = 0; t < ic; ++t) {
           const int kt = p.items[5 * (ib + t) + 1];
           const int s = kv_iter % C::NS;
@@ -124,11 +125,11 @@ __global__ void __launch_bounds__(192, 1)
           if (!mbar_wait(k_empty + s, ph ^ 1, guard, kErrTimeoutLoad)) { ok = false; break; }
           mbar_arrive_expect_tx(k_full + s, C::KVBYTES);
           for (int b = 0; b < D / 64; ++b)
-            tma_load_3d(smem + C::OFF_K + s * C::KVBYTES + b * C::BOX, &tmK, k_full + s, 64 * b, g, kt * 128);
+            tma_load_3d(smem + C::OFF_K + s * C::KVBYTES + b * C::BOX, &tmK, k_full + s, 64 * b, g, kt * 128 - (int)p.kv0);
           if (!mbar_wait(v_empty + s, ph ^ 1, guard, kErrTimeoutLoad)) { ok = false; break; }
           mbar_arrive_expect_tx(v_full + s, C::KVBYTES);
           for (int b = 0; b < D / 64; ++b)
-            tma_load_3d(smem + C::OFF_V + s * C::KVBYTES + b * C::BOX, &tmV, v_full + s, 64 * b, g, kt * 128);
+            tma_load_3d(smem + C::OFF_V + s * C::KVBYTES + b * C::BOX, &tmV, v_full + s, 64 * b, g, kt * 128 - (int)p.kv0);
           ++kv_iter;
         }
         ++unit_iter;
@@ -214,8 +215,8 @@ __global__ void __launch_bounds__(192, 1)
       const int u = p.order[w / p.hq], h = w % p.hq;
       const int qt = p.units[4 * u], ib = p.units[4 * u + 1], ic = p.units[4 * u + 2], slot = p.units[4 * u + 3];
       const int64_t i = (int64_t)qt * 128 + r;
-      const bool real_row = i < p.n;
-      const int row_lo = real_row ? p.tok_lo[i] : 1;  // empty key range for rows past N
+      const bool real_row = i < p.q_end;
+      const int row_lo = real_row ? p.tok_lo[i] : 1;  // empty key range for rows past the window
       const int row_hi = real_row ? (int)i : 0;
       float m = -INFINITY, l = 0.f;
       bool ok = true;
@@ -298,7 +299,7 @@ __global__ void __launch_bounds__(192, 1)
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
       const float lse_val = l > 0.f ? (m + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
       if (slot < 0) {
-        __nv_bfloat16* orow = p.o + ((size_t)i * p.hq + h) * D;
+        __nv_bfloat16* orow = p.o + ((size_t)(i - p.q0) * p.hq + h) * D;
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
           float ov[32];
@@ -315,7 +316,7 @@ __global__ void __launch_bounds__(192, 1)
             }
           }
         }
-        if (real_row) p.lse[(size_t)h * p.n + i] = lse_val;
+        if (real_row) p.lse[(size_t)h * p.lse_ld + (i - p.q0)] = lse_val;
       } else {
         float* orow = p.o_part + (((size_t)slot * p.hq + h) * 128 + r) * D;
 #pragma unroll 1
@@ -448,8 +449,8 @@ __global__ void __launch_bounds__(320, 1)
         if (!mbar_wait(q_empty, (unit_iter & 1) ^ 1, guard, kErrTimeoutLoad)) break;
         mbar_arrive_expect_tx(q_full, 2 * C::QBYTES);
         for (int b = 0; b < D / 64; ++b) {
-          tma_load_3d(smem + C::OFF_Q0 + b * C::BOX, &tmQ, q_full, 64 * b, h0, qt * 128);
-          tma_load_3d(smem + C::OFF_Q1 + b * C::BOX, &tmQ, q_full, 64 * b, h0 + 1, qt * 128);
+          tma_load_3d(smem + C::OFF_Q0 + b * C::BOX, &tmQ, q_full, 64 * b, h0, qt * 128 - (int)p.q0);
+          tma_load_3d(smem + C::OFF_Q1 + b * C::BOX, &tmQ, q_full, 64 * b, h0 + 1, qt * 128 - (int)p.q0);
         }
         int kt_next = p.items[5 * ib + 1];
         for (int t = 0; t < ic; ++t) {
@@ -460,11 +461,11 @@ __global__ void __launch_bounds__(320, 1)
           if (!mbar_wait(k_empty + s, ph ^ 1, guard, kErrTimeoutLoad)) { ok = false; break; }
           mbar_arrive_expect_tx(k_full + s, C::KVBYTES);
           for (int b = 0; b < D / 64; ++b)
-            tma_load_3d(smem + C::OFF_K + s * C::KVBYTES + b * C::BOX, &tmK, k_full + s, 64 * b, g, kt * 128);
+            tma_load_3d(smem + C::OFF_K + s * C::KVBYTES + b * C::BOX, &tmK, k_full + s, 64 * b, g, kt * 128 - (int)p.kv0);
           if (!mbar_wait(v_empty + s, ph ^ 1, guard, kErrTimeoutLoad)) { ok = false; break; }
           mbar_arrive_expect_tx(v_full + s, C::KVBYTES);
           for (int b = 0; b < D / 64; ++b)
-            tma_load_3d(smem + C::OFF_V + s * C::KVBYTES + b * C::BOX, &tmV, v_full + s, 64 * b, g, kt * 128);
+            tma_load_3d(smem + C::OFF_V + s * C::KVBYTES + b * C::BOX, &tmV, v_full + s, 64 * b, g, kt * 128 - (int)p.kv0);
           ++kv_iter;
         }
         ++unit_iter;
@@ -565,7 +566,7 @@ __global__ void __launch_bounds__(320, 1)
       const int u = p.order[w / pairs], h = 2 * (w % pairs) + tile;
       const int qt = p.units[4 * u], ib = p.units[4 * u + 1], ic = p.units[4 * u + 2], slot = p.units[4 * u + 3];
       const int64_t i = (int64_t)qt * 128 + r;
-      const bool real_row = i < p.n;
+      const bool real_row = i < p.q_end;
       const int row_lo = real_row ? p.tok_lo[i] : 1;
       const int row_hi = real_row ? (int)i : 0;
       float m = -INFINITY, l = 0.f;
@@ -649,7 +650,7 @@ __global__ void __launch_bounds__(320, 1)
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
       const float lse_val = l > 0.f ? (m + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
       if (slot < 0) {
-        __nv_bfloat16* orow = p.o + ((size_t)i * p.hq + h) * D;
+        __nv_bfloat16* orow = p.o + ((size_t)(i - p.q0) * p.hq + h) * D;
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
           float ov[32];
@@ -666,7 +667,7 @@ __global__ void __launch_bounds__(320, 1)
             }
           }
         }
-        if (real_row) p.lse[(size_t)h * p.n + i] = lse_val;
+        if (real_row) p.lse[(size_t)h * p.lse_ld + (i - p.q0)] = lse_val;
       } else {
         float* orow = p.o_part + (((size_t)slot * p.hq + h) * 128 + r) * D;
 #pragma unroll 1

@@ -15,10 +15,13 @@ struct FwdParams {
   const int32_t* tok_lo;  // [N] first token of each token's document
   int32_t n_units;
   int32_t hq, group;      // query heads, hq / hkv
-  int64_t n;              // packed tokens
+  // Buffer windows (global token indices): Q, O and LSE hold rows [q0, q_end), K and V rows
+  // [kv0, q_end); tiles, items and the per-token arrays stay in global coordinates.
+  int64_t q0, kv0, q_end;
+  int64_t lse_ld;         // row stride of LSE (q_end - q0)
   float scale_log2;       // softmax_scale * log2(e)
-  __nv_bfloat16* o;       // [N][hq][D]
-  float* lse;             // [hq][N]
+  __nv_bfloat16* o;       // [q rows][hq][D]
+  float* lse;             // [hq][lse_ld]
   float* o_part;          // [slots][hq][128][D]
   float* lse_part;        // [slots][hq][128]
   int* err;               // device error word
@@ -30,11 +33,13 @@ struct BwdParams {
   const int32_t* tok_hi;      // [N] last token of each token's document
   int32_t n_kv_units;
   int32_t hq, hkv, group;
-  int64_t n, n_pad;           // tokens, tokens rounded up to 128
+  // Buffer windows as in FwdParams: query-side rows [q0, q_end), key/value-side rows [kv0, q_end).
+  int64_t q0, kv0, q_end;
+  int64_t n_pad, n_pad_kv;    // query / key-value window rows rounded up to 128
   float scale_log2;           // softmax_scale * log2(e)
   float scale;                // softmax_scale
-  const float* lse2;          // [hq][n_pad] LSE * log2(e) (+inf past N)
-  const float* dvec;          // [hq][n_pad] D_i = <dO_i, O_i> (0 past N)
+  const float* lse2;          // [hq][n_pad] LSE * log2(e) (+inf past the window)
+  const float* dvec;          // [hq][n_pad] D_i = <dO_i, O_i> (0 past the window)
   float* dq_acc;              // [n_pad][hq][D] fp32 dQ accumulator (reduced into through the tdq map)
   int* err;
 };
@@ -48,14 +53,23 @@ cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
                        const CUtensorMap& tdq, const CUtensorMap& tdkv, const BwdParams& p, int grid,
                        cudaStream_t stream);
 
+// Merge into O rows [q0, q_end) (O and LSE hold the window's rows; LSE row stride q_end - q0).
 template <int D>
-cudaError_t launch_merge(const int32_t* merges, int64_t n_merges, int32_t hq, int64_t n, const float* o_part,
-                         const float* lse_part, __nv_bfloat16* o, float* lse, cudaStream_t stream);
+cudaError_t launch_merge(const int32_t* merges, int64_t n_merges, int32_t hq, int64_t q0, int64_t q_end,
+                         const float* o_part, const float* lse_part, __nv_bfloat16* o, float* lse,
+                         cudaStream_t stream);
 
+// n rows of O, dO and LSE (padded to n_pad); n_pad_kv rows of each dK/dV accumulator.
 template <int D>
 cudaError_t launch_bwd_pre(const __nv_bfloat16* o, const __nv_bfloat16* dout, const float* lse, int64_t n,
-                           int64_t n_pad, int32_t hq, int32_t hkv, float* dvec, float* lse2, float* dq_acc,
-                           float* dkv_acc, cudaStream_t stream);
+                           int64_t n_pad, int64_t n_pad_kv, int32_t hq, int32_t hkv, float* dvec, float* lse2,
+                           float* dq_acc, float* dkv_acc, cudaStream_t stream);
+
+// dkv_acc rows [row0, row0 + rows) += the fp32 partials dk_part, dv_part ([rows][hkv][D] each), then
+// those rows of dk and dv (same row numbering as the accumulator) are rewritten as bf16.
+cudaError_t launch_kv_add(float* dkv_acc, int64_t dv_offset, const float* dk_part, const float* dv_part,
+                          int64_t row0, int64_t rows, int64_t row_elems, __nv_bfloat16* dk, __nv_bfloat16* dv,
+                          cudaStream_t stream);
 
 // fp32 accumulators -> bf16: dq (count_q values), dk and dv (count_kv values each; the dV
 // accumulator starts dv_offset values after the dK one).

@@ -14,6 +14,13 @@
 // of one q-tile are contiguous and together cover [s, last row].  Tags need
 // O(1) work per item because the first key of a row is non-decreasing in the
 // row.
+//
+// Chunks are contiguous token ranges: P equal ones, or explicit tile-aligned
+// bounds (for example the balanced cut below).  A rank plan keeps the items of
+// one q chunk -- the work of one device under sequence parallelism -- and the
+// window of tokens that device holds: its own chunk for the queries, and for
+// keys and values the span from the start of the document that reaches into
+// the chunk (the only earlier tokens any of its queries may see).
 #include <algorithm>
 #include <numeric>
 
@@ -66,87 +73,26 @@ void sap_plan_build_fwd_schedule(sap_plan_s* p, bool fused) {
   });
 }
 
-int sap_plan_build(const int32_t* cu, int32_t num_docs, int64_t n, int32_t num_chunks, int32_t block_m,
-                   int32_t block_n, sap_plan_s* p) {
-  if (!cu || !p || num_docs < 0 || n < 0 || block_m <= 0 || block_n <= 0) return SAP_ERR_INVALID_ARG;
+namespace {
+
+int check_cu(const int32_t* cu, int32_t num_docs, int64_t n) {
+  if (!cu || num_docs < 0 || n < 0) return SAP_ERR_INVALID_ARG;
   if (n > INT32_MAX - 256) return SAP_ERR_INVALID_ARG;
   if (cu[0] != 0) return SAP_ERR_BAD_SEQLENS;
   for (int32_t k = 0; k < num_docs; ++k)
     if (cu[k + 1] < cu[k]) return SAP_ERR_BAD_SEQLENS;
   if ((int64_t)cu[num_docs] != n) return SAP_ERR_BAD_SEQLENS;
-  if (num_chunks < 1) return SAP_ERR_BAD_CHUNKS;
-  int64_t chunk = n > 0 ? n : 1;
-  if (num_chunks > 1) {
-    if (n % num_chunks) return SAP_ERR_BAD_CHUNKS;
-    chunk = n / num_chunks;
-    if (chunk % block_m || chunk % block_n) return SAP_ERR_BAD_CHUNKS;
-  }
-  p->n = n;
-  p->num_docs = num_docs;
-  p->num_chunks = num_chunks;
-  p->block_m = block_m;
-  p->block_n = block_n;
-  p->chunk = chunk;
-  p->cu.assign(cu, cu + num_docs + 1);
+  return SAP_OK;
+}
 
-  // per-token document bounds
-  p->tok_lo.assign((size_t)n, 0);
-  p->tok_hi.assign((size_t)n, 0);
-  p->unmasked_pairs = 0;
-  std::vector<int32_t> doc_of((size_t)n);
-  for (int32_t k = 0; k < num_docs; ++k) {
-    int64_t L = (int64_t)cu[k + 1] - cu[k];
-    p->unmasked_pairs += L * (L + 1) / 2;
-    for (int64_t i = cu[k]; i < cu[k + 1]; ++i) {
-      p->tok_lo[i] = cu[k];
-      p->tok_hi[i] = cu[k + 1] - 1;
-      doc_of[i] = k;
-    }
-  }
-
-  // items, canonical order
-  p->items.clear();
-  const int64_t ntq = (n + block_m - 1) / block_m;
-  for (int64_t qt = 0; qt < ntq; ++qt) {
-    const int64_t i0 = qt * block_m;
-    const int64_t ilast = std::min<int64_t>(i0 + block_m, n) - 1;  // last real row
-    const bool tile_complete = (i0 + block_m) <= n;
-    const int64_t kt_first = p->tok_lo[i0] / block_n, kt_last = ilast / block_n;
-    for (int64_t kt = kt_first; kt <= kt_last; ++kt) {
-      const int64_t j0 = kt * block_n, j1 = j0 + block_n - 1;
-      int32_t tag;
-      // every nominal row exists, the latest-starting row starts at or before j0,
-      // and the earliest row ends at or after j1
-      if (tile_complete && p->tok_lo[ilast] <= j0 && j1 <= i0)
-        tag = SAP_TAG_FULL;
-      else if (block_m == block_n && kt == qt && doc_of[i0] == doc_of[ilast])
-        tag = SAP_TAG_CAUSAL;
-      else
-        tag = SAP_TAG_MASKED;
-      p->items.push_back(
-          sap_item_t{(int32_t)qt, (int32_t)kt, (int32_t)(i0 / chunk), (int32_t)(j0 / chunk), tag});
-    }
-  }
-
-  // chunk pairs
-  {
-    std::vector<char> seen((size_t)num_chunks * num_chunks, 0);
-    p->n_chunk_pairs = 0;
-    for (const auto& it : p->items) {
-      char& s = seen[(size_t)it.q_chunk * num_chunks + it.kv_chunk];
-      if (!s) s = 1, ++p->n_chunk_pairs;
-    }
-  }
-
-  sap_plan_build_fwd_schedule(p, false);
-
-  // backward: items grouped by kv tile, q-tile descending within a kv tile, and each kv tile's
-  // list cut into bands of kBwdBandTiles q tiles.  A unit is one (kv tile, band) piece; units are
-  // ordered band-major from the top band down, heavy-first within a band.  The persistent CTAs take
-  // units in this order, so at any time they all work on Q, dO and dQ rows of about one band (a few
-  // tens of MB at 32 heads) and those rows stay in L2; the price is one fp32 dK/dV reduction per unit
-  // instead of one bf16 store per kv tile.
-  const int64_t ntk = (n + block_n - 1) / block_n;
+// Backward: items grouped by kv tile, q-tile descending within a kv tile, and each kv tile's
+// list cut into bands of kBwdBandTiles q tiles.  A unit is one (kv tile, band) piece; units are
+// ordered band-major from the top band down, heavy-first within a band.  The persistent CTAs take
+// units in this order, so at any time they all work on Q, dO and dQ rows of about one band (a few
+// tens of MB at 32 heads) and those rows stay in L2; the price is one fp32 dK/dV reduction per unit
+// instead of one bf16 store per kv tile.
+void build_bwd_schedule(sap_plan_s* p) {
+  const int64_t ntk = (p->n + p->block_n - 1) / p->block_n;
   std::vector<int64_t> cnt((size_t)ntk + 1, 0);
   for (const auto& it : p->items) cnt[(size_t)it.kv_tile + 1]++;
   for (int64_t t = 0; t < ntk; ++t) cnt[t + 1] += cnt[t];
@@ -179,5 +125,187 @@ int sap_plan_build(const int32_t* cu, int32_t num_docs, int64_t n, int32_t num_c
   p->kv_units.clear();
   p->kv_units.reserve(units.size() * 3);
   for (const Unit& u : units) p->kv_units.insert(p->kv_units.end(), {u.kv_tile, u.first, u.count});
+}
+
+void count_chunk_pairs(sap_plan_s* p) {
+  std::vector<char> seen((size_t)p->num_chunks * p->num_chunks, 0);
+  p->n_chunk_pairs = 0;
+  for (const auto& it : p->items) {
+    char& s = seen[(size_t)it.q_chunk * p->num_chunks + it.kv_chunk];
+    if (!s) s = 1, ++p->n_chunk_pairs;
+  }
+}
+
+// Number of kv tiles a q tile touches: floor(first key / bn) .. floor(last row / bn).
+int64_t tile_cost(const std::vector<int32_t>& tok_lo, int64_t n, int64_t qt, int32_t bm, int32_t bn) {
+  const int64_t i0 = qt * bm, ilast = std::min<int64_t>(i0 + bm, n) - 1;
+  return ilast / bn - tok_lo[i0] / bn + 1;
+}
+
+}  // namespace
+
+int sap_plan_build(const int32_t* cu, int32_t num_docs, int64_t n, int32_t num_chunks, const int64_t* bounds,
+                   int32_t block_m, int32_t block_n, sap_plan_s* p) {
+  if (!p || block_m <= 0 || block_n <= 0) return SAP_ERR_INVALID_ARG;
+  int rc = check_cu(cu, num_docs, n);
+  if (rc) return rc;
+  if (num_chunks < 1) return SAP_ERR_BAD_CHUNKS;
+  std::vector<int64_t> b((size_t)num_chunks + 1);
+  if (bounds) {
+    // explicit contiguous chunks: non-empty, interior bounds on tile boundaries of both tile sizes
+    if (bounds[0] != 0 || bounds[num_chunks] != n) return SAP_ERR_BAD_CHUNKS;
+    for (int32_t c = 0; c < num_chunks; ++c) {
+      if (bounds[c + 1] <= bounds[c] && !(num_chunks == 1 && n == 0)) return SAP_ERR_BAD_CHUNKS;
+      if (c > 0 && (bounds[c] % block_m || bounds[c] % block_n)) return SAP_ERR_BAD_CHUNKS;
+    }
+    b.assign(bounds, bounds + num_chunks + 1);
+  } else if (num_chunks == 1) {
+    b = {0, n};
+  } else {
+    if (n % num_chunks) return SAP_ERR_BAD_CHUNKS;
+    const int64_t chunk = n / num_chunks;
+    if (chunk % block_m || chunk % block_n) return SAP_ERR_BAD_CHUNKS;
+    for (int32_t c = 0; c <= num_chunks; ++c) b[c] = c * chunk;
+  }
+  p->n = n;
+  p->num_docs = num_docs;
+  p->num_chunks = num_chunks;
+  p->block_m = block_m;
+  p->block_n = block_n;
+  p->bounds = b;
+  p->cu.assign(cu, cu + num_docs + 1);
+  p->rank_chunk = -1;
+  p->q_begin = 0, p->q_end = n, p->kv_begin = 0, p->span_begin = 0;
+
+  // per-token document bounds
+  p->tok_lo.assign((size_t)n, 0);
+  p->tok_hi.assign((size_t)n, 0);
+  p->unmasked_pairs = 0;
+  std::vector<int32_t> doc_of((size_t)n);
+  for (int32_t k = 0; k < num_docs; ++k) {
+    int64_t L = (int64_t)cu[k + 1] - cu[k];
+    p->unmasked_pairs += L * (L + 1) / 2;
+    for (int64_t i = cu[k]; i < cu[k + 1]; ++i) {
+      p->tok_lo[i] = cu[k];
+      p->tok_hi[i] = cu[k + 1] - 1;
+      doc_of[i] = k;
+    }
+  }
+  auto chunk_of = [&](int64_t tok) {
+    return (int32_t)(std::upper_bound(p->bounds.begin(), p->bounds.end(), tok) - p->bounds.begin() - 1);
+  };
+
+  // items, canonical order
+  p->items.clear();
+  const int64_t ntq = (n + block_m - 1) / block_m;
+  for (int64_t qt = 0; qt < ntq; ++qt) {
+    const int64_t i0 = qt * block_m;
+    const int64_t ilast = std::min<int64_t>(i0 + block_m, n) - 1;  // last real row
+    const bool tile_complete = (i0 + block_m) <= n;
+    const int64_t kt_first = p->tok_lo[i0] / block_n, kt_last = ilast / block_n;
+    const int32_t qc = chunk_of(i0);
+    for (int64_t kt = kt_first; kt <= kt_last; ++kt) {
+      const int64_t j0 = kt * block_n, j1 = j0 + block_n - 1;
+      int32_t tag;
+      // every nominal row exists, the latest-starting row starts at or before j0,
+      // and the earliest row ends at or after j1
+      if (tile_complete && p->tok_lo[ilast] <= j0 && j1 <= i0)
+        tag = SAP_TAG_FULL;
+      else if (block_m == block_n && kt == qt && doc_of[i0] == doc_of[ilast])
+        tag = SAP_TAG_CAUSAL;
+      else
+        tag = SAP_TAG_MASKED;
+      p->items.push_back(sap_item_t{(int32_t)qt, (int32_t)kt, qc, chunk_of(j0), tag});
+    }
+  }
+  count_chunk_pairs(p);
+  sap_plan_build_fwd_schedule(p, false);
+  build_bwd_schedule(p);
+  return SAP_OK;
+}
+
+int sap_plan_build_rank(const sap_plan_s* f, int32_t chunk, sap_plan_s* r) {
+  if (!f || !r || f->rank_chunk >= 0 || chunk < 0 || chunk >= f->num_chunks) return SAP_ERR_INVALID_ARG;
+  r->n = f->n;
+  r->num_docs = f->num_docs;
+  r->num_chunks = f->num_chunks;
+  r->block_m = f->block_m;
+  r->block_n = f->block_n;
+  r->bounds = f->bounds;
+  r->cu = f->cu;
+  r->tok_lo = f->tok_lo;
+  r->tok_hi = f->tok_hi;
+  r->rank_chunk = chunk;
+  r->q_begin = f->bounds[chunk];
+  r->q_end = f->bounds[chunk + 1];
+  r->span_begin = r->q_begin < f->n ? f->tok_lo[r->q_begin] : r->q_begin;
+  r->kv_begin = r->span_begin / f->block_n * f->block_n;
+  r->items.clear();
+  for (const auto& it : f->items)
+    if (it.q_chunk == chunk) r->items.push_back(it);
+  r->unmasked_pairs = 0;
+  for (int64_t i = r->q_begin; i < r->q_end; ++i) r->unmasked_pairs += i - f->tok_lo[i] + 1;
+  count_chunk_pairs(r);
+  sap_plan_build_fwd_schedule(r, f->fused_merge);
+  build_bwd_schedule(r);
+  return SAP_OK;
+}
+
+// Balanced cut.  The cost of a q tile is the number of kv tiles it touches (one 128 x 128 tile of
+// both passes' GEMMs each, masked or not).  M* = the smallest possible maximum over chunks of the
+// summed cost, found by bisection with a greedy feasibility test (pack tiles left to right into
+// chunks of cost <= M; feasible iff at most num_chunks chunks are needed).  Among the cuts that
+// reach M*, the bounds are the lexicographically largest: each chunk takes as many tiles as fit
+// while leaving at least one tile for every later chunk.
+int sap_balanced_bounds(const int32_t* cu, int32_t num_docs, int64_t n, int32_t num_chunks, int32_t block,
+                        int64_t* bounds) {
+  if (!bounds || block <= 0) return SAP_ERR_INVALID_ARG;
+  int rc = check_cu(cu, num_docs, n);
+  if (rc) return rc;
+  if (num_chunks < 1) return SAP_ERR_BAD_CHUNKS;
+  const int64_t T = (n + block - 1) / block;
+  if (n == 0) {
+    if (num_chunks != 1) return SAP_ERR_BAD_CHUNKS;
+    bounds[0] = bounds[1] = 0;
+    return SAP_OK;
+  }
+  if (num_chunks > T) return SAP_ERR_BAD_CHUNKS;
+  std::vector<int32_t> tok_lo((size_t)n, 0);
+  for (int32_t k = 0; k < num_docs; ++k)
+    for (int64_t i = cu[k]; i < cu[k + 1]; ++i) tok_lo[i] = cu[k];
+  std::vector<int64_t> cost((size_t)T);
+  int64_t total = 0, top = 0;
+  for (int64_t t = 0; t < T; ++t) {
+    cost[t] = tile_cost(tok_lo, n, t, block, block);
+    total += cost[t];
+    top = std::max(top, cost[t]);
+  }
+  auto chunks_needed = [&](int64_t cap) {
+    int64_t used = 1, acc = 0;
+    for (int64_t t = 0; t < T; ++t) {
+      if (acc + cost[t] > cap) ++used, acc = 0;
+      acc += cost[t];
+    }
+    return used;
+  };
+  int64_t lo = top, hi = total;  // chunks_needed(hi) == 1
+  while (lo < hi) {
+    const int64_t mid = lo + (hi - lo) / 2;
+    if (chunks_needed(mid) <= num_chunks)
+      hi = mid;
+    else
+      lo = mid + 1;
+  }
+  const int64_t cap = lo;
+  int64_t pos = 0;
+  bounds[0] = 0;
+  for (int32_t k = 0; k + 1 < num_chunks; ++k) {
+    const int64_t later = num_chunks - k - 1;  // chunks still to fill after this one
+    int64_t e = pos, acc = 0;
+    while (e < T - later && acc + cost[e] <= cap) acc += cost[e++];
+    bounds[k + 1] = e * block;
+    pos = e;
+  }
+  bounds[num_chunks] = n;
   return SAP_OK;
 }
