@@ -250,6 +250,14 @@ def main():
                     help="one forward pass over all kv chunks of a q tile (no partials, no merge kernel)")
     ap.add_argument("--tokens", type=int, default=None,
                     help="run the workload's recipe at a smaller token count (profiling captures only)")
+    ap.add_argument("--parallelism", default="dp", choices=["dp", "sap", "hsap"],
+                    help="dp: independent replicas (default); sap / hsap: one batch split across the ranks "
+                         "(sequence-aware exchange, with a Ulysses head split of degree --ulysses for hsap)")
+    ap.add_argument("--ulysses", type=int, default=1, help="Ulysses (head-split) degree for --parallelism hsap")
+    ap.add_argument("--equal-chunks", action="store_true", help="sap / hsap / emulation: equal chunks, not balanced")
+    ap.add_argument("--emulate-ranks", type=int, default=0,
+                    help="one GPU: run the rank plans of a W-way sequence split one after another and report "
+                         "per-rank kernel times (the exchange is emulated by device copies)")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -262,6 +270,10 @@ def main():
 
     if args.impl == "reference":
         return run_reference(args, w, rank, world)
+    if args.emulate_ranks:
+        return run_emulated_ranks(args, w)
+    if args.parallelism != "dp":
+        return run_split(args, w, rank, world, local_rank)
 
     import torch
     import torch.distributed as dist
@@ -498,6 +510,170 @@ def main():
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def _split_ranks(w, b, nranks, balanced):
+    from packed_sequence_causal_b200 import sap_dist
+    return [sap_dist.SapAttention(b.cu_seqlens, w.n, w.hq, w.hkv, w.d, c, nranks, balanced=balanced)
+            for c in range(nranks)]
+
+
+def run_emulated_ranks(args, w):
+    """The rank plans of a W-way sequence-parallel split, run one after another on this GPU.
+
+    Per step and rank: the forward (sap_attn_fwd + sap_merge on the rank's windowed buffers) and the
+    backward (sap_attn_bwd, then sap_attn_bwd_kv_add of the partials later ranks computed for its
+    tokens), each timed with CUDA events on the launching stream.  The key/value windows are
+    assembled once from the batch (what the exchange delivers); the partial dK/dV rows are handed
+    over by device copies, outside the per-rank times.  Reported: the slowest rank's time per step
+    (the step time of W GPUs if the transfers were free) and the whole job's TFLOP/s at that time,
+    each rank's time and the bytes it would receive, for the balanced or the equal cut."""
+    import torch
+
+    import packed_sequence_causal_b200 as sap
+
+    W = args.emulate_ranks
+    balanced = not args.equal_chunks
+    torch.cuda.set_device(0)
+    b = workloads.make_batch(w, args.seed, device="cuda", with_do=True)
+    ranks = _split_ranks(w, b, W, balanced)
+    q, k, v, do = b.q, b.k, b.v, b.do
+    wins = []
+    for r in ranks:
+        wd = r.window
+        kv0, q0, q1, s0 = wd["kv_begin"], wd["q_begin"], wd["q_end"], wd["span_begin"]
+        k_win = torch.zeros((q1 - kv0, w.hkv, w.d), dtype=k.dtype, device="cuda")
+        v_win = torch.zeros_like(k_win)
+        k_win[s0 - kv0:] = k[s0:q1]
+        v_win[s0 - kv0:] = v[s0:q1]
+        wins.append((q[q0:q1].contiguous(), k_win, v_win, do[q0:q1].contiguous()))
+    stream = torch.cuda.current_stream()
+
+    def step(times=None):
+        received = {c: [] for c in range(W)}
+        for c, (r, (qr, kw, vw, dor)) in enumerate(zip(ranks, wins)):
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(2)] if times is not None else None
+            if e:
+                e[0].record(stream)
+            r.attend(qr, kw, vw)
+            r.local_backward(dor)
+            if e:
+                e[1].record(stream)
+                times[c].append(e)
+        for r in ranks:
+            kv0 = r.window["kv_begin"]
+            for src, lo, hi in r.recv:
+                received[src].append((lo, hi, r._dk_acc[lo - kv0:hi - kv0].clone(),
+                                      r._dv_acc[lo - kv0:hi - kv0].clone()))
+        for c, r in enumerate(ranks):
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(2)] if times is not None else None
+            if e:
+                e[0].record(stream)
+            r.add_partials(received[c])
+            if e:
+                e[1].record(stream)
+                times[c].append(e)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if sap.sap_device_status() != 0:
+        raise RuntimeError("device error word set after warm-up")
+    times = [[] for _ in range(W)]
+    for _ in range(args.steps):
+        step(times)
+    torch.cuda.synchronize()
+    if sap.sap_device_status() != 0:
+        raise RuntimeError("device error word set after the timed steps")
+    per_rank = [sum(e[0].elapsed_time(e[1]) for e in t) / args.steps for t in times]
+    pairs = sap.sap_plan_stats(ranks[0].full)["unmasked_pairs"]
+    f_fwd, f_bwd = _flops(w, pairs)
+    row = 2 * w.hkv * w.d * 2
+    recv_bytes = [sum(int(hi - lo) for _, lo, hi in r.recv) * row for r in ranks]
+    items = sap.sap_plan_chunk_stats(ranks[0].full)["items"]
+    slow = max(per_rank)
+    line = {
+        "metric": METRIC + " (emulated sequence split: slowest rank)", "value": round((f_fwd + f_bwd) / (slow / 1e3) / 1e12, 2),
+        "unit": "TFLOP/s", "n_gpus_emulated": W, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step_slowest_rank": round(slow, 3), "ms_per_rank": [round(t, 3) for t in per_rank],
+        "max_over_mean": round(slow / (sum(per_rank) / W), 4), "cut": "balanced" if balanced else "equal",
+        "chunk_bounds": ranks[0].bounds.tolist(), "items_per_rank": items.tolist(),
+        "kv_bytes_received_per_rank": recv_bytes, "ring_kv_bytes": _ring(ranks[0].bounds, row),
+        "dtype": "bf16", "data": "synthetic (seeded packed documents, bf16 N(0,1) Q/K/V/dO)",
+        "config": {"workload": w.name, "tokens": w.n, "hq": w.hq, "hkv": w.hkv, "head_dim": w.d},
+        "note": "all ranks on one GPU in turn; transfers not timed",
+    }
+    print(json.dumps(line), flush=True)
+
+
+def _ring(bounds, row):
+    from packed_sequence_causal_b200 import sap_dist
+    return sap_dist.ring_bytes(bounds, row)
+
+
+def run_split(args, w, rank, world, local_rank):
+    """One packed batch split across the ranks: SAP (chunk per rank) or HSAP (Ulysses groups of
+    --ulysses ranks, SAP across them).  Every rank builds the same seeded batch and takes its token
+    block; one step = HsapAttention.forward + backward with their NCCL exchanges.  Whole-job
+    TFLOP/s = the batch's unmasked FLOPs / the slowest rank's time (strong scaling: the work is
+    fixed as the ranks grow).  Unmeasured on hardware in this repository: every GPU call it had
+    was a single GPU."""
+    import torch
+    import torch.distributed as dist
+
+    import packed_sequence_causal_b200 as sap
+    from packed_sequence_causal_b200 import sap_dist
+
+    U = args.ulysses if args.parallelism == "hsap" else 1
+    if world % U:
+        raise SystemExit("--ulysses must divide the number of ranks")
+    S = world // U
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    b = workloads.make_batch(w, args.seed, device=str(dev), with_do=True)
+    ug = sap_dist.make_hsap_groups(S, U) if world > 1 else None
+    h = sap_dist.HsapAttention(b.cu_seqlens, w.n, w.hq, w.hkv, w.d, S, U, rank=rank, ulysses_group=ug,
+                               balanced=not args.equal_chunks)
+    lo, hi = h.block
+    q, k, v, do = (t[lo:hi].contiguous() for t in (b.q, b.k, b.v, b.do))
+    stream = torch.cuda.current_stream()
+
+    def step():
+        h.forward(q, k, v)
+        h.backward(do)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(args.steps):
+        step()
+    end.record(stream)
+    torch.cuda.synchronize()
+    elapsed = max_over_ranks(start.elapsed_time(end), dist if world > 1 else None, dev)
+    if sap.sap_device_status() != 0:
+        raise RuntimeError("device error word set after the timed steps")
+    pairs = sap.sap_plan_stats(h.sap.full)["unmasked_pairs"]
+    f_fwd, f_bwd = _flops(w, pairs)
+    value = (f_fwd + f_bwd) * args.steps / (elapsed / 1e3) / 1e12
+    if rank == 0:
+        print(json.dumps({
+            "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(elapsed / args.steps, 3), "higher_is_better": True,
+            "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded packed documents, bf16 N(0,1) Q/K/V/dO)",
+            "config": {"workload": w.name, "tokens": w.n, "hq": w.hq, "hkv": w.hkv, "head_dim": w.d,
+                       "parallelism": f"sap{S}" + (f"xulysses{U}" if U > 1 else ""),
+                       "cut": "equal" if args.equal_chunks else "balanced"},
+            "kv_bytes_received_rank0": h.sap.bytes["kv_received"], "gpu_launches": None}), flush=True)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
