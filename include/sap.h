@@ -285,6 +285,23 @@ const char* sap_error_string(int status);
 /* The last cudaError_t seen by a call that returned SAP_ERR_CUDA. */
 int sap_last_cuda_error(void);
 
+/* Pipeline wait limit of every later kernel launch, in nanoseconds (0 restores the default of
+ * 4 s; accepted range 1 ms .. 600 s, else SAP_ERR_INVALID_ARG).  A wait that runs past it sets
+ * the device error word (read by sap_device_status) and winds its CTA down: copies and MMAs in
+ * flight are waited for, again within the limit, before shared memory and tensor memory are
+ * released; that CTA's remaining outputs are left unwritten.  A limit shorter than the longest
+ * legitimate wait (a forward unit's whole pass over its kv tiles: milliseconds for long
+ * documents) reports false timeouts.  Process-wide; no counterpart in the pages. */
+int sap_set_wait_limit_ns(uint64_t limit_ns);
+
+/* Failure-detection test hook (no counterpart in the pages): arms the next sap_attn_fwd call
+ * so that its launch uses wait_limit_ns (100 us .. 10 s, else SAP_ERR_INVALID_ARG) and its first
+ * CTA leaves its first V tile out -- no copy is issued, so nothing is in flight -- and the MMA
+ * wait on that tile runs out.  The call returns SAP_OK; sap_device_status() then reports
+ * SAP_ERR_DEVICE with the MMA timeout bit, and the outputs of that launch are incomplete.  The
+ * hook disarms itself at that launch; later calls are normal. */
+int sap_test_arm_wait_timeout(uint64_t wait_limit_ns);
+
 #ifdef __cplusplus
 }
 #endif

@@ -91,6 +91,10 @@ def load_library():
     L.sap_error_string.argtypes = [ctypes.c_int]
     L.sap_last_cuda_error.restype = ctypes.c_int
     L.sap_last_cuda_error.argtypes = []
+    L.sap_set_wait_limit_ns.restype = ctypes.c_int
+    L.sap_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+    L.sap_test_arm_wait_timeout.restype = ctypes.c_int
+    L.sap_test_arm_wait_timeout.argtypes = [ctypes.c_uint64]
     _lib = L
     return L
 
@@ -345,3 +349,8 @@ def sap_device_status() -> int:
     if st not in (SAP_OK, -6):
         raise SapError(st, "sap_device_status")
     return c.value
+
+
+def sap_set_wait_limit_ns(limit_ns: int):
+    """Pipeline wait limit of later kernel launches (0: the default 4 s)."""
+    _check(load_library().sap_set_wait_limit_ns(int(limit_ns)), "sap_set_wait_limit_ns")

@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <cstring>
 #include <mutex>
 #include <new>
@@ -15,6 +16,11 @@
 namespace {
 
 thread_local int g_last_cuda_error = 0;
+
+// Pipeline wait limit given to every kernel launch (sap_set_wait_limit_ns), and the armed
+// wait-timeout test hook (sap_test_arm_wait_timeout): its limit, 0 when disarmed.
+std::atomic<uint64_t> g_wait_limit_ns{4000000000ull};
+std::atomic<uint64_t> g_test_timeout_ns{0};
 
 // Device error word (bitwise OR of sap::kErr* codes), one per device.
 __device__ int g_device_err;
@@ -166,6 +172,8 @@ sap::FwdParams fwd_params(const sap_plan_s* p, int32_t hq, int32_t hkv, float so
   fp.q_end = p->q_end;
   fp.lse_ld = p->q_rows();
   fp.scale_log2 = softmax_scale * 1.4426950408889634f;
+  fp.wait_ns = g_wait_limit_ns.load();
+  fp.skip_v_load = 0;
   return fp;
 }
 
@@ -476,6 +484,10 @@ int sap_attn_fwd(sap_plan_t p, const void* q, const void* k, const void* v, int3
   if ((rc = make_map(&tk, k, p->kv_rows(), hkv, head_dim))) return rc;
   if ((rc = make_map(&tv, v, p->kv_rows(), hkv, head_dim))) return rc;
   sap::FwdParams fp = fwd_params(p, hq, hkv, softmax_scale);
+  if (const uint64_t t = g_test_timeout_ns.exchange(0)) {  // armed test hook: this launch only
+    fp.skip_v_load = 1;
+    fp.wait_ns = t;
+  }
   fp.o = static_cast<__nv_bfloat16*>(o);
   fp.lse = lse;
   uint8_t* wsb = static_cast<uint8_t*>(workspace);
@@ -578,6 +590,7 @@ int sap_attn_bwd(sap_plan_t p, const void* q, const void* k, const void* v, cons
   bp.dvec = dvec;
   bp.dq_acc = dq_acc;
   bp.err = di->err;
+  bp.wait_ns = g_wait_limit_ns.load();
   const int64_t work = (int64_t)bp.n_kv_units * hkv;
   if (work > 0) {
     const int grid = (int)(work < di->sms ? work : di->sms);
@@ -646,6 +659,19 @@ const char* sap_error_string(int status) {
 }
 
 int sap_last_cuda_error(void) { return g_last_cuda_error; }
+
+int sap_set_wait_limit_ns(uint64_t limit_ns) {
+  if (limit_ns == 0) limit_ns = 4000000000ull;
+  if (limit_ns < 1000000ull || limit_ns > 600000000000ull) return SAP_ERR_INVALID_ARG;
+  g_wait_limit_ns.store(limit_ns);
+  return SAP_OK;
+}
+
+int sap_test_arm_wait_timeout(uint64_t wait_limit_ns) {
+  if (wait_limit_ns < 100000ull || wait_limit_ns > 10000000000ull) return SAP_ERR_INVALID_ARG;
+  g_test_timeout_ns.store(wait_limit_ns);
+  return SAP_OK;
+}
 
 int sap_attn_fwd_static_scratch(sap_plan_t p, const void* q, const void* k, const void* v, int32_t hq, int32_t hkv,
                                 int32_t head_dim, float softmax_scale, void* o, float* lse, void* stream) {

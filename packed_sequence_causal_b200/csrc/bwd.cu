@@ -116,7 +116,7 @@ __global__ void __launch_bounds__(448, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const Guard guard{abort_flag, p.err};
+  const Guard guard{abort_flag, p.err, p.wait_ns};
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
@@ -196,9 +196,9 @@ __global__ void __launch_bounds__(448, 1)
         }
         ++unit_iter;
       }
-      if (unit_iter > 0) drain_wait(kv_full, (unit_iter - 1) & 1);
+      if (unit_iter > 0) drain_wait(kv_full, (unit_iter - 1) & 1, p.wait_ns);
       for (uint32_t t = (q_iter > (uint32_t)C::NSQ ? q_iter - C::NSQ : 0); t < q_iter; ++t)
-        drain_wait(q_full + t % C::NSQ, (t / C::NSQ) & 1);
+        drain_wait(q_full + t % C::NSQ, (t / C::NSQ) & 1, p.wait_ns);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -287,7 +287,7 @@ __global__ void __launch_bounds__(448, 1)
         ++unit_iter;
       }
       tc_commit(mma_drain);
-      drain_wait(mma_drain, 0);
+      drain_wait(mma_drain, 0, p.wait_ns);
     }
   } else if (warp < 10) {
     // ----------------------------------------------------- P^T and dS^T

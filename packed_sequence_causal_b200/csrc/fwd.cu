@@ -71,7 +71,7 @@ __global__ void __launch_bounds__(192, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const Guard guard{abort_flag, p.err};
+  const Guard guard{abort_flag, p.err, p.wait_ns};
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -125,22 +125,27 @@ __global__ void __launch_bounds__(192, 1)
           if (!mbar_wait(k_empty + s, ph ^ 1, guard, kErrTimeoutLoad)) { ok = false; break; }
           mbar_arrive_expect_tx(k_full + s, C::KVBYTES);
           for (int b = 0; b < D / 64; ++b)
-            tma_load_3d(smem + C::OFF_K + s * C::KVBYTES + b * C::BOX, &tmK, k_full + s, 64 * b, g, kt * 128 - (int)p.kv0);
+            tma_load_3d(smem + C::OFF_K + s * C::KVBYTES + b * C::BOX, &tmK, k_full + s, 64 * b, g,
+                        kt * 128 - (int)p.kv0);
           if (!mbar_wait(v_empty + s, ph ^ 1, guard, kErrTimeoutLoad)) { ok = false; break; }
-          mbar_arrive_expect_tx(v_full + s, C::KVBYTES);
-          for (int b = 0; b < D / 64; ++b)
-            tma_load_3d(smem + C::OFF_V + s * C::KVBYTES + b * C::BOX, &tmV, v_full + s, 64 * b, g, kt * 128 - (int)p.kv0);
+          // test hook: CTA 0 leaves its first V tile out (nothing is issued), so the MMA wait on it runs out
+          if (!(p.skip_v_load && blockIdx.x == 0 && kv_iter == 0)) {
+            mbar_arrive_expect_tx(v_full + s, C::KVBYTES);
+            for (int b = 0; b < D / 64; ++b)
+              tma_load_3d(smem + C::OFF_V + s * C::KVBYTES + b * C::BOX, &tmV, v_full + s, 64 * b, g,
+                          kt * 128 - (int)p.kv0);
+          }
           ++kv_iter;
         }
         ++unit_iter;
       }
       // Let every copy this thread started land before the CTA can exit.
-      if (unit_iter > 0) drain_wait(q_full, (unit_iter - 1) & 1);
+      if (unit_iter > 0) drain_wait(q_full, (unit_iter - 1) & 1, p.wait_ns);
       for (uint32_t t = (kv_iter > (uint32_t)C::NS ? kv_iter - C::NS : 0); t < kv_iter; ++t) {
         const int s = t % C::NS;
         const uint32_t ph = (t / C::NS) & 1;
-        drain_wait(k_full + s, ph);
-        drain_wait(v_full + s, ph);
+        drain_wait(k_full + s, ph, p.wait_ns);
+        drain_wait(v_full + s, ph, p.wait_ns);
       }
     }
   } else if (warp == 1) {
@@ -201,7 +206,7 @@ __global__ void __launch_bounds__(192, 1)
       }
       // Wait for every MMA this thread issued before TMEM is released.
       tc_commit(mma_drain);
-      drain_wait(mma_drain, 0);
+      drain_wait(mma_drain, 0, p.wait_ns);
     }
   } else {
     // ------------------------------------------------------------- softmax
@@ -402,7 +407,7 @@ __global__ void __launch_bounds__(320, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const Guard guard{abort_flag, p.err};
+  const Guard guard{abort_flag, p.err, p.wait_ns};
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -461,19 +466,24 @@ __global__ void __launch_bounds__(320, 1)
           if (!mbar_wait(k_empty + s, ph ^ 1, guard, kErrTimeoutLoad)) { ok = false; break; }
           mbar_arrive_expect_tx(k_full + s, C::KVBYTES);
           for (int b = 0; b < D / 64; ++b)
-            tma_load_3d(smem + C::OFF_K + s * C::KVBYTES + b * C::BOX, &tmK, k_full + s, 64 * b, g, kt * 128 - (int)p.kv0);
+            tma_load_3d(smem + C::OFF_K + s * C::KVBYTES + b * C::BOX, &tmK, k_full + s, 64 * b, g,
+                        kt * 128 - (int)p.kv0);
           if (!mbar_wait(v_empty + s, ph ^ 1, guard, kErrTimeoutLoad)) { ok = false; break; }
-          mbar_arrive_expect_tx(v_full + s, C::KVBYTES);
-          for (int b = 0; b < D / 64; ++b)
-            tma_load_3d(smem + C::OFF_V + s * C::KVBYTES + b * C::BOX, &tmV, v_full + s, 64 * b, g, kt * 128 - (int)p.kv0);
+          // test hook: CTA 0 leaves its first V tile out (nothing is issued), so the MMA wait on it runs out
+          if (!(p.skip_v_load && blockIdx.x == 0 && kv_iter == 0)) {
+            mbar_arrive_expect_tx(v_full + s, C::KVBYTES);
+            for (int b = 0; b < D / 64; ++b)
+              tma_load_3d(smem + C::OFF_V + s * C::KVBYTES + b * C::BOX, &tmV, v_full + s, 64 * b, g,
+                          kt * 128 - (int)p.kv0);
+          }
           ++kv_iter;
         }
         ++unit_iter;
       }
-      if (unit_iter > 0) drain_wait(q_full, (unit_iter - 1) & 1);
+      if (unit_iter > 0) drain_wait(q_full, (unit_iter - 1) & 1, p.wait_ns);
       for (uint32_t t = (kv_iter > (uint32_t)C::NS ? kv_iter - C::NS : 0); t < kv_iter; ++t) {
-        drain_wait(k_full + t % C::NS, (t / C::NS) & 1);
-        drain_wait(v_full + t % C::NS, (t / C::NS) & 1);
+        drain_wait(k_full + t % C::NS, (t / C::NS) & 1, p.wait_ns);
+        drain_wait(v_full + t % C::NS, (t / C::NS) & 1, p.wait_ns);
       }
     }
   } else if (warp == 1) {
@@ -550,7 +560,7 @@ __global__ void __launch_bounds__(320, 1)
         ++unit_iter;
       }
       tc_commit(mma_drain);
-      drain_wait(mma_drain, 0);
+      drain_wait(mma_drain, 0, p.wait_ns);
     }
   } else {
     // ------------------------------------------------------------- softmax

@@ -25,6 +25,8 @@ struct FwdParams {
   float* o_part;          // [slots][hq][128][D]
   float* lse_part;        // [slots][hq][128]
   int* err;               // device error word
+  uint64_t wait_ns;       // pipeline wait limit of this launch
+  int32_t skip_v_load;    // test hook: CTA 0 leaves its first V load out, so a wait runs out
 };
 
 struct BwdParams {
@@ -42,6 +44,7 @@ struct BwdParams {
   const float* dvec;          // [hq][n_pad] D_i = <dO_i, O_i> (0 past the window)
   float* dq_acc;              // [n_pad][hq][D] fp32 dQ accumulator (reduced into through the tdq map)
   int* err;
+  uint64_t wait_ns;           // pipeline wait limit of this launch
 };
 
 template <int D>

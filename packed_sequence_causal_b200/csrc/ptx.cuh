@@ -18,8 +18,9 @@ enum : int {
   kErrSmemAlign = 1 << 4,
 };
 
-// A pipeline wait that has not completed after this long is treated as a
-// deadlock: the waiting role records an error and the CTA winds down.
+// Default time after which a pipeline wait that has not completed is treated
+// as a deadlock: the waiting role records an error and the CTA winds down.
+// Each launch carries its own limit (sap_set_wait_limit_ns).
 constexpr uint64_t kWaitLimitNs = 4000000000ull;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -67,18 +68,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 struct Guard {
   volatile int* abort_flag;  // shared memory, 0 = running
   int* err_word;             // global device error word
+  uint64_t limit_ns;         // this launch's wait limit
 };
 
 // Wait for the phase of `bar` with the given parity to complete.  Returns
-// false (after recording `code`) if the wait exceeds kWaitLimitNs or another
-// role of the CTA has already aborted.
+// false (after recording `code`) if the wait exceeds the launch's limit or
+// another role of the CTA has already aborted.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const Guard& g, int code) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*g.abort_flag) return false;
-    if (globaltimer() - t0 > kWaitLimitNs) {
+    if (globaltimer() - t0 > g.limit_ns) {
       *g.abort_flag = 1;
       atomicOr(g.err_word, code);
       return false;
@@ -97,10 +99,10 @@ __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, c
 // Bounded wait used while a CTA winds down: ignores the abort flag so that
 // copies and MMAs already in flight land before shared memory or TMEM is
 // released.
-__device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity) {
+__device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
   const uint64_t t0 = globaltimer();
   while (!mbar_try_wait(bar, parity))
-    if (globaltimer() - t0 > kWaitLimitNs) return false;
+    if (globaltimer() - t0 > limit_ns) return false;
   return true;
 }
 

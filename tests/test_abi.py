@@ -55,3 +55,11 @@ def test_misaligned_workspace_rejected_without_gpu():
     assert st == -4
     st = lib.sap_merge(plan.handle, bad_ws, need + 64, 2, 64, fake, fake, None)
     assert st == -4
+
+
+def test_wait_limit_arguments_checked_without_gpu():
+    lib = sap.load_library()
+    assert lib.sap_set_wait_limit_ns(10) == -1          # below 1 ms
+    assert lib.sap_set_wait_limit_ns(0) == 0            # default restored
+    assert lib.sap_test_arm_wait_timeout(0) == -1       # below 100 us
+    assert lib.sap_test_arm_wait_timeout(11_000_000_000) == -1
