@@ -82,7 +82,10 @@ typedef struct {
   int32_t q_tile, kv_tile, q_chunk, kv_chunk, tag;
 } sap_item_t;
 
-/* Build a plan on the host (no device work).  Validates cu_seqlens and the
+/* Build a plan on the host (no device work) -- the ahead-of-time schedule of the irregular,
+ * document-bounded attention of a packed batch (HSAP page, method details: the SAP schedule is
+ * generated before the run for the hybrid-context attention pattern; abstract: no attention
+ * across documents).  Validates cu_seqlens and the
  * chunking, lists the non-empty tiles in canonical order (q-tile ascending,
  * then kv-tile ascending; bit-exact with the tile-list definition above), and
  * derives the work schedule: forward units = (q-tile, kv-chunk) groups of
@@ -152,15 +155,18 @@ int sap_plan_window(sap_plan_t plan, int64_t* q_begin, int64_t* q_end, int64_t* 
  * transfer of the HSAP abstract, instead of a ring that passes every chunk. */
 int sap_plan_rank_spans(sap_plan_t plan, int32_t chunk, int64_t* spans, int32_t* n_spans);
 
-/* Canonical item list; host memory owned by the plan. */
+/* Canonical item list (see sap_item_t and sap_plan); host memory owned by the plan. */
 int sap_plan_items(sap_plan_t plan, const sap_item_t** items, int64_t* n_items);
 
-/* unmasked_pairs = sum over documents of L(L+1)/2 (per head);
+/* Plan statistics.  unmasked_pairs = sum over documents of L(L+1)/2 (per head) -- the pairs the
+ * packed causal mask keeps (HSAP abstract: attention only inside each document), the unit of the
+ * FLOP count;
  * n_partial_slots = forward units that write a partial (q-tiles with > 1 unit);
  * n_chunk_pairs = distinct (q_chunk, kv_chunk) pairs that hold an item. */
 int sap_plan_stats(sap_plan_t plan, int64_t* unmasked_pairs, int64_t* n_partial_slots, int32_t* n_chunk_pairs);
 
-/* Forward schedule, host memory owned by the plan:
+/* Forward schedule (the work order of sap_attn_fwd: one unit per partial of the HSAP abstract's
+ * partial attention computation), host memory owned by the plan:
  *   units: int32[n_units][4] = (q_tile, item_begin, item_count, slot), slot = -1
  *          when the unit writes O/LSE directly, else its partial slot;
  *   order: int32[n_units], heavy-first (item_count descending; ties by the kv chunk
@@ -169,7 +175,7 @@ int sap_plan_stats(sap_plan_t plan, int64_t* unmasked_pairs, int64_t* n_partial_
 int sap_plan_fwd_schedule(sap_plan_t plan, const int32_t** units, int64_t* n_units, const int32_t** order,
                           const int32_t** merges, int64_t* n_merges);
 
-/* Backward schedule, host memory owned by the plan:
+/* Backward schedule (the work order of sap_attn_bwd), host memory owned by the plan:
  *   entries:  int32[n_items][2] = (q_tile, tag), grouped by kv tile, q-tile descending;
  *   kv_units: int32[n_kv_units][3] = (kv_tile, first_entry, n_entries).  A unit is the part of one
  *             kv tile's entries whose q tiles fall in one band of 16 q tiles (q_tile / 16 equal), so a
@@ -177,7 +183,9 @@ int sap_plan_fwd_schedule(sap_plan_t plan, const int32_t** units, int64_t* n_uni
  *             heavy-first (n_entries descending, ties by kv tile) within a band. */
 int sap_plan_bwd_schedule(sap_plan_t plan, const int32_t** kv_units, int64_t* n_kv_units, const int32_t** entries);
 
-/* Fused-merge mode (enable != 0): the forward schedule gets one unit per
+/* Fused-merge mode (enable != 0; the pages have no such mode: it computes the merged result of
+ * the partials of sap_attn_fwd + sap_merge in one pass, which the exactness of the merge --
+ * explainer page, FAQ on equivalence with one device -- allows): the forward schedule gets one unit per
  * q-tile spanning all of its kv chunks, so sap_attn_fwd carries the online
  * softmax across chunk boundaries and writes O and LSE directly -- no fp32
  * partials, no forward workspace, and sap_merge has nothing to do.  The result
@@ -188,21 +196,25 @@ int sap_plan_bwd_schedule(sap_plan_t plan, const int32_t** kv_units, int64_t* n_
  * device call. */
 int sap_plan_set_fused_merge(sap_plan_t plan, int enable);
 
-/* Copy the plan's device arrays to the current device on `stream`.  Called
+/* Copy the plan's device arrays to the current device on `stream` (plumbing; no counterpart in
+ * the pages).  Called
  * implicitly by the first device call that needs them; calling it first keeps
  * the one host-to-device transfer out of later timed calls. */
 int sap_plan_upload(sap_plan_t plan, void* stream);
 
 void sap_plan_destroy(sap_plan_t plan);
 
-/* Workspace bytes for a call with these head counts (which = SAP_WS_FWD for
+/* Workspace bytes (plumbing; no counterpart in the pages) for a call with these head counts
+ * (which = SAP_WS_FWD for
  * sap_attn_fwd + sap_merge, SAP_WS_BWD for sap_attn_bwd).  The forward
  * workspace holds the fp32 partial outputs and LSEs of the partial slots; the
  * backward one holds the fp32 dQ, dK and dV accumulators and the per-row D and
  * LSE*log2(e). */
 int sap_workspace_size(sap_plan_t plan, int32_t hq, int32_t hkv, int32_t head_dim, int32_t which, size_t* bytes);
 
-/* Forward: for every forward unit (q-tile, kv-chunk) and head, the partial
+/* Forward (HSAP page, abstract: the partial attention computation of each part of the sequence
+ * against each part of its keys; method details: the attention pattern of hybrid-context
+ * sequences): for every forward unit (q-tile, kv-chunk) and head, the partial
  * attention of the q-tile's rows over that chunk's kv tiles (masked per tag),
  * with online softmax in fp32 on tcgen05 tensor cores.  A q-tile with one unit
  * writes bf16 O and fp32 LSE directly; the others leave fp32 partials (O, LSE)
@@ -212,14 +224,35 @@ int sap_attn_fwd(sap_plan_t plan, const void* q, const void* k, const void* v, i
                  int32_t head_dim, float softmax_scale, void* o, float* lse, void* workspace, size_t ws_bytes,
                  void* stream);
 
-/* Merge: for every q-tile with several partials, per (row, head)
+/* One part of the forward, so that the key/value exchange of sequence parallelism can overlap
+ * the device's own work (explainer page, compute-communication overlap bullet: compute the current
+ * block while the next one arrives).  In a rank plan the forward order lists first the units whose
+ * kv tiles all lie in the device's own chunk (sap_plan_fwd_local_units): part 1 runs those -- they
+ * read no received keys --, part 2 the others, part 0 all (= sap_attn_fwd).  max_ctas > 0 caps the
+ * persistent grid, leaving SMs to a transfer kernel running at the same time (0 = every SM).  The
+ * parts write disjoint outputs and partial slots of the same workspace; run parts 1 and 2 before
+ * sap_merge.  For a full plan part 1 is every unit and part 2 none.  Other arguments, layouts and
+ * errors as sap_attn_fwd (part or max_ctas out of range: SAP_ERR_INVALID_ARG). */
+int sap_attn_fwd_part(sap_plan_t plan, int32_t part, int32_t max_ctas, const void* q, const void* k, const void* v,
+                      int32_t hq, int32_t hkv, int32_t head_dim, float softmax_scale, void* o, float* lse,
+                      void* workspace, size_t ws_bytes, void* stream);
+
+/* Forward units of a plan, and how many of them (listed first in the forward order) lie entirely
+ * in a rank plan's own chunk; for a full plan both are the number of units. */
+int sap_plan_fwd_local_units(sap_plan_t plan, int64_t* n_local, int64_t* n_units);
+
+/* Merge (HSAP abstract: partial attention results combined into the attention of the whole
+ * sequence; explainer page, FAQ: the split computation equals the single-device one -- exact
+ * here up to rounding): for every q-tile with several partials, per (row, head)
  *   LSE = M + log sum_b exp(LSE_b - M), M = max_b LSE_b;  O = sum_b exp(LSE_b - LSE) O_b,
  * written as bf16 O and fp32 LSE.  Must follow sap_attn_fwd with the same
  * workspace; a no-op when no q-tile has more than one partial. */
 int sap_merge(sap_plan_t plan, const void* workspace, size_t ws_bytes, int32_t hq, int32_t head_dim, void* o,
               float* lse, void* stream);
 
-/* Backward with the merged O and LSE:  D_i = <dO_i, O_i>, P_ij = exp(S_ij - LSE_i),
+/* Backward (HSAP page, abstract: training of packed sequences; the gradient is the exact
+ * derivative of <dO, O> of the forward above) with the merged O and LSE:
+ * D_i = <dO_i, O_i>, P_ij = exp(S_ij - LSE_i),
  * dV_j = sum P_ij dO_i, dS_ij = P_ij (<dO_i, V_j> - D_i), dQ_i = scale sum_j dS_ij K_j,
  * dK_j = scale sum_i dS_ij Q_i, with dK/dV summed over the q heads of each kv
  * head.  Chunk pairs need no merge here: the final LSE normalises every pair
@@ -274,15 +307,16 @@ int sap_attn_fwd_static_scratch(sap_plan_t plan, const void* q, const void* k, c
                                 int32_t hkv, int32_t head_dim, float softmax_scale, void* o, float* lse,
                                 void* stream);
 
-/* Synchronise the current device and return SAP_OK, or SAP_ERR_DEVICE if a
+/* Failure detection (no counterpart in the pages).  Synchronise the current device and return
+ * SAP_OK, or SAP_ERR_DEVICE if a
  * kernel set the device error word (its code is stored in *code, then the word
  * is cleared). */
 int sap_device_status(int32_t* code);
 
-/* Text for a status code. */
+/* Text for a status code (no counterpart in the pages). */
 const char* sap_error_string(int status);
 
-/* The last cudaError_t seen by a call that returned SAP_ERR_CUDA. */
+/* The last cudaError_t seen by a call that returned SAP_ERR_CUDA (no counterpart in the pages). */
 int sap_last_cuda_error(void);
 
 /* Pipeline wait limit of every later kernel launch, in nanoseconds (0 restores the default of

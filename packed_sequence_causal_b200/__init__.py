@@ -20,6 +20,7 @@ from ._capi import (  # noqa: F401
     sap_attn_bwd,
     sap_attn_bwd_kv_add,
     sap_attn_fwd,
+    sap_attn_fwd_part,
     sap_attn_fwd_static_scratch,
     sap_device_status,
     sap_error_string,
@@ -30,6 +31,7 @@ from ._capi import (  # noqa: F401
     sap_plan_chunk_bounds,
     sap_plan_chunk_stats,
     sap_plan_chunks,
+    sap_plan_fwd_local_units,
     sap_plan_destroy,
     sap_plan_fwd_schedule,
     sap_plan_items,

@@ -79,6 +79,10 @@ def load_library():
     L.sap_workspace_size.argtypes = [P, i32, i32, i32, i32, ctypes.POINTER(sz)]
     L.sap_attn_fwd.restype = ctypes.c_int
     L.sap_attn_fwd.argtypes = [P, P, P, P, i32, i32, i32, f32, P, P, P, sz, P]
+    L.sap_attn_fwd_part.restype = ctypes.c_int
+    L.sap_attn_fwd_part.argtypes = [P, i32, i32, P, P, P, i32, i32, i32, f32, P, P, P, sz, P]
+    L.sap_plan_fwd_local_units.restype = ctypes.c_int
+    L.sap_plan_fwd_local_units.argtypes = [P, ctypes.POINTER(i64), ctypes.POINTER(i64)]
     L.sap_merge.restype = ctypes.c_int
     L.sap_merge.argtypes = [P, P, sz, i32, i32, P, P, P]
     L.sap_attn_bwd.restype = ctypes.c_int
@@ -289,6 +293,27 @@ def sap_attn_fwd(plan: Plan, q, k, v, softmax_scale: float, o, lse, workspace, s
     _check(load_library().sap_attn_fwd(plan.handle, _ptr(q), _ptr(k), _ptr(v), hq, hkv, d, float(softmax_scale),
                                        _ptr(o), _ptr(lse), _ptr(workspace), _nbytes(workspace),
                                        ctypes.c_void_p(_stream_ptr(stream))), "sap_attn_fwd")
+
+
+def sap_attn_fwd_part(plan: Plan, part: int, q, k, v, softmax_scale: float, o, lse, workspace, stream=None,
+                      max_ctas: int = 0):
+    """One part of the forward (1: own-chunk units of a rank plan, 2: the others, 0: all)."""
+    for t, nme in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
+        _bf16_3d(t, nme)
+    _, hq, d = q.shape
+    hkv = k.shape[1]
+    _check(load_library().sap_attn_fwd_part(plan.handle, int(part), int(max_ctas), _ptr(q), _ptr(k), _ptr(v), hq,
+                                            hkv, d, float(softmax_scale), _ptr(o), _ptr(lse), _ptr(workspace),
+                                            _nbytes(workspace), ctypes.c_void_p(_stream_ptr(stream))),
+           "sap_attn_fwd_part")
+
+
+def sap_plan_fwd_local_units(plan: Plan):
+    """(n_local, n_units): forward units, and those of a rank plan's own chunk (listed first)."""
+    a, b = ctypes.c_int64(), ctypes.c_int64()
+    _check(load_library().sap_plan_fwd_local_units(plan.handle, ctypes.byref(a), ctypes.byref(b)),
+           "sap_plan_fwd_local_units")
+    return a.value, b.value
 
 
 def sap_merge(plan: Plan, workspace, hq: int, head_dim: int, o, lse, stream=None):

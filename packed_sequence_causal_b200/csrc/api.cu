@@ -466,8 +466,22 @@ int sap_workspace_size(sap_plan_t plan, int32_t hq, int32_t hkv, int32_t head_di
 int sap_attn_fwd(sap_plan_t p, const void* q, const void* k, const void* v, int32_t hq, int32_t hkv,
                  int32_t head_dim, float softmax_scale, void* o, float* lse, void* workspace, size_t ws_bytes,
                  void* stream) {
+  return sap_attn_fwd_part(p, 0, 0, q, k, v, hq, hkv, head_dim, softmax_scale, o, lse, workspace, ws_bytes, stream);
+}
+
+int sap_plan_fwd_local_units(sap_plan_t plan, int64_t* n_local, int64_t* n_units) {
+  if (!plan) return SAP_ERR_INVALID_ARG;
+  if (n_local) *n_local = plan->n_local_units;
+  if (n_units) *n_units = (int64_t)plan->fwd_units.size() / 4;
+  return SAP_OK;
+}
+
+int sap_attn_fwd_part(sap_plan_t p, int32_t part, int32_t max_ctas, const void* q, const void* k, const void* v,
+                      int32_t hq, int32_t hkv, int32_t head_dim, float softmax_scale, void* o, float* lse,
+                      void* workspace, size_t ws_bytes, void* stream) {
   int rc = check_kernel_plan(p);
   if (rc) return rc;
+  if (part < 0 || part > 2 || max_ctas < 0) return SAP_ERR_INVALID_ARG;
   if ((rc = check_heads(hq, hkv, head_dim))) return rc;
   if (p->q_rows() == 0) return SAP_OK;
   if (!q || !k || !v || !o || !lse) return SAP_ERR_INVALID_ARG;
@@ -484,6 +498,12 @@ int sap_attn_fwd(sap_plan_t p, const void* q, const void* k, const void* v, int3
   if ((rc = make_map(&tk, k, p->kv_rows(), hkv, head_dim))) return rc;
   if ((rc = make_map(&tv, v, p->kv_rows(), hkv, head_dim))) return rc;
   sap::FwdParams fp = fwd_params(p, hq, hkv, softmax_scale);
+  // part 1: the first n_local_units of the order; part 2: the rest; part 0: all
+  const int64_t n_all = (int64_t)(p->fwd_units.size() / 4);
+  const int64_t first = part == 2 ? p->n_local_units : 0;
+  const int64_t count = part == 0 ? n_all : part == 1 ? p->n_local_units : n_all - p->n_local_units;
+  fp.order += first;
+  fp.n_units = (int32_t)count;
   if (const uint64_t t = g_test_timeout_ns.exchange(0)) {  // armed test hook: this launch only
     fp.skip_v_load = 1;
     fp.wait_ns = t;
@@ -497,7 +517,8 @@ int sap_attn_fwd(sap_plan_t p, const void* q, const void* k, const void* v, int3
   const int64_t work = (int64_t)fp.n_units * hq;
   if (work == 0) return SAP_OK;
   if (work > INT32_MAX) return SAP_ERR_INVALID_ARG;
-  const int grid = (int)(work < di->sms ? work : di->sms);
+  const int sms = max_ctas > 0 && max_ctas < di->sms ? max_ctas : di->sms;
+  const int grid = (int)(work < sms ? work : sms);
   cudaError_t e = head_dim == 64 ? sap::launch_fwd<64>(tq, tk, tv, fp, grid, static_cast<cudaStream_t>(stream))
                                  : sap::launch_fwd<128>(tq, tk, tv, fp, grid, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e);

@@ -71,6 +71,19 @@ void sap_plan_build_fwd_schedule(sap_plan_s* p, bool fused) {
     const int32_t cx = p->fwd_units[4 * x + 2], cy = p->fwd_units[4 * y + 2];
     return cx != cy ? cx > cy : chunk_of(x) < chunk_of(y);
   });
+  // A rank plan runs its own-chunk units first (each part keeps the heavy-first order), so that
+  // they can run while the keys of earlier chunks are still arriving.
+  p->n_local_units = (int64_t)nu;
+  if (p->rank_chunk >= 0) {
+    auto local = [&](int32_t u) {
+      const int32_t b = p->fwd_units[4 * u + 1], c = p->fwd_units[4 * u + 2];
+      for (int32_t e = b; e < b + c; ++e)
+        if (p->items[e].kv_chunk != p->rank_chunk) return false;
+      return true;
+    };
+    auto mid = std::stable_partition(p->fwd_order.begin(), p->fwd_order.end(), local);
+    p->n_local_units = mid - p->fwd_order.begin();
+  }
 }
 
 namespace {

@@ -37,6 +37,9 @@ struct sap_plan_s {
   std::vector<int32_t> merges;      // [M][3] (q_tile, first_slot, n_slots)
   int64_t n_slots = 0;
   bool fused_merge = false;  // forward units span all kv chunks of a q-tile (no partials)
+  // Rank plans list first (in fwd_order) the units whose kv tiles all lie in the device's own
+  // chunk: they read no received keys.  n_local_units of them; full plans count every unit.
+  int64_t n_local_units = 0;
 
   // backward schedule
   std::vector<int32_t> kv_units;    // [V][3] (kv_tile, first_entry, n_entries): band-major, heavy-first in a band

@@ -20,7 +20,8 @@ Data path of one device (rank plan of its chunk, see ``sap_plan_rank`` in includ
 
 Every step of the arithmetic runs in libsap.so's kernels; this module moves tensors and marshals
 arguments.  Each transfer lands in this device's own memory before a kernel reads it: no kernel
-reads another GPU's memory.  The exchanges are not overlapped with the local partial attention.
+reads another GPU's memory.  The forward's key/value exchange overlaps the units of the device's
+own chunk (they read no received keys); the backward's exchange of partials is not overlapped.
 """
 from __future__ import annotations
 
@@ -73,7 +74,18 @@ def exchange_kv(recv: Sequence[Span], send: Sequence[Span], window: dict, k_own,
                 group=None):
     """Assemble this device's key/value window [kv_begin, q_end) from its own K/V (rows [q_begin,
     q_end)) and the spans received from earlier devices; rows [kv_begin, span_begin) are zeros.
-    Returns (k_win, v_win, bytes_sent, bytes_received)."""
+    Returns (k_win, v_win, bytes_sent, bytes_received) once the transfers have completed."""
+    k_win, v_win, works, sent, got = start_exchange_kv(recv, send, window, k_own, v_own, peers, group)
+    for r in works:
+        r.wait()
+    return k_win, v_win, sent, got
+
+
+def start_exchange_kv(recv: Sequence[Span], send: Sequence[Span], window: dict, k_own, v_own,
+                      peers: Sequence[int], group=None):
+    """exchange_kv without waiting: returns (k_win, v_win, works, bytes_sent, bytes_received); the
+    received rows of the window are valid once every work has been waited for (on a CUDA device,
+    work.wait() orders the current stream after the transfer)."""
     import torch.distributed as dist
     kv0, q0, q1 = window["kv_begin"], window["q_begin"], window["q_end"]
     shape = (q1 - kv0,) + tuple(k_own.shape[1:])
@@ -91,10 +103,8 @@ def exchange_kv(recv: Sequence[Span], send: Sequence[Span], window: dict, k_own,
         ops.append(dist.P2POp(dist.isend, k_own[lo - q0:hi - q0].contiguous(), peers[dst], group))
         ops.append(dist.P2POp(dist.isend, v_own[lo - q0:hi - q0].contiguous(), peers[dst], group))
         sent += 2 * (hi - lo) * row_bytes
-    if ops:
-        for r in dist.batch_isend_irecv(ops):
-            r.wait()
-    return k_win, v_win, sent, got
+    works = dist.batch_isend_irecv(ops) if ops else []
+    return k_win, v_win, works, sent, got
 
 
 def exchange_kv_partials(recv: Sequence[Span], send: Sequence[Span], window: dict, dk_acc, dv_acc,
@@ -179,7 +189,7 @@ class SapAttention:
 
     def __init__(self, cu_seqlens, n: int, hq: int, hkv: int, head_dim: int, chunk: int, num_chunks: int, *,
                  peers: Optional[Sequence[int]] = None, group=None, balanced: bool = True,
-                 softmax_scale: Optional[float] = None, bounds=None):
+                 softmax_scale: Optional[float] = None, bounds=None, overlap_sms: int = 8):
         self.cu = np.asarray(cu_seqlens, dtype=np.int32)
         self.n, self.hq, self.hkv, self.d = int(n), int(hq), int(hkv), int(head_dim)
         self.chunk, self.num_chunks = int(chunk), int(num_chunks)
@@ -194,6 +204,8 @@ class SapAttention:
         self.group = group
         self.bytes = {"kv_sent": 0, "kv_received": 0, "dkv_sent": 0}
         self._ws_f = self._ws_b = None
+        # SMs left free for the transfer kernels while the own-chunk part of the forward runs
+        self.overlap_sms = int(overlap_sms)
         import torch.distributed as dist
         if dist.is_available() and dist.is_initialized():
             # point-to-point must not be the first collective of the group with NCCL
@@ -205,23 +217,37 @@ class SapAttention:
 
     # -- forward
     def forward(self, q, k, v):
-        k_win, v_win, sent, got = exchange_kv(self.recv, self.send, self.window, k, v, self.peers, self.group)
+        """Post the key/value exchange, run the units of the own chunk while it is in flight (on all
+        but overlap_sms SMs), then the units that read received keys, and the merge."""
+        k_win, v_win, works, sent, got = start_exchange_kv(self.recv, self.send, self.window, k, v, self.peers,
+                                                           self.group)
         self.bytes["kv_sent"], self.bytes["kv_received"] = sent, got
-        return self.attend(q, k_win, v_win)
+        self.attend(q, k_win, v_win, part=1)
+        for r in works:
+            r.wait()
+        return self.attend(q, k_win, v_win, part=2)
 
-    def attend(self, q, k_win, v_win):
-        """The local partial attention and merge over an assembled key/value window."""
+    def attend(self, q, k_win, v_win, part: int = 0):
+        """Local partial attention over an assembled key/value window: part 0 all units and the
+        merge; part 1 the own-chunk units only (returns None); part 2 the other units and the merge."""
         import torch
         self._q, self._k, self._v = q, k_win, v_win
         if self._ws_f is None:
             sap.sap_plan_upload(self.plan)
             self._ws_f = sap.alloc_workspace(self.plan, self.hq, self.hkv, self.d, sap.SAP_WS_FWD, q.device)
-        o = torch.empty_like(q)
-        lse = torch.empty((self.hq, max(self.q_rows, 1)), dtype=torch.float32, device=q.device)
-        sap.sap_attn_fwd(self.plan, q, k_win, v_win, self.scale, o, lse, self._ws_f)
-        sap.sap_merge(self.plan, self._ws_f, self.hq, self.d, o, lse)
-        self._o, self._lse = o, lse
-        return o, lse[:, : self.q_rows]
+        if part in (0, 1):
+            self._o = torch.empty_like(q)
+            self._lse = torch.empty((self.hq, max(self.q_rows, 1)), dtype=torch.float32, device=q.device)
+        max_ctas = 0
+        if part == 1 and self.recv and self.overlap_sms > 0:
+            sms = torch.cuda.get_device_properties(q.device).multi_processor_count
+            max_ctas = max(1, sms - self.overlap_sms)
+        sap.sap_attn_fwd_part(self.plan, part, q, k_win, v_win, self.scale, self._o, self._lse, self._ws_f,
+                              max_ctas=max_ctas)
+        if part == 1:
+            return None
+        sap.sap_merge(self.plan, self._ws_f, self.hq, self.d, self._o, self._lse)
+        return self._o, self._lse[:, : self.q_rows]
 
     # -- backward
     def backward(self, do):

@@ -63,6 +63,31 @@ def emulate_ranks(b, nchunks, balanced=True, bounds=None):
     return o, lse, dq, dk, dv, ranks
 
 
+def test_forward_parts_equal_the_whole_forward():
+    """Own-chunk units (part 1, on a capped grid) then the others (part 2) give the bytes of the
+    one-launch forward: the forward is deterministic and the parts write disjoint outputs."""
+    import packed_sequence_causal_b200 as sap
+    b = workloads.custom_batch([700, 60, 1500, 300, 37, 900, 599], 4, 2, 128, seed=54, with_do=False)
+    n = b.q.shape[0]
+    q, k, v = (t.to("cuda").contiguous() for t in (b.q, b.k, b.v))
+    for c in range(4):
+        r = sap_dist.SapAttention(b.cu_seqlens, n, 4, 2, 128, c, 4)
+        n_local, n_units = sap.sap_plan_fwd_local_units(r.plan)
+        assert 0 <= n_local <= n_units
+        w = r.window
+        k_win = torch.zeros((w["q_end"] - w["kv_begin"], 2, 128), dtype=k.dtype, device="cuda")
+        v_win = torch.zeros_like(k_win)
+        k_win[w["span_begin"] - w["kv_begin"]:] = k[w["span_begin"]:w["q_end"]]
+        v_win[w["span_begin"] - w["kv_begin"]:] = v[w["span_begin"]:w["q_end"]]
+        qr = q[w["q_begin"]:w["q_end"]].contiguous()
+        o0, l0 = (t.clone() for t in r.attend(qr, k_win, v_win))
+        r.overlap_sms = 100  # part 1 on a grid of far fewer CTAs than SMs
+        assert r.attend(qr, k_win, v_win, part=1) is None
+        o2, l2 = r.attend(qr, k_win, v_win, part=2)
+        assert torch.equal(o0, o2) and torch.equal(l0, l2)
+        assert sap.sap_device_status() == 0
+
+
 def _check(lens, hq, hkv, d, nchunks, balanced=True, seed=0):
     b = workloads.custom_batch(lens, hq, hkv, d, seed=seed, with_do=True)
     o, lse, dq, dk, dv, ranks = emulate_ranks(b, nchunks, balanced)

@@ -47,14 +47,27 @@ def _check_schedules(plan, items, n, nchunks, bm, bn):
     assert mi == len(merges)
     assert sap.sap_plan_stats(plan)["n_partial_slots"] == next_slot
     # heavy-first order: a permutation, non-increasing item counts; among equal counts the kv chunk
-    # of the unit's items ascending, then the unit index
+    # of the unit's items ascending, then the unit index.  A rank plan lists its own-chunk units
+    # first (units whose items all have kv_chunk = the plan's chunk) and keeps that order in each part.
     assert sorted(order.tolist()) == list(range(len(units)))
-    counts = units[order, 2]
-    assert np.all(np.diff(counts) <= 0)
+    n_local, n_units = sap.sap_plan_fwd_local_units(plan)
+    assert n_units == len(units)
+    rank = sap.sap_plan_window(plan)
+    own = None
+    if rank["q_end"] - rank["q_begin"] < n or rank["kv_begin"] > 0:
+        own = int(items[0, 2]) if len(items) else None
+    if own is not None:
+        for i, u in enumerate(order):
+            is_local = bool(np.all(items[units[u, 1]:units[u, 1] + units[u, 2], 3] == own))
+            assert is_local == (i < n_local)
+    else:
+        assert n_local == n_units
     chunk = {u: items[units[u, 1]][3] for u in range(len(units))}
-    for a, b in zip(order[:-1], order[1:]):
-        if units[a, 2] == units[b, 2]:
-            assert (chunk[a], a) < (chunk[b], b)
+    for part in (order[:n_local], order[n_local:]):
+        assert np.all(np.diff(units[part, 2]) <= 0)
+        for a, b in zip(part[:-1], part[1:]):
+            if units[a, 2] == units[b, 2]:
+                assert (chunk[a], a) < (chunk[b], b)
     # backward: every item once; each unit is the part of one kv tile's q-descending list that
     # falls in one band of 16 q tiles; units band-major (top band first), heavy-first within a
     # band, ties by kv tile

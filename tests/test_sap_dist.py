@@ -37,7 +37,9 @@ def _window_batch(self):
 class OracleSap(sap_dist.SapAttention):
     """SapAttention whose local steps are the fp64 oracle over the rank's window (test only)."""
 
-    def attend(self, q, k_win, v_win):
+    def attend(self, q, k_win, v_win, part=0):
+        if part == 1:  # the own-chunk part runs while the exchange is in flight; the oracle does it all below
+            return None
         kv0, q0, q1, cu = _window_batch(self)
         qw = torch.zeros(k_win.shape[:1] + q.shape[1:], dtype=torch.float64)
         qw[q0 - kv0:] = q  # window rows before the chunk are not this rank's queries
