@@ -255,6 +255,9 @@ def main():
                          "(sequence-aware exchange, with a Ulysses head split of degree --ulysses for hsap)")
     ap.add_argument("--ulysses", type=int, default=1, help="Ulysses (head-split) degree for --parallelism hsap")
     ap.add_argument("--equal-chunks", action="store_true", help="sap / hsap / emulation: equal chunks, not balanced")
+    ap.add_argument("--fwd-variant", default="1cta", choices=["1cta", "2cta"],
+                    help="forward kernel: one CTA per work item (default) or two-CTA clusters (tcgen05 "
+                         "cta_group::2; head_dim 128 with hq/hkv a multiple of 4)")
     ap.add_argument("--emulate-ranks", type=int, default=0,
                     help="one GPU: run the rank plans of a W-way sequence split one after another and report "
                          "per-rank kernel times (the exchange is emulated by device copies)")
@@ -284,6 +287,8 @@ def main():
     dev = torch.device("cuda", local_rank)
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    if args.fwd_variant == "2cta":
+        sap.sap_set_forward_variant(1)
 
     b = workloads.make_batch(w, rank_seed(args.seed, rank), device=str(dev), with_do=True)
     n, hq, hkv, d = w.n, w.hq, w.hkv, w.d
@@ -484,7 +489,7 @@ def main():
             "config": {"workload": w.name, "tokens": n, "docs": int(len(b.cu_seqlens) - 1), "hq": hq, "hkv": hkv,
                        "head_dim": d, "chunks": w.p, "tiles": n_items, "unmasked_pairs_per_head": pairs,
                        "flops_per_step": f_step, "parallelism": f"dp{world}" if world > 1 else "single",
-                       "fused_merge": bool(args.fused_merge),
+                       "fused_merge": bool(args.fused_merge), "fwd_variant": args.fwd_variant,
                        "l2": "inputs larger than L2 (Q, dO, O 1 GiB each); no flush"},
             "tokens_per_s": round(tokens_s, 1),
             "pct_bf16_peak": round(100 * value / world / burst, 2),

@@ -328,6 +328,17 @@ int sap_last_cuda_error(void);
  * documents) reports false timeouts.  Process-wide; no counterpart in the pages. */
 int sap_set_wait_limit_ns(uint64_t limit_ns);
 
+/* Forward kernel variant for later sap_attn_fwd / sap_attn_fwd_part calls (process-wide; the
+ * pages have no counterpart -- a B200 form of the same computation):
+ *   0 (default)  one CTA per work item: two query heads of a kv group share each K/V tile load;
+ *   1            two-CTA clusters (tcgen05 cta_group::2) where head_dim = 128 and hq / hkv is a
+ *                multiple of 4: a pair of SMs runs every MMA of four query heads of a kv group as
+ *                one M = 256 MMA, each SM loading half of every K and V tile; other shapes keep
+ *                variant 0.
+ * Both compute the same partials (within rounding: the MMAs' summation order may differ).
+ * SAP_ERR_INVALID_ARG for other values. */
+int sap_set_forward_variant(int32_t variant);
+
 /* Failure-detection test hook (no counterpart in the pages): arms the next sap_attn_fwd call
  * so that its launch uses wait_limit_ns (100 us .. 10 s, else SAP_ERR_INVALID_ARG) and its first
  * CTA leaves its first V tile out -- no copy is issued, so nothing is in flight -- and the MMA

@@ -41,6 +41,7 @@ from ._capi import (  # noqa: F401
     sap_plan_stats,
     sap_plan_upload,
     sap_plan_window,
+    sap_set_forward_variant,
     sap_set_wait_limit_ns,
     sap_workspace_kv_offsets,
     sap_workspace_size,

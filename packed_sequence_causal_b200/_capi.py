@@ -97,6 +97,8 @@ def load_library():
     L.sap_last_cuda_error.argtypes = []
     L.sap_set_wait_limit_ns.restype = ctypes.c_int
     L.sap_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+    L.sap_set_forward_variant.restype = ctypes.c_int
+    L.sap_set_forward_variant.argtypes = [i32]
     L.sap_test_arm_wait_timeout.restype = ctypes.c_int
     L.sap_test_arm_wait_timeout.argtypes = [ctypes.c_uint64]
     _lib = L
@@ -379,3 +381,8 @@ def sap_device_status() -> int:
 def sap_set_wait_limit_ns(limit_ns: int):
     """Pipeline wait limit of later kernel launches (0: the default 4 s)."""
     _check(load_library().sap_set_wait_limit_ns(int(limit_ns)), "sap_set_wait_limit_ns")
+
+
+def sap_set_forward_variant(variant: int):
+    """Forward kernel variant of later calls: 0 one CTA per work item, 1 two-CTA clusters (cta_group::2)."""
+    _check(load_library().sap_set_forward_variant(int(variant)), "sap_set_forward_variant")

@@ -22,6 +22,9 @@ thread_local int g_last_cuda_error = 0;
 std::atomic<uint64_t> g_wait_limit_ns{4000000000ull};
 std::atomic<uint64_t> g_test_timeout_ns{0};
 
+// Forward kernel variant (sap_set_forward_variant): 0 one CTA per work item, 1 two-CTA clusters.
+std::atomic<int> g_fwd_variant{0};
+
 // Device error word (bitwise OR of sap::kErr* codes), one per device.
 __device__ int g_device_err;
 
@@ -71,11 +74,11 @@ int device_info(DeviceInfo** out) {
   return SAP_OK;
 }
 
-// [rows][heads][hd] bf16 -> 3-D map with 128-row x 64-column boxes, 128-byte swizzle.
-int make_map(CUtensorMap* map, const void* base, int64_t rows, int32_t heads, int32_t hd) {
+// [rows][heads][hd] bf16 -> 3-D map with box_rows-row x 64-column boxes, 128-byte swizzle.
+int make_map(CUtensorMap* map, const void* base, int64_t rows, int32_t heads, int32_t hd, uint32_t box_rows = 128) {
   cuuint64_t dims[3] = {(cuuint64_t)hd, (cuuint64_t)heads, (cuuint64_t)rows};
   cuuint64_t strides[2] = {(cuuint64_t)hd * 2, (cuuint64_t)heads * hd * 2};
-  cuuint32_t box[3] = {64, 1, 128};
+  cuuint32_t box[3] = {64, 1, box_rows};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -493,9 +496,12 @@ int sap_attn_fwd_part(sap_plan_t p, int32_t part, int32_t max_ctas, const void* 
   DeviceInfo* di = nullptr;
   if ((rc = device_info(&di))) return rc;
   if ((rc = sap_plan_upload(p, stream))) return rc;
+  // the two-CTA variant where it applies (head_dim 128, GQA group a multiple of 4); each CTA of a
+  // pair loads 64-row halves of the K tiles
+  const bool two_cta = g_fwd_variant.load() == 1 && head_dim == 128 && (hq / hkv) % 4 == 0;
   CUtensorMap tq, tk, tv;
   if ((rc = make_map(&tq, q, p->q_rows(), hq, head_dim))) return rc;
-  if ((rc = make_map(&tk, k, p->kv_rows(), hkv, head_dim))) return rc;
+  if ((rc = make_map(&tk, k, p->kv_rows(), hkv, head_dim, two_cta ? 64 : 128))) return rc;
   if ((rc = make_map(&tv, v, p->kv_rows(), hkv, head_dim))) return rc;
   sap::FwdParams fp = fwd_params(p, hq, hkv, softmax_scale);
   // part 1: the first n_local_units of the order; part 2: the rest; part 0: all
@@ -519,8 +525,9 @@ int sap_attn_fwd_part(sap_plan_t p, int32_t part, int32_t max_ctas, const void* 
   if (work > INT32_MAX) return SAP_ERR_INVALID_ARG;
   const int sms = max_ctas > 0 && max_ctas < di->sms ? max_ctas : di->sms;
   const int grid = (int)(work < sms ? work : sms);
-  cudaError_t e = head_dim == 64 ? sap::launch_fwd<64>(tq, tk, tv, fp, grid, static_cast<cudaStream_t>(stream))
-                                 : sap::launch_fwd<128>(tq, tk, tv, fp, grid, static_cast<cudaStream_t>(stream));
+  cudaError_t e = head_dim == 64
+                      ? sap::launch_fwd<64>(tq, tk, tv, fp, grid, static_cast<cudaStream_t>(stream))
+                      : sap::launch_fwd<128>(tq, tk, tv, fp, grid, static_cast<cudaStream_t>(stream), two_cta);
   if (e != cudaSuccess) return cuda_fail(e);
   return SAP_OK;
 }
@@ -685,6 +692,12 @@ int sap_set_wait_limit_ns(uint64_t limit_ns) {
   if (limit_ns == 0) limit_ns = 4000000000ull;
   if (limit_ns < 1000000ull || limit_ns > 600000000000ull) return SAP_ERR_INVALID_ARG;
   g_wait_limit_ns.store(limit_ns);
+  return SAP_OK;
+}
+
+int sap_set_forward_variant(int32_t variant) {
+  if (variant != 0 && variant != 1) return SAP_ERR_INVALID_ARG;
+  g_fwd_variant.store(variant);
   return SAP_OK;
 }
 

@@ -364,28 +364,42 @@ __global__ void __launch_bounds__(192, 1)
 // Threads: warp 0 TMA, warp 1 MMA, warps 2..5 softmax of tile 0 (head 2p),
 // warps 6..9 softmax of tile 1 (head 2p+1).
 // TMEM columns: S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [256+D,256+2D).
-template <int D>
+//
+// CTA2 = true (D = 128, GQA group a multiple of 4): a cluster of two CTAs takes one q tile of
+// four query heads of a kv group, two per CTA, and runs every MMA as one two-CTA tcgen05.mma
+// (cta_group::2, M = 256) issued by the leader (cluster rank 0): rows 0..127 of the product are
+// the leader's tile, rows 128..255 the other CTA's.  The B operand is split between the pair:
+// each CTA loads only its half of every K tile (64 of the 128 kv rows) and of every V tile (64 of
+// the D columns), so a kv tile is read once per four heads and each SM's shared-memory operand
+// traffic for B halves.  Both CTAs' copies complete on the leader's barriers; the leader's
+// commits arrive on both CTAs' barriers; the other CTA's softmax threads arrive on the leader's
+// P barriers.  Softmax and epilogue are unchanged: each CTA owns the TMEM rows of its tiles.
+template <int D, bool CTA2>
 struct Fwd2Cfg {
-  static constexpr int NS = (D == 64) ? 3 : 2;
+  static_assert(!CTA2 || D == 128, "the two-CTA variant is built for head_dim 128");
+  static constexpr int NS = CTA2 ? 4 : (D == 64) ? 3 : 2;
   static constexpr int BOX = 128 * 128;
   static constexpr int QBYTES = D * 128 * 2;
-  static constexpr int KVBYTES = D * 128 * 2;
+  // one stage: this CTA's K tile and V tile (CTA2: its 64 kv rows of K, its 64 columns of V)
+  static constexpr int KBYTES = CTA2 ? D * 64 * 2 : D * 128 * 2;
+  static constexpr int VBYTES = CTA2 ? 64 * 128 * 2 : D * 128 * 2;
+  static constexpr int KSLAB = CTA2 ? 64 * 128 : BOX;  // bytes between the 64-column slabs of a K tile
   static constexpr int OFF_Q0 = 0;
   static constexpr int OFF_Q1 = QBYTES;
   static constexpr int OFF_K = 2 * QBYTES;
-  static constexpr int OFF_V = OFF_K + NS * KVBYTES;
-  static constexpr int OFF_BAR = OFF_V + NS * KVBYTES;
+  static constexpr int OFF_V = OFF_K + NS * KBYTES;
+  static constexpr int OFF_BAR = OFF_V + NS * VBYTES;
   static constexpr int NBAR = 2 + 4 * NS + 2 + 2 + 2 + 2;
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16;
   static constexpr int THREADS = 320;
   static constexpr uint32_t COL_O = 256;
 };
 
-template <int D>
+template <int D, bool CTA2>
 __global__ void __launch_bounds__(320, 1)
     sap_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
-  using C = Fwd2Cfg<D>;
+  using C = Fwd2Cfg<D, CTA2>;
   extern __shared__ __align__(1024) uint8_t smem[];
   if (smem_u32(smem) & 1023u) {
     if (threadIdx.x == 0) atomicOr(p.err, kErrSmemAlign);
@@ -408,6 +422,17 @@ __global__ void __launch_bounds__(320, 1)
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const Guard guard{abort_flag, p.err, p.wait_ns};
+  const uint32_t rank = CTA2 ? cluster_ctarank() : 0u;  // CTA2: 0 = leader of the pair
+  const bool leader = rank == 0;
+  // CTA2: the leader's barrier at the same offset (shared::cluster address); where the loads of
+  // both CTAs complete and the P arrivals of both CTAs land
+  auto at_leader = [&](uint64_t* bar) { return mapa_shared(smem_u32(bar), 0); };
+  auto commit = [&](uint64_t* bar) {  // arrives on this barrier in both CTAs (CTA2) or in this CTA
+    if constexpr (CTA2)
+      tc_commit_pair(bar, 0x3);
+    else
+      tc_commit(bar);
+  };
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -420,8 +445,8 @@ __global__ void __launch_bounds__(320, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(s_full + b, 1);
-      mbar_init(p_full + b, 128);
-      mbar_init(p_half + b, 128);
+      mbar_init(p_full + b, CTA2 ? 256 : 128);
+      mbar_init(p_half + b, CTA2 ? 256 : 128);
     }
     mbar_init(o_done, 1);
     mbar_init(mma_drain, 1);
@@ -429,16 +454,25 @@ __global__ void __launch_bounds__(320, 1)
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, 512);
-    tmem_relinquish();
+    if constexpr (CTA2) {
+      tmem_alloc_pair(tmem_slot, 512);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, 512);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (CTA2) cluster_sync();  // both CTAs' barriers are initialised before any remote use
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  const int pairs = p.hq / 2;
+  constexpr int HEADS = CTA2 ? 4 : 2;  // query heads per work item (two per CTA)
+  const int pairs = p.hq / HEADS;
   const int total = p.n_units * pairs;
+  const int w0 = CTA2 ? (int)(blockIdx.x / 2) : (int)blockIdx.x;  // work items are per cluster
+  const int wstep = CTA2 ? (int)(gridDim.x / 2) : (int)gridDim.x;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -448,14 +482,21 @@ __global__ void __launch_bounds__(320, 1)
       prefetch_tmap(&tmV);
       uint32_t kv_iter = 0, unit_iter = 0;
       bool ok = true;
-      for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
-        const int u = p.order[w / pairs], h0 = 2 * (w % pairs), g = h0 / p.group;
+      for (int w = w0; w < total && ok; w += wstep) {
+        const int u = p.order[w / pairs], h0 = HEADS * (w % pairs) + 2 * (int)rank, g = h0 / p.group;
         const int qt = p.units[4 * u], ib = p.units[4 * u + 1], ic = p.units[4 * u + 2];
         if (!mbar_wait(q_empty, (unit_iter & 1) ^ 1, guard, kErrTimeoutLoad)) break;
-        mbar_arrive_expect_tx(q_full, 2 * C::QBYTES);
+        if (leader) mbar_arrive_expect_tx(q_full, (CTA2 ? 4 : 2) * C::QBYTES);
         for (int b = 0; b < D / 64; ++b) {
-          tma_load_3d(smem + C::OFF_Q0 + b * C::BOX, &tmQ, q_full, 64 * b, h0, qt * 128 - (int)p.q0);
-          tma_load_3d(smem + C::OFF_Q1 + b * C::BOX, &tmQ, q_full, 64 * b, h0 + 1, qt * 128 - (int)p.q0);
+          if constexpr (CTA2) {
+            tma_load_3d_pair(smem + C::OFF_Q0 + b * C::BOX, &tmQ, at_leader(q_full), 64 * b, h0,
+                             qt * 128 - (int)p.q0);
+            tma_load_3d_pair(smem + C::OFF_Q1 + b * C::BOX, &tmQ, at_leader(q_full), 64 * b, h0 + 1,
+                             qt * 128 - (int)p.q0);
+          } else {
+            tma_load_3d(smem + C::OFF_Q0 + b * C::BOX, &tmQ, q_full, 64 * b, h0, qt * 128 - (int)p.q0);
+            tma_load_3d(smem + C::OFF_Q1 + b * C::BOX, &tmQ, q_full, 64 * b, h0 + 1, qt * 128 - (int)p.q0);
+          }
         }
         int kt_next = p.items[5 * ib + 1];
         for (int t = 0; t < ic; ++t) {
@@ -464,33 +505,53 @@ __global__ void __launch_bounds__(320, 1)
           const int s = kv_iter % C::NS;
           const uint32_t ph = (kv_iter / C::NS) & 1;
           if (!mbar_wait(k_empty + s, ph ^ 1, guard, kErrTimeoutLoad)) { ok = false; break; }
-          mbar_arrive_expect_tx(k_full + s, C::KVBYTES);
-          for (int b = 0; b < D / 64; ++b)
-            tma_load_3d(smem + C::OFF_K + s * C::KVBYTES + b * C::BOX, &tmK, k_full + s, 64 * b, g,
-                        kt * 128 - (int)p.kv0);
+          if (leader) mbar_arrive_expect_tx(k_full + s, (CTA2 ? 2 : 1) * C::KBYTES);
+          for (int b = 0; b < D / 64; ++b) {
+            if constexpr (CTA2)  // this CTA's 64 kv rows of the tile (the K map has 64-row boxes)
+              tma_load_3d_pair(smem + C::OFF_K + s * C::KBYTES + b * C::KSLAB, &tmK, at_leader(k_full + s), 64 * b,
+                               g, kt * 128 - (int)p.kv0 + 64 * (int)rank);
+            else
+              tma_load_3d(smem + C::OFF_K + s * C::KBYTES + b * C::BOX, &tmK, k_full + s, 64 * b, g,
+                          kt * 128 - (int)p.kv0);
+          }
           if (!mbar_wait(v_empty + s, ph ^ 1, guard, kErrTimeoutLoad)) { ok = false; break; }
           // test hook: CTA 0 leaves its first V tile out (nothing is issued), so the MMA wait on it runs out
           if (!(p.skip_v_load && blockIdx.x == 0 && kv_iter == 0)) {
-            mbar_arrive_expect_tx(v_full + s, C::KVBYTES);
-            for (int b = 0; b < D / 64; ++b)
-              tma_load_3d(smem + C::OFF_V + s * C::KVBYTES + b * C::BOX, &tmV, v_full + s, 64 * b, g,
-                          kt * 128 - (int)p.kv0);
+            if (leader) mbar_arrive_expect_tx(v_full + s, (CTA2 ? 2 : 1) * C::VBYTES);
+            if constexpr (CTA2)  // this CTA's 64 of the D columns, all 128 kv rows
+              tma_load_3d_pair(smem + C::OFF_V + s * C::VBYTES, &tmV, at_leader(v_full + s), 64 * (int)rank, g,
+                               kt * 128 - (int)p.kv0);
+            else
+              for (int b = 0; b < D / 64; ++b)
+                tma_load_3d(smem + C::OFF_V + s * C::VBYTES + b * C::BOX, &tmV, v_full + s, 64 * b, g,
+                            kt * 128 - (int)p.kv0);
           }
           ++kv_iter;
         }
         ++unit_iter;
       }
-      if (unit_iter > 0) drain_wait(q_full, (unit_iter - 1) & 1, p.wait_ns);
-      for (uint32_t t = (kv_iter > (uint32_t)C::NS ? kv_iter - C::NS : 0); t < kv_iter; ++t) {
-        drain_wait(k_full + t % C::NS, (t / C::NS) & 1, p.wait_ns);
-        drain_wait(v_full + t % C::NS, (t / C::NS) & 1, p.wait_ns);
+      // Let every copy land before the CTA can exit.  CTA2: the full barriers live in the leader and
+      // count both CTAs' copies; the other CTA is held at the final cluster barrier until then.
+      if (leader) {
+        if (unit_iter > 0) drain_wait(q_full, (unit_iter - 1) & 1, p.wait_ns);
+        for (uint32_t t = (kv_iter > (uint32_t)C::NS ? kv_iter - C::NS : 0); t < kv_iter; ++t) {
+          drain_wait(k_full + t % C::NS, (t / C::NS) & 1, p.wait_ns);
+          drain_wait(v_full + t % C::NS, (t / C::NS) & 1, p.wait_ns);
+        }
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    if (lane == 0 && leader) {  // CTA2: only the leader issues the pair's MMAs
       // ----------------------------------------------------------------- MMA
-      constexpr uint32_t idesc_qk = idesc_bf16(128, 128, false, false);
-      constexpr uint32_t idesc_pv = idesc_bf16(128, D, false, true);
+      constexpr uint32_t idesc_qk = idesc_bf16(CTA2 ? 256 : 128, 128, false, false);
+      constexpr uint32_t idesc_pv = idesc_bf16(CTA2 ? 256 : 128, D, false, true);
+      // P arrivals come from both CTAs' threads under CTA2: wait at cluster scope
+      auto wait_p = [&](uint64_t* bar, uint32_t parity) {
+        if constexpr (CTA2)
+          return mbar_wait_cluster(bar, parity, guard, kErrTimeoutMma);
+        else
+          return mbar_wait(bar, parity, guard, kErrTimeoutMma);
+      };
       const uint32_t sQ0 = smem_u32(smem + C::OFF_Q0), sQ1 = smem_u32(smem + C::OFF_Q1);
       const uint32_t sK = smem_u32(smem + C::OFF_K), sV = smem_u32(smem + C::OFF_V);
       uint32_t kv_iter = 0, unit_iter = 0, tile_iter = 0;  // tile_iter counts kv tiles (per tile barrier phases)
@@ -500,21 +561,29 @@ __global__ void __launch_bounds__(320, 1)
         const int s = it % C::NS;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t ko = (kk / 4) * C::BOX + (kk % 4) * 32;
-          mma_bf16(tmem + 128 * tile, sdesc_sw128(sQ + ko, 16, 1024),
-                   sdesc_sw128(sK + s * C::KVBYTES + ko, 16, 1024), idesc_qk, kk > 0);
+          const uint64_t a = sdesc_sw128(sQ + (kk / 4) * C::BOX + (kk % 4) * 32, 16, 1024);
+          const uint64_t bd = sdesc_sw128(sK + s * C::KBYTES + (kk / 4) * C::KSLAB + (kk % 4) * 32, 16, 1024);
+          if constexpr (CTA2)
+            mma_bf16_pair(tmem + 128 * tile, a, bd, idesc_qk, kk > 0);
+          else
+            mma_bf16(tmem + 128 * tile, a, bd, idesc_qk, kk > 0);
         }
-        tc_commit(s_full + tile);
+        commit(s_full + tile);
       };
       auto issue_pv = [&](int tile, uint32_t it, bool first, int part) {  // O_tile += P_tile V_it (half), P from TMEM
         const int s = it % C::NS;
 #pragma unroll
-        for (int kk = 4 * part; kk < 4 * part + 4; ++kk)
-          mma_bf16_tmem_a(tmem + C::COL_O + D * tile, tmem + 128 * tile + kk * 8,
-                          sdesc_sw128(sV + s * C::KVBYTES + kk * 2048, C::BOX, 1024), idesc_pv,
-                          (first && kk == 0) ? 0u : 1u);
+        for (int kk = 4 * part; kk < 4 * part + 4; ++kk) {
+          const uint64_t bd = sdesc_sw128(sV + s * C::VBYTES + kk * 2048, C::BOX, 1024);
+          if constexpr (CTA2)
+            mma_bf16_tmem_a_pair(tmem + C::COL_O + D * tile, tmem + 128 * tile + kk * 8, bd, idesc_pv,
+                                 (first && kk == 0) ? 0u : 1u);
+          else
+            mma_bf16_tmem_a(tmem + C::COL_O + D * tile, tmem + 128 * tile + kk * 8, bd, idesc_pv,
+                            (first && kk == 0) ? 0u : 1u);
+        }
       };
-      for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
+      for (int w = w0; w < total && ok; w += wstep) {
         const int u = p.order[w / pairs];
         const int ic = p.units[4 * u + 2];
         if (!mbar_wait(q_full, unit_iter & 1, guard, kErrTimeoutMma)) break;
@@ -522,14 +591,14 @@ __global__ void __launch_bounds__(320, 1)
         tc_fence_after();
         issue_s(0, kv_iter);
         issue_s(1, kv_iter);
-        tc_commit(k_empty + kv_iter % C::NS);
+        commit(k_empty + kv_iter % C::NS);
         for (int j = 0; j < ic; ++j, ++tile_iter) {
           const uint32_t it = kv_iter + j;
           if (!mbar_wait(v_full + it % C::NS, (it / C::NS) & 1, guard, kErrTimeoutMma)) { ok = false; break; }
-          if (!mbar_wait(p_half + 0, tile_iter & 1, guard, kErrTimeoutMma)) { ok = false; break; }
+          if (!wait_p(p_half + 0, tile_iter & 1)) { ok = false; break; }
           tc_fence_after();
           issue_pv(0, it, j == 0, 0);
-          if (!mbar_wait(p_full + 0, tile_iter & 1, guard, kErrTimeoutMma)) { ok = false; break; }
+          if (!wait_p(p_full + 0, tile_iter & 1)) { ok = false; break; }
           tc_fence_after();
           issue_pv(0, it, j == 0, 1);
           const bool more = j + 1 < ic;
@@ -541,25 +610,29 @@ __global__ void __launch_bounds__(320, 1)
             tc_fence_after();
             issue_s(0, it + 1);  // rewrites S0/P0 only after PV0 (issued above) has read P0
           }
-          if (!mbar_wait(p_half + 1, tile_iter & 1, guard, kErrTimeoutMma)) { ok = false; break; }
+          if (!wait_p(p_half + 1, tile_iter & 1)) { ok = false; break; }
           tc_fence_after();
           issue_pv(1, it, j == 0, 0);
-          if (!mbar_wait(p_full + 1, tile_iter & 1, guard, kErrTimeoutMma)) { ok = false; break; }
+          if (!wait_p(p_full + 1, tile_iter & 1)) { ok = false; break; }
           tc_fence_after();
           issue_pv(1, it, j == 0, 1);
-          tc_commit(v_empty + it % C::NS);
+          commit(v_empty + it % C::NS);
           if (more) {
             issue_s(1, it + 1);
-            tc_commit(k_empty + (it + 1) % C::NS);
+            commit(k_empty + (it + 1) % C::NS);
           }
         }
         if (!ok) break;
-        tc_commit(o_done);
-        tc_commit(q_empty);
+        commit(o_done);
+        commit(q_empty);
         kv_iter += ic;
         ++unit_iter;
       }
-      tc_commit(mma_drain);
+      // Wait for every MMA this thread issued before TMEM is released (CTA2: the leader's own barrier).
+      if constexpr (CTA2)
+        tc_commit_pair(mma_drain, 0x1);
+      else
+        tc_commit(mma_drain);
       drain_wait(mma_drain, 0, p.wait_ns);
     }
   } else {
@@ -572,8 +645,8 @@ __global__ void __launch_bounds__(320, 1)
     uint32_t tile_iter = 0, unit_iter = 0;
     const float sl2 = p.scale_log2;
     bool ok = true;
-    for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
-      const int u = p.order[w / pairs], h = 2 * (w % pairs) + tile;
+    for (int w = w0; w < total && ok; w += wstep) {
+      const int u = p.order[w / pairs], h = HEADS * (w % pairs) + 2 * (int)rank + tile;
       const int qt = p.units[4 * u], ib = p.units[4 * u + 1], ic = p.units[4 * u + 2], slot = p.units[4 * u + 3];
       const int64_t i = (int64_t)qt * 128 + r;
       const bool real_row = i < p.q_end;
@@ -645,12 +718,18 @@ __global__ void __launch_bounds__(320, 1)
           tmem_st32_u(lane_base + colS + 32 * half, pk);  // P over the S columns already read
           if (half == 0) {  // PV over kv rows 0..63 may start while the second half is computed
             tc_fence_before();
-            mbar_arrive(p_half + tile);
+            if constexpr (CTA2)
+              mbar_arrive_remote(at_leader(p_half + tile));
+            else
+              mbar_arrive(p_half + tile);
           }
         }
         l += (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
         tc_fence_before();
-        mbar_arrive(p_full + tile);
+        if constexpr (CTA2)
+          mbar_arrive_remote(at_leader(p_full + tile));
+        else
+          mbar_arrive(p_full + tile);
       }
       if (!ok) break;
       // ------------------------------------------------------------ epilogue
@@ -698,10 +777,16 @@ __global__ void __launch_bounds__(320, 1)
 
   tc_fence_before();
   __syncthreads();
+  // CTA2: the leader's MMAs read this CTA's shared and tensor memory, and this CTA's copies
+  // complete on the leader's barriers; neither CTA leaves before the leader has drained both.
+  if constexpr (CTA2) cluster_sync();
   tc_fence_after();
   if (warp == 1) {
     __syncwarp();
-    tmem_dealloc(tmem, 512);
+    if constexpr (CTA2)
+      tmem_dealloc_pair(tmem, 512);
+    else
+      tmem_dealloc(tmem, 512);
   }
 }
 
@@ -712,14 +797,49 @@ int fwd_smem_bytes() {
 
 template <int D>
 cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
-                       int grid, cudaStream_t stream) {
+                       int grid, cudaStream_t stream, bool two_cta) {
+  if constexpr (D == 128) {
+    if (two_cta) {  // clusters of two CTAs, four heads of a kv group per cluster (group % 4 == 0)
+      if (p.group % 4 != 0) return cudaErrorInvalidValue;
+      auto kern = sap_fwd_pair_kernel<128, true>;
+      using C2 = Fwd2Cfg<128, true>;
+      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C2::SMEM);
+      if (e != cudaSuccess) return e;
+      cudaLaunchConfig_t cfg = {};
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 2;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.blockDim = dim3(C2::THREADS);
+      cfg.dynamicSmemBytes = C2::SMEM;
+      cfg.stream = stream;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      // persistent clusters: no more than can be resident at once, nor than there is work
+      int max_clusters = 0;
+      cfg.gridDim = dim3(2 * (grid / 2 > 0 ? grid / 2 : 1));
+      e = cudaOccupancyMaxActiveClusters(&max_clusters, kern, &cfg);
+      if (e != cudaSuccess) return e;
+      const int64_t work = (int64_t)p.n_units * (p.hq / 4);
+      int64_t clusters = grid / 2;
+      if (max_clusters > 0 && clusters > max_clusters) clusters = max_clusters;
+      if (clusters > work) clusters = work;
+      if (clusters <= 0) return cudaSuccess;
+      cfg.gridDim = dim3((unsigned)(2 * clusters));
+      e = cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, p);
+      if (e != cudaSuccess) return e;
+      return cudaGetLastError();
+    }
+  }
   if (p.group % 2 == 0) {  // two heads of one kv group per CTA
     const int64_t work = (int64_t)p.n_units * (p.hq / 2);
     const int g2 = (int)(work < grid ? work : grid);
-    auto kern2 = sap_fwd_pair_kernel<D>;
-    cudaError_t e = cudaFuncSetAttribute(kern2, cudaFuncAttributeMaxDynamicSharedMemorySize, Fwd2Cfg<D>::SMEM);
+    auto kern2 = sap_fwd_pair_kernel<D, false>;
+    cudaError_t e =
+        cudaFuncSetAttribute(kern2, cudaFuncAttributeMaxDynamicSharedMemorySize, Fwd2Cfg<D, false>::SMEM);
     if (e != cudaSuccess) return e;
-    if (g2 > 0) kern2<<<g2, Fwd2Cfg<D>::THREADS, Fwd2Cfg<D>::SMEM, stream>>>(tq, tk, tv, p);
+    if (g2 > 0) kern2<<<g2, Fwd2Cfg<D, false>::THREADS, Fwd2Cfg<D, false>::SMEM, stream>>>(tq, tk, tv, p);
     return cudaGetLastError();
   }
   auto kern = sap_fwd_kernel<D>;
@@ -730,8 +850,8 @@ cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
 }
 
 template cudaError_t launch_fwd<64>(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const FwdParams&,
-                                    int, cudaStream_t);
+                                    int, cudaStream_t, bool);
 template cudaError_t launch_fwd<128>(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const FwdParams&,
-                                     int, cudaStream_t);
+                                     int, cudaStream_t, bool);
 
 }  // namespace sap

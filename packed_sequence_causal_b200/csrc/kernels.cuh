@@ -47,9 +47,11 @@ struct BwdParams {
   uint64_t wait_ns;           // pipeline wait limit of this launch
 };
 
+// two_cta (D = 128, hq / hkv a multiple of 4): the two-CTA cluster variant; tk must then be a map
+// with 64-row boxes (each CTA of a pair loads half of every K tile).  grid: CTAs (SMs) to use.
 template <int D>
 cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
-                       int grid, cudaStream_t stream);
+                       int grid, cudaStream_t stream, bool two_cta = false);
 
 template <int D>
 cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,

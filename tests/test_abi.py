@@ -63,3 +63,10 @@ def test_wait_limit_arguments_checked_without_gpu():
     assert lib.sap_set_wait_limit_ns(0) == 0            # default restored
     assert lib.sap_test_arm_wait_timeout(0) == -1       # below 100 us
     assert lib.sap_test_arm_wait_timeout(11_000_000_000) == -1
+
+
+def test_forward_variant_argument_checked_without_gpu():
+    lib = sap.load_library()
+    assert lib.sap_set_forward_variant(2) == -1
+    assert lib.sap_set_forward_variant(-1) == -1
+    assert lib.sap_set_forward_variant(0) == 0
