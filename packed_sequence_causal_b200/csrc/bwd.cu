@@ -82,10 +82,10 @@ struct BwdCfg {
   static constexpr uint32_t COL_DQ = DQ_T ? COL_R2 : 384;
 };
 
-// 448 threads x 144 registers fit the SM's 64K registers (one CTA per SM); the register cap
-// keeps the compiler from settling on 128 registers with spills.
+// 448 threads are granted registers as 16 warps, so 128 registers per thread is the ceiling
+// (the compiler spills a few bytes at d = 128 and d = 64 to stay under it).
 template <int D>
-__global__ void __maxnreg__(144)
+__global__ void __launch_bounds__(448, 1)
     sap_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                    const __grid_constant__ CUtensorMap tmDQ, const __grid_constant__ CUtensorMap tmDKV,
