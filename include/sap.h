@@ -341,10 +341,11 @@ int sap_set_forward_variant(int32_t variant);
 
 /* Failure-detection test hook (no counterpart in the pages): arms the next sap_attn_fwd call
  * so that its launch uses wait_limit_ns (100 us .. 10 s, else SAP_ERR_INVALID_ARG) and its first
- * CTA leaves its first V tile out -- no copy is issued, so nothing is in flight -- and the MMA
- * wait on that tile runs out.  The call returns SAP_OK; sap_device_status() then reports
- * SAP_ERR_DEVICE with the MMA timeout bit, and the outputs of that launch are incomplete.  The
- * hook disarms itself at that launch; later calls are normal. */
+ * CTA leaves its first V tile out -- no copy is issued, so nothing is in flight --: the MMA
+ * issuer's wait for that tile, or the producer's wait for its ring stage to be released,
+ * whichever started first, runs out.  The call returns SAP_OK; sap_device_status() then reports
+ * SAP_ERR_DEVICE with that wait's timeout bit, and the outputs of that launch are incomplete.
+ * The hook disarms itself at that launch; later calls are normal. */
 int sap_test_arm_wait_timeout(uint64_t wait_limit_ns);
 
 #ifdef __cplusplus
