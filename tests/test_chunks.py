@@ -114,13 +114,17 @@ def test_planner_balanced_cut_matches_oracle_workloads(name):
 @pytest.mark.parametrize("name,nchunks", [("llama31_8b_128k", 8), ("hybrid_512k", 16), ("llama32_1b_32k", 8),
                                           ("llama2_13b_64k_short", 16)])
 def test_balanced_cut_evens_out_the_work(name, nchunks):
-    """Per-chunk item counts: max / mean <= 1.1 with the balanced cut (equal chunks reach ~3x at 128K)."""
+    """Per-chunk item counts and unmasked pairs: max / mean <= 1.1 with the balanced cut (equal
+    chunks reach ~3x at 128K and 512K)."""
     w = workloads.WORKLOADS[name]
     cu = workloads.cu_seqlens_from_lengths(workloads.doc_lengths(w, 0))
     plan = sap.sap_plan_chunks(cu, w.n, sap.sap_balanced_chunks(cu, w.n, nchunks))
-    items = sap.sap_plan_chunk_stats(plan)["items"]
+    st = sap.sap_plan_chunk_stats(plan)
+    items, pairs = st["items"], st["pairs"]
     assert items.sum() == len(sap.sap_plan_items(plan))
+    assert pairs.sum() == oracle.unmasked_pairs(cu)
     assert items.max() / items.mean() <= 1.1, items
+    assert pairs.max() / pairs.mean() <= 1.1, pairs
     eq = sap.sap_plan_chunk_stats(sap.sap_plan(cu, w.n, nchunks))["items"]
     assert items.max() <= eq.max()
 
