@@ -373,7 +373,8 @@ __global__ void __launch_bounds__(192, 1)
 // the D columns), so a kv tile is read once per four heads and each SM's shared-memory operand
 // traffic for B halves.  Both CTAs' copies complete on the leader's barriers; the leader's
 // commits arrive on both CTAs' barriers; the other CTA's softmax threads arrive on the leader's
-// P barriers.  Softmax and epilogue are unchanged: each CTA owns the TMEM rows of its tiles.
+// P barriers (remote arrivals; the tensor-memory fences order their P writes before the MMAs).
+// Softmax and epilogue are unchanged: each CTA owns the TMEM rows of its tiles.
 template <int D, bool CTA2>
 struct Fwd2Cfg {
   static_assert(!CTA2 || D == 128, "the two-CTA variant is built for head_dim 128");
@@ -545,13 +546,8 @@ __global__ void __launch_bounds__(320, 1)
       // ----------------------------------------------------------------- MMA
       constexpr uint32_t idesc_qk = idesc_bf16(CTA2 ? 256 : 128, 128, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16(CTA2 ? 256 : 128, D, false, true);
-      // P arrivals come from both CTAs' threads under CTA2: wait at cluster scope
-      auto wait_p = [&](uint64_t* bar, uint32_t parity) {
-        if constexpr (CTA2)
-          return mbar_wait_cluster(bar, parity, guard, kErrTimeoutMma);
-        else
-          return mbar_wait(bar, parity, guard, kErrTimeoutMma);
-      };
+      // P arrivals (CTA2: from both CTAs' softmax threads)
+      auto wait_p = [&](uint64_t* bar, uint32_t parity) { return mbar_wait(bar, parity, guard, kErrTimeoutMma); };
       const uint32_t sQ0 = smem_u32(smem + C::OFF_Q0), sQ1 = smem_u32(smem + C::OFF_Q1);
       const uint32_t sK = smem_u32(smem + C::OFF_K), sV = smem_u32(smem + C::OFF_V);
       uint32_t kv_iter = 0, unit_iter = 0, tile_iter = 0;  // tile_iter counts kv tiles (per tile barrier phases)

@@ -106,34 +106,6 @@ __device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity, uint6
   return true;
 }
 
-// Cluster-scope form of mbar_try_wait, for barriers that threads of the other CTA of a
-// two-CTA cluster arrive on (their release at cluster scope pairs with this acquire).
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, const Guard& g, int code) {
-  if (mbar_try_wait_cluster(bar, parity)) return true;
-  const uint64_t t0 = globaltimer();
-  while (true) {
-    if (mbar_try_wait_cluster(bar, parity)) return true;
-    if (*g.abort_flag) return false;
-    if (globaltimer() - t0 > g.limit_ns) {
-      *g.abort_flag = 1;
-      atomicOr(g.err_word, code);
-      return false;
-    }
-  }
-}
-
 // ------------------------------------------------------------------ clusters
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {
@@ -149,9 +121,13 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t local_addr, uint32_t ra
   return r;
 }
 
-// Arrive (release at cluster scope) on an mbarrier given by its shared::cluster address.
+// Arrive on an mbarrier given by its shared::cluster address (possibly the other CTA's).  The
+// arrivals order tensor-memory writes (tcgen05.st, then tcgen05.wait::st and
+// tcgen05.fence::before_thread_sync) before the MMAs the waiter issues after
+// tcgen05.fence::after_thread_sync; no generic-memory data is handed over, so the default
+// (CTA-scope) release suffices and no cluster-scope memory fence is paid per arrival.
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
 // Every thread of both CTAs of the cluster arrives and waits (release / acquire at cluster scope).
