@@ -24,13 +24,17 @@ from packed_sequence_causal_b200 import sap_dist
 pytestmark = pytest.mark.gpu
 
 
-def emulate_ranks(b, nchunks, balanced=True, bounds=None):
+def emulate_ranks(b, nchunks, balanced=True, bounds=None, fused_merge=False):
     """Run every rank plan of the split on this GPU; returns the assembled (O, LSE, dQ, dK, dV)."""
+    import packed_sequence_causal_b200 as sap
     n, hq, d = b.q.shape
     hkv = b.k.shape[1]
     q, k, v, do = (t.to("cuda").contiguous() for t in (b.q, b.k, b.v, b.do))
     ranks = [sap_dist.SapAttention(b.cu_seqlens, n, hq, hkv, d, c, nchunks, balanced=balanced, bounds=bounds)
              for c in range(nchunks)]
+    if fused_merge:
+        for r in ranks:
+            sap.sap_plan_set_fused_merge(r.plan, True)
     o = torch.empty_like(q)
     lse = torch.empty((hq, n), dtype=torch.float32, device="cuda")
     for r in ranks:
@@ -88,9 +92,9 @@ def test_forward_parts_equal_the_whole_forward():
         assert sap.sap_device_status() == 0
 
 
-def _check(lens, hq, hkv, d, nchunks, balanced=True, seed=0):
+def _check(lens, hq, hkv, d, nchunks, balanced=True, seed=0, fused_merge=False):
     b = workloads.custom_batch(lens, hq, hkv, d, seed=seed, with_do=True)
-    o, lse, dq, dk, dv, ranks = emulate_ranks(b, nchunks, balanced)
+    o, lse, dq, dk, dv, ranks = emulate_ranks(b, nchunks, balanced, fused_merge=fused_merge)
     scale = 1.0 / math.sqrt(d)
     ro, rl = oracle.attn_fwd(b.q, b.k, b.v, b.cu_seqlens, scale)
     assert_close(o, ro, "O (rank plans)")
@@ -120,3 +124,9 @@ def test_rank_plans_ragged_tail_and_long_span():
     ranks = _check([70, 3000, 1, 929, 1000], 8, 2, 128, 5, seed=53)
     assert max(len(r.recv) for r in ranks) >= 2
     assert any(r.window["kv_begin"] < r.window["span_begin"] for r in ranks if r.recv)
+
+
+def test_rank_plans_with_fused_merge():
+    """Each device's rank plan in fused-merge mode (one forward unit per q tile over every kv chunk
+    it sees, received spans included): same result as the oracle."""
+    _check([700, 60, 1500, 300, 37, 900, 599], 4, 2, 128, 4, seed=55, fused_merge=True)
