@@ -147,7 +147,7 @@ __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* m
 
 // Two-CTA form: the tile lands in this CTA's shared memory and its bytes complete the
 // transaction of the mbarrier at `bar_cluster` -- the leader CTA's barrier of the pair
-// (a shared::cluster address).  Not a multicast load: every CTA fetches its own tile.
+// (a shared::cluster address).  Each CTA fetches its own tile; no copy is shared between CTAs.
 __device__ __forceinline__ void tma_load_3d_pair(void* smem_dst, const CUtensorMap* map, uint32_t bar_cluster, int x,
                                                  int y, int z) {
   asm volatile(
