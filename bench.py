@@ -316,7 +316,11 @@ def main():
     ws_f = sap.alloc_workspace(plan, hq, hkv, d, sap.SAP_WS_FWD, dev)
     ws_b = sap.alloc_workspace(plan, hq, hkv, d, sap.SAP_WS_BWD, dev)
     stream = torch.cuda.current_stream()
-    launches_per_step = 1 + (1 if len(merges) else 0) + 3
+    # forward, merge (when some q tile has several partials), backward pre-pass, backward, dQ
+    # conversion, dK/dV conversion (when some kv tile goes through the fp32 accumulators; one launch
+    # per 65535 such tiles)
+    n_acc = len(sap.sap_plan_bwd_direct(plan)) - int(sap.sap_plan_bwd_direct(plan).sum())
+    launches_per_step = 1 + (1 if len(merges) else 0) + 3 + (n_acc + 65534) // 65535
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
 

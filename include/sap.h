@@ -177,11 +177,19 @@ int sap_plan_fwd_schedule(sap_plan_t plan, const int32_t** units, int64_t* n_uni
 
 /* Backward schedule (the work order of sap_attn_bwd), host memory owned by the plan:
  *   entries:  int32[n_items][2] = (q_tile, tag), grouped by kv tile, q-tile descending;
- *   kv_units: int32[n_kv_units][3] = (kv_tile, first_entry, n_entries).  A unit is the part of one
- *             kv tile's entries whose q tiles fall in one band of 16 q tiles (q_tile / 16 equal), so a
- *             kv tile may have several units.  Units are ordered band-major (top band first) and
- *             heavy-first (n_entries descending, ties by kv tile) within a band. */
+ *   kv_units: int32[n_kv_units][3] = (kv_tile, first_entry, n_entries).  A kv tile whose entries
+ *             number at most 16 is one unit; a longer list is cut into the parts whose q tiles fall
+ *             in one band of 16 q tiles (q_tile / 16 equal), so such a kv tile has several units.
+ *             Units are ordered band-major (top band first; a unit's band is that of its first,
+ *             highest q tile) and heavy-first (n_entries descending, ties by kv tile) within a band. */
 int sap_plan_bwd_schedule(sap_plan_t plan, const int32_t** kv_units, int64_t* n_kv_units, const int32_t** entries);
+
+/* Direct dK/dV stores of sap_attn_bwd, host memory owned by the plan: int32[n_tiles] over the kv
+ * tiles of the plan's key/value window (tile l = rows [kv_begin + l * block_n, ...)), 1 where the
+ * tile has exactly one backward unit in a full plan.  That unit writes the tile's dK and dV as
+ * bf16 directly; every other tile (all tiles of a rank plan, whose dK/dV rows may still receive
+ * other devices' partials) is accumulated in fp32 in the workspace and converted at the end. */
+int sap_plan_bwd_direct(sap_plan_t plan, const int32_t** flags, int64_t* n_tiles);
 
 /* Fused-merge mode (enable != 0; the pages have no such mode: it computes the merged result of
  * the partials of sap_attn_fwd + sap_merge in one pass, which the exactness of the merge --
@@ -258,24 +266,26 @@ int sap_merge(sap_plan_t plan, const void* workspace, size_t ws_bytes, int32_t h
  * head.  Chunk pairs need no merge here: the final LSE normalises every pair
  * and their gradients add.  dQ, dK and dV are accumulated in fp32 in the
  * workspace (dQ once per (q tile, kv tile, head), dK/dV once per backward unit)
- * and converted to bf16 at the end. */
+ * and converted to bf16 at the end, except the dK/dV of kv tiles with a single unit in a full
+ * plan (sap_plan_bwd_direct), which that unit stores as bf16 directly. */
 int sap_attn_bwd(sap_plan_t plan, const void* q, const void* k, const void* v, const void* o, const float* lse,
                  const void* dout, int32_t hq, int32_t hkv, int32_t head_dim, float softmax_scale, void* dq,
                  void* dk, void* dv, void* workspace, size_t ws_bytes, void* stream);
 
 /* Byte offsets, inside the backward workspace, of the fp32 dK and dV accumulators that
  * sap_attn_bwd leaves behind: [rows][hkv][head_dim] each, row r = token kv_begin + r of the plan's
- * window (row stride hkv * head_dim floats).  Under sequence parallelism the rows below q_begin
- * hold this device's partial dK/dV for other devices' tokens: sent to their owners and added
- * there with sap_attn_bwd_kv_add. */
+ * window (row stride hkv * head_dim floats).  Under sequence parallelism (rank plans) the rows
+ * below q_begin hold this device's partial dK/dV for other devices' tokens: sent to their owners
+ * and added there with sap_attn_bwd_kv_add.  In a full plan the rows of directly stored tiles
+ * (sap_plan_bwd_direct) are not written. */
 int sap_workspace_kv_offsets(sap_plan_t plan, int32_t hq, int32_t hkv, int32_t head_dim, size_t* dk_offset,
                              size_t* dv_offset);
 
 /* Adds received fp32 partial gradients into the dK/dV accumulators that the last sap_attn_bwd with
- * this plan and workspace left behind, and rewrites the bf16 dK/dV of those rows:
+ * this rank plan and workspace left behind, and rewrites the bf16 dK/dV of those rows:
  *   acc[t] += part[t - row_begin]; dk[t] = bf16(acc_dK[t]); dv[t] = bf16(acc_dV[t])
  * for tokens t in [row_begin, row_begin + rows), which must lie in the plan's key/value window
- * (SAP_ERR_INVALID_ARG otherwise).  dk_part, dv_part: fp32 [rows][hkv][head_dim], 16-byte
+ * (SAP_ERR_INVALID_ARG otherwise, and for a full plan, whose accumulators skip direct tiles).  dk_part, dv_part: fp32 [rows][hkv][head_dim], 16-byte
  * aligned; dk, dv: the bf16 window buffers sap_attn_bwd wrote.  Several calls add up (the chunk
  * pair gradients of the backward add, as on one device); calls on one stream are ordered. */
 int sap_attn_bwd_kv_add(sap_plan_t plan, void* workspace, size_t ws_bytes, int32_t hq, int32_t hkv, int32_t head_dim,

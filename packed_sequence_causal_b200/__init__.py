@@ -27,6 +27,7 @@ from ._capi import (  # noqa: F401
     sap_balanced_chunks,
     sap_merge,
     sap_plan,
+    sap_plan_bwd_direct,
     sap_plan_bwd_schedule,
     sap_plan_chunk_bounds,
     sap_plan_chunk_stats,

@@ -69,6 +69,8 @@ def load_library():
     L.sap_plan_fwd_schedule.argtypes = [P, PP, ctypes.POINTER(i64), PP, PP, ctypes.POINTER(i64)]
     L.sap_plan_bwd_schedule.restype = ctypes.c_int
     L.sap_plan_bwd_schedule.argtypes = [P, PP, ctypes.POINTER(i64), PP]
+    L.sap_plan_bwd_direct.restype = ctypes.c_int
+    L.sap_plan_bwd_direct.argtypes = [P, PP, ctypes.POINTER(i64)]
     L.sap_plan_set_fused_merge.restype = ctypes.c_int
     L.sap_plan_set_fused_merge.argtypes = [P, ctypes.c_int]
     L.sap_plan_upload.restype = ctypes.c_int
@@ -242,6 +244,13 @@ def sap_plan_bwd_schedule(plan: Plan):
            "sap_plan_bwd_schedule")
     n_items = len(sap_plan_items(plan))
     return _copy_i32(k, nk.value, 3), _copy_i32(e, n_items, 2)
+
+
+def sap_plan_bwd_direct(plan: Plan) -> np.ndarray:
+    """int32 [kv tiles of the window]: 1 where sap_attn_bwd stores the tile's dK/dV directly."""
+    f, nt = ctypes.c_void_p(), ctypes.c_int64()
+    _check(load_library().sap_plan_bwd_direct(plan.handle, ctypes.byref(f), ctypes.byref(nt)), "sap_plan_bwd_direct")
+    return _copy_i32(f, nt.value, 1)
 
 
 def _stream_ptr(stream) -> Optional[int]:

@@ -144,7 +144,7 @@ FwdWs fwd_ws(const sap_plan_s* p, int32_t hq, int32_t hd) {
   return w;
 }
 struct BwdWs {
-  size_t dq_acc = 0, dkv_acc = 0, dvec = 0, lse2 = 0, total = 0;
+  size_t dq_acc = 0, dkv_acc = 0, dvec = 0, lse2 = 0, work_next = 0, total = 0;
   int64_t n_pad = 0, n_pad_kv = 0;  // query-side and key/value-side window rows, rounded up to 128
 };
 BwdWs bwd_ws(const sap_plan_s* p, int32_t hq, int32_t hkv, int32_t hd) {
@@ -155,7 +155,8 @@ BwdWs bwd_ws(const sap_plan_s* p, int32_t hq, int32_t hkv, int32_t hd) {
   w.dkv_acc = round_up(w.n_pad * hq * hd * 4, 1024);                        // [2][n_pad_kv][hkv][hd] fp32
   w.dvec = w.dkv_acc + round_up(2 * w.n_pad_kv * hkv * hd * 4, 256);        // [hq][n_pad]
   w.lse2 = w.dvec + round_up(w.n_pad * hq * 4, 256);                        // [hq][n_pad]
-  w.total = w.lse2 + round_up(w.n_pad * hq * 4, 256);
+  w.work_next = w.lse2 + round_up(w.n_pad * hq * 4, 256);                   // int: work counter
+  w.total = w.work_next + 256;
   return w;
 }
 
@@ -365,6 +366,13 @@ int sap_plan_bwd_schedule(sap_plan_t plan, const int32_t** kv_units, int64_t* n_
   return SAP_OK;
 }
 
+int sap_plan_bwd_direct(sap_plan_t plan, const int32_t** flags, int64_t* n_tiles) {
+  if (!plan) return SAP_ERR_INVALID_ARG;
+  if (flags) *flags = plan->kv_direct.data();
+  if (n_tiles) *n_tiles = (int64_t)plan->kv_direct.size();
+  return SAP_OK;
+}
+
 int sap_plan_upload(sap_plan_t p, void* stream) {
   if (!p) return SAP_ERR_INVALID_ARG;
   int dev = 0;
@@ -387,6 +395,8 @@ int sap_plan_upload(sap_plan_t p, void* stream) {
   p->off_merges = place(p->merges.size());
   p->off_kv_units = place(p->kv_units.size());
   p->off_kv_entries = place(p->kv_entries.size());
+  p->off_kv_direct = place(p->kv_direct.size());
+  p->off_kv_acc_tiles = place(p->kv_acc_tiles.size());
   p->off_tok_lo = place(p->tok_lo.size());
   p->off_tok_hi = place(p->tok_hi.size());
   p->dev_words = off > 0 ? off : 64;
@@ -405,6 +415,8 @@ int sap_plan_upload(sap_plan_t p, void* stream) {
   if (e == cudaSuccess) e = put(p->off_merges, p->merges.data(), p->merges.size());
   if (e == cudaSuccess) e = put(p->off_kv_units, p->kv_units.data(), p->kv_units.size());
   if (e == cudaSuccess) e = put(p->off_kv_entries, p->kv_entries.data(), p->kv_entries.size());
+  if (e == cudaSuccess) e = put(p->off_kv_direct, p->kv_direct.data(), p->kv_direct.size());
+  if (e == cudaSuccess) e = put(p->off_kv_acc_tiles, p->kv_acc_tiles.data(), p->kv_acc_tiles.size());
   if (e == cudaSuccess) e = put(p->off_tok_lo, p->tok_lo.data(), p->tok_lo.size());
   if (e == cudaSuccess) e = put(p->off_tok_hi, p->tok_hi.data(), p->tok_hi.size());
   // The host arrays stay alive with the plan, but copies from pageable memory
@@ -593,12 +605,19 @@ int sap_attn_bwd(sap_plan_t p, const void* q, const void* k, const void* v, cons
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const __nv_bfloat16* ob = static_cast<const __nv_bfloat16*>(o);
   const __nv_bfloat16* dob = static_cast<const __nv_bfloat16*>(dout);
-  cudaError_t e = head_dim == 64 ? sap::launch_bwd_pre<64>(ob, dob, lse, p->q_rows(), ws.n_pad, ws.n_pad_kv, hq, hkv,
-                                                           dvec, lse2, dq_acc, dkv_acc, s)
-                                 : sap::launch_bwd_pre<128>(ob, dob, lse, p->q_rows(), ws.n_pad, ws.n_pad_kv, hq, hkv,
-                                                            dvec, lse2, dq_acc, dkv_acc, s);
-  if (e != cudaSuccess) return cuda_fail(e);
+  // bf16 dK / dV outputs, stored directly by the units of kv tiles that have no other unit
+  CUtensorMap tdk, tdv;
+  if ((rc = make_map(&tdk, dk, p->kv_rows(), hkv, head_dim))) return rc;
+  if ((rc = make_map(&tdv, dv, p->kv_rows(), hkv, head_dim))) return rc;
   const int32_t* base = static_cast<const int32_t*>(p->dev);
+  const int32_t* kv_direct = base + p->off_kv_direct;
+  cudaError_t e = head_dim == 64 ? sap::launch_bwd_pre<64>(ob, dob, lse, p->q_rows(), ws.n_pad, ws.n_pad_kv, hq, hkv,
+                                                           dvec, lse2, dq_acc, dkv_acc, kv_direct,
+                                                           reinterpret_cast<int*>(wsb + ws.work_next), s)
+                                 : sap::launch_bwd_pre<128>(ob, dob, lse, p->q_rows(), ws.n_pad, ws.n_pad_kv, hq, hkv,
+                                                            dvec, lse2, dq_acc, dkv_acc, kv_direct,
+                                                            reinterpret_cast<int*>(wsb + ws.work_next), s);
+  if (e != cudaSuccess) return cuda_fail(e);
   sap::BwdParams bp;
   bp.kv_units = base + p->off_kv_units;
   bp.entries = base + p->off_kv_entries;
@@ -617,18 +636,21 @@ int sap_attn_bwd(sap_plan_t p, const void* q, const void* k, const void* v, cons
   bp.lse2 = lse2;
   bp.dvec = dvec;
   bp.dq_acc = dq_acc;
+  bp.kv_direct = kv_direct;
+  bp.work_next = reinterpret_cast<int*>(wsb + ws.work_next);  // zeroed by the pre-pass
   bp.err = di->err;
   bp.wait_ns = g_wait_limit_ns.load();
   const int64_t work = (int64_t)bp.n_kv_units * hkv;
   if (work > 0) {
     const int grid = (int)(work < di->sms ? work : di->sms);
-    e = head_dim == 64 ? sap::launch_bwd<64>(tq, tk, tv, tdo, tdq, tdkv, bp, grid, s)
-                       : sap::launch_bwd<128>(tq, tk, tv, tdo, tdq, tdkv, bp, grid, s);
+    e = head_dim == 64 ? sap::launch_bwd<64>(tq, tk, tv, tdo, tdq, tdkv, tdk, tdv, bp, grid, s)
+                       : sap::launch_bwd<128>(tq, tk, tv, tdo, tdq, tdkv, tdk, tdv, bp, grid, s);
     if (e != cudaSuccess) return cuda_fail(e);
   }
   e = sap::launch_bwd_post(dq_acc, static_cast<__nv_bfloat16*>(dq), p->q_rows() * hq * head_dim, dkv_acc,
                            static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv),
-                           p->kv_rows() * hkv * head_dim, ws.n_pad_kv * hkv * head_dim, s);
+                           p->kv_rows() * hkv * head_dim, ws.n_pad_kv * hkv * head_dim, base + p->off_kv_acc_tiles,
+                           (int64_t)p->kv_acc_tiles.size(), (int64_t)hkv * head_dim, s);
   if (e != cudaSuccess) return cuda_fail(e);
   return SAP_OK;
 }
@@ -639,6 +661,7 @@ int sap_attn_bwd_kv_add(sap_plan_t p, void* workspace, size_t ws_bytes, int32_t 
   if (!p) return SAP_ERR_INVALID_ARG;
   int rc = check_heads(hq, hkv, head_dim);
   if (rc) return rc;
+  if (p->rank_chunk < 0) return SAP_ERR_INVALID_ARG;  // a full plan's accumulators may skip direct tiles
   if (rows == 0) return SAP_OK;
   if (rows < 0 || row_begin < p->kv_begin || row_begin + rows > p->q_end) return SAP_ERR_INVALID_ARG;
   if (!dk_part || !dv_part || !dk || !dv || !aligned16(dk_part) || !aligned16(dv_part) || !aligned16(dk) ||

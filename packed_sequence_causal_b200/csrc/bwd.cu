@@ -8,7 +8,9 @@
 //
 // Persistent CTA, warp-specialised (448 threads), transposed so that a TMEM
 // lane is a key/value row:
-//   warp 0       TMA producer: K, V per work item; per iteration Q, dO and the
+//   warp 0       work index of each item (dynamic: the next free item in
+//                schedule order, shared with the other roles through a ring);
+//                TMA producer: K, V per work item; per iteration Q, dO and the
 //                128 LSE*log2(e) and D values of the q tile, through an
 //                NSQ-stage ring.
 //   warp 1       TMEM owner and tcgen05.mma issuer (one thread); S^T_j = K Q_j^T
@@ -37,7 +39,8 @@
 //                buffer; D = 64: dQ staged as two 128-byte-swizzled boxes of 32
 //                features), and at the end of a work item add its dK and dV into
 //                fp32 accumulators the same way (the conversion to bf16 is a
-//                separate elementwise kernel).
+//                separate elementwise kernel), or, when the kv tile has no other
+//                unit, store them as bf16 directly.
 //
 // TMEM columns: dK [0,D), dV [D,2D), R1 = S^T/P^T [2D, 2D+128),
 // R2 = dP^T [2D+128, 2D+256); dQ shares R2 for D = 128 (dP^T is consumed
@@ -70,10 +73,11 @@ struct BwdCfg {
   static constexpr int EPI_BYTES = 128 * 64 * 4;
   static constexpr int OFF_EPI = (D == 128) ? OFF_DS : OFF_ST + NSQ * STAGE;
   static constexpr int OFF_BAR = (D == 128) ? OFF_ST + NSQ * STAGE : OFF_EPI + EPI_BYTES;
-  static constexpr int NBAR = 2 + 2 * NSQ + 13;
+  static constexpr int NW = 4;  // work-index ring depth
+  static constexpr int NBAR = 2 + 2 * NSQ + 13 + 2 * NW;
   // The dynamic shared window starts 1024-byte aligned (checked at run time),
-  // so no alignment slack is reserved: the D = 128 layout needs 231,592 bytes.
-  static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16;
+  // so no alignment slack is reserved: the D = 128 layout needs 231,672 bytes.
+  static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 4 * NW;
   static_assert(SMEM <= 232448, "shared memory per block");
   static_assert(OFF_EPI % 1024 == 0 && OFF_ST % 1024 == 0 && STAGE % 1024 == 0, "128-byte swizzle alignment");
   static constexpr int THREADS = 448;
@@ -89,6 +93,7 @@ __global__ void __launch_bounds__(448, 1)
     sap_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                    const __grid_constant__ CUtensorMap tmDQ, const __grid_constant__ CUtensorMap tmDKV,
+                   const __grid_constant__ CUtensorMap tmDK, const __grid_constant__ CUtensorMap tmDV,
                    const BwdParams p) {
   using C = BwdCfg<D>;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -114,8 +119,11 @@ __global__ void __launch_bounds__(448, 1)
   uint64_t* stg_ready = mma_drain + 1;  // the staging buffer holds a dQ or dK/dV piece
   uint64_t* stg_free = stg_ready + 1;   // its reduction has read the staging buffer
   uint64_t* dv_done = stg_free + 1;     // dV has read dO: dS^T may go over it (d = 128)
+  uint64_t* sched_full = dv_done + 1;   // [NW] the producer wrote the next work index
+  uint64_t* sched_empty = sched_full + C::NW;  // [NW] every other role has read it
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBAR);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* sched_w = reinterpret_cast<volatile int*>(smem + C::OFF_BAR + C::NBAR * 8 + 16);  // [NW]
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const Guard guard{abort_flag, p.err, p.wait_ns};
@@ -140,6 +148,10 @@ __global__ void __launch_bounds__(448, 1)
     mbar_init(stg_ready, 128);
     mbar_init(stg_free, 1);
     mbar_init(dv_done, 1);
+    for (int s = 0; s < C::NW; ++s) {
+      mbar_init(sched_full + s, 1);
+      mbar_init(sched_empty + s, 1 + 8 + 4);  // the MMA thread, the 8 softmax and 4 drain warps
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -154,6 +166,19 @@ __global__ void __launch_bounds__(448, 1)
 
   const int total = p.n_kv_units * p.hkv;
   const int G = p.group;
+  // Work items are handed out dynamically in schedule order: the first one of a CTA is blockIdx.x,
+  // the next ones come from a global counter, so a CTA that finishes early takes the next item
+  // (list scheduling of the heavy-first order).  The producer fetches each index and publishes it
+  // through a ring of NW slots; every other role reads the indices in the same order.  -1 ends the
+  // sequence; -2 marks a wait that ran out.
+  auto take_work = [&](uint32_t i, int code) -> int {  // warp-wide (softmax and drain warps)
+    const int s = i % C::NW;
+    if (!mbar_wait_warp(sched_full + s, (i / C::NW) & 1, guard, code)) return -2;
+    const int w = sched_w[s];
+    __syncwarp();
+    if (lane == 0) mbar_arrive(sched_empty + s);
+    return w;
+  };
 
   if (warp == 0) {
     if (lane == 0) {
@@ -164,7 +189,14 @@ __global__ void __launch_bounds__(448, 1)
       prefetch_tmap(&tmDO);
       uint32_t unit_iter = 0, q_iter = 0;
       bool ok = true;
-      for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
+      for (uint32_t wi = 0; ok; ++wi) {
+        const int ws = wi % C::NW;
+        if (!mbar_wait(sched_empty + ws, ((wi / C::NW) & 1) ^ 1, guard, kErrTimeoutLoad)) break;
+        int w = wi == 0 ? (int)blockIdx.x : (int)gridDim.x + atomicAdd(p.work_next, 1);
+        if (w >= total) w = -1;
+        sched_w[ws] = w;
+        mbar_arrive(sched_full + ws);
+        if (w < 0) break;
         const int u = w / p.hkv, g = w % p.hkv;
         const int kt = p.kv_units[3 * u], e0 = p.kv_units[3 * u + 1], ne = p.kv_units[3 * u + 2];
         if (!mbar_wait(kv_empty, (unit_iter & 1) ^ 1, guard, kErrTimeoutLoad)) break;
@@ -227,7 +259,12 @@ __global__ void __launch_bounds__(448, 1)
         tc_commit(s_full);
         return true;
       };
-      for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
+      for (uint32_t wi = 0; ok; ++wi) {
+        const int ws = wi % C::NW;
+        if (!mbar_wait(sched_full + ws, (wi / C::NW) & 1, guard, kErrTimeoutMma)) break;
+        const int w = sched_w[ws];
+        mbar_arrive(sched_empty + ws);
+        if (w < 0) break;
         const int u = w / p.hkv;
         const int n_it = p.kv_units[3 * u + 2] * G;
         if (!mbar_wait(kv_full, unit_iter & 1, guard, kErrTimeoutMma)) break;
@@ -301,7 +338,12 @@ __global__ void __launch_bounds__(448, 1)
     const float sl2 = p.scale_log2;
     uint32_t it = 0;
     bool ok = true;
-    for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
+    for (uint32_t wi = 0; ok; ++wi) {
+      const int w = take_work(wi, kErrTimeoutSoftmax);
+      if (w < 0) {
+        ok = w == -1;
+        break;
+      }
       const int u = w / p.hkv;
       const int kt = p.kv_units[3 * u], e0 = p.kv_units[3 * u + 1], ne = p.kv_units[3 * u + 2];
       const int64_t jrow = (int64_t)kt * 128 + t;
@@ -396,7 +438,12 @@ __global__ void __launch_bounds__(448, 1)
     const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
     uint32_t it = 0, unit_iter = 0, hs = 0;  // hs: uses of the staging buffer (dQ halves, dK/dV pieces)
     bool ok = true;
-    for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
+    for (uint32_t wi = 0; ok; ++wi) {
+      const int w = take_work(wi, kErrTimeoutEpilogue);
+      if (w < 0) {
+        ok = w == -1;
+        break;
+      }
       const int u = w / p.hkv, g = w % p.hkv;
       const int kt = p.kv_units[3 * u], e0 = p.kv_units[3 * u + 1], ne = p.kv_units[3 * u + 2];
       int qt_next = p.entries[2 * e0];
@@ -491,10 +538,13 @@ __global__ void __launch_bounds__(448, 1)
       if (!ok) break;
       if (!mbar_wait_warp(dkdv_full, unit_iter & 1, guard, kErrTimeoutEpilogue)) break;
       tc_fence_after();
-      // This unit's dK (times the softmax scale left out of dS) and dV are added to the fp32
-      // accumulators, 64 features at a time: lane t holds row t, stages it into two 128-byte-
-      // swizzled boxes [128 rows][32 fp32], and thread 0 reduces both boxes with the TMA.  Rows past
-      // N hold zeros (their keys and values were loaded as zeros and all their pairs are masked).
+      // This unit's dK (times the softmax scale left out of dS) and dV leave TMEM 64 features at a
+      // time: lane t holds row t and stages it into the epilogue buffer, and thread 0 issues the TMA.
+      // A kv tile with other units adds its partial to the fp32 accumulators: two 128-byte-swizzled
+      // boxes [128 rows][32 fp32] reduced into them (rows past N hold zeros: their keys and values
+      // were loaded as zeros and all their pairs are masked).  A kv tile with no other unit (direct)
+      // is final: one 128-byte-swizzled box [128 rows][64 bf16] stored to the bf16 output.
+      const bool direct = p.kv_direct[(kt * 128 - (int)p.kv0) >> 7] != 0;
       uint8_t* epi = smem + C::OFF_EPI;
       constexpr int NCH = 2 * (D / 64);
 #pragma unroll 1
@@ -510,22 +560,37 @@ __global__ void __launch_bounds__(448, 1)
           tc_fence_before();
           mbar_arrive(dkdv_free);
         }
+        if (direct) {
 #pragma unroll
-        for (int c16 = 0; c16 < 8; ++c16) {
-          const uint32_t off = sw128_offset(t, c16);
-          st_shared_v4(smem_u32(epi + off), __float_as_uint(v0[4 * c16] * f), __float_as_uint(v0[4 * c16 + 1] * f),
-                       __float_as_uint(v0[4 * c16 + 2] * f), __float_as_uint(v0[4 * c16 + 3] * f));
-          st_shared_v4(smem_u32(epi + C::EPI_BYTES / 2 + off), __float_as_uint(v1[4 * c16] * f),
-                       __float_as_uint(v1[4 * c16 + 1] * f), __float_as_uint(v1[4 * c16 + 2] * f),
-                       __float_as_uint(v1[4 * c16 + 3] * f));
+          for (int c16 = 0; c16 < 8; ++c16) {
+            const float* v = c16 < 4 ? v0 + 8 * c16 : v1 + 8 * (c16 - 4);
+            st_shared_v4(smem_u32(epi + sw128_offset(t, c16)), pack_bf16x2(v[0] * f, v[1] * f),
+                         pack_bf16x2(v[2] * f, v[3] * f), pack_bf16x2(v[4] * f, v[5] * f),
+                         pack_bf16x2(v[6] * f, v[7] * f));
+          }
+        } else {
+#pragma unroll
+          for (int c16 = 0; c16 < 8; ++c16) {
+            const uint32_t off = sw128_offset(t, c16);
+            st_shared_v4(smem_u32(epi + off), __float_as_uint(v0[4 * c16] * f), __float_as_uint(v0[4 * c16 + 1] * f),
+                         __float_as_uint(v0[4 * c16 + 2] * f), __float_as_uint(v0[4 * c16 + 3] * f));
+            st_shared_v4(smem_u32(epi + C::EPI_BYTES / 2 + off), __float_as_uint(v1[4 * c16] * f),
+                         __float_as_uint(v1[4 * c16 + 1] * f), __float_as_uint(v1[4 * c16 + 2] * f),
+                         __float_as_uint(v1[4 * c16 + 3] * f));
+          }
         }
         fence_async_smem();
         mbar_arrive(stg_ready);
         if (!mbar_wait_warp(stg_ready, hs & 1, guard, kErrTimeoutEpilogue)) { ok = false; break; }
         if (t == 0) {
-          const int row0 = (which == 0 ? 0 : (int)p.n_pad_kv) + kt * 128 - (int)p.kv0;
-          tma_reduce_add_3d(&tmDKV, epi, 64 * cb, g, row0);
-          tma_reduce_add_3d(&tmDKV, epi + C::EPI_BYTES / 2, 64 * cb + 32, g, row0);
+          const int row = kt * 128 - (int)p.kv0;  // first row of the kv tile in the key/value-side buffers
+          if (direct) {
+            tma_store_3d(which == 0 ? &tmDK : &tmDV, epi, 64 * cb, g, row);
+          } else {
+            const int row0 = (which == 0 ? 0 : (int)p.n_pad_kv) + row;
+            tma_reduce_add_3d(&tmDKV, epi, 64 * cb, g, row0);
+            tma_reduce_add_3d(&tmDKV, epi + C::EPI_BYTES / 2, 64 * cb + 32, g, row0);
+          }
           bulk_commit_group();
           bulk_wait_group_read0();
           mbar_arrive(stg_free);
@@ -549,18 +614,20 @@ __global__ void __launch_bounds__(448, 1)
 
 template <int D>
 cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
-                       const CUtensorMap& tdq, const CUtensorMap& tdkv, const BwdParams& p, int grid,
-                       cudaStream_t stream) {
+                       const CUtensorMap& tdq, const CUtensorMap& tdkv, const CUtensorMap& tdk,
+                       const CUtensorMap& tdv, const BwdParams& p, int grid, cudaStream_t stream) {
   auto kern = sap_bwd_kernel<D>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, BwdCfg<D>::SMEM);
   if (e != cudaSuccess) return e;
-  kern<<<grid, BwdCfg<D>::THREADS, BwdCfg<D>::SMEM, stream>>>(tq, tk, tv, tdo, tdq, tdkv, p);
+  kern<<<grid, BwdCfg<D>::THREADS, BwdCfg<D>::SMEM, stream>>>(tq, tk, tv, tdo, tdq, tdkv, tdk, tdv, p);
   return cudaGetLastError();
 }
 
 template cudaError_t launch_bwd<64>(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
-                                    const CUtensorMap&, const CUtensorMap&, const BwdParams&, int, cudaStream_t);
+                                    const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
+                                    const BwdParams&, int, cudaStream_t);
 template cudaError_t launch_bwd<128>(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
-                                     const CUtensorMap&, const CUtensorMap&, const BwdParams&, int, cudaStream_t);
+                                     const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
+                                     const BwdParams&, int, cudaStream_t);
 
 }  // namespace sap

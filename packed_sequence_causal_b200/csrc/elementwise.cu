@@ -114,13 +114,14 @@ template <int D>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32)
     bwd_pre_kernel(const __nv_bfloat16* o, const __nv_bfloat16* dout, const float* lse, int64_t n, int64_t n_pad,
                    int64_t n_pad_kv, int32_t hq, int32_t hkv, float* dvec, float* lse2, float* dq_acc,
-                   float* dkv_acc) {
+                   float* dkv_acc, const int32_t* kv_direct, int* work_next) {
   constexpr int E = D / 32;
   const int64_t wid = (int64_t)blockIdx.x * kWarpsPerBlock + threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
+  if (wid == 0 && lane == 0) *work_next = 0;
   const int64_t i = wid / hq;
   const int h = (int)(wid % hq);
-  if (i < n_pad_kv && h < hkv) {
+  if (i < n_pad_kv && h < hkv && !kv_direct[i >> 7]) {  // tiles stored directly need no accumulator
     const size_t kv_row = ((size_t)i * hkv + h) * D + lane * E;
     Vec<E>::store_zero(dkv_acc + kv_row);
     Vec<E>::store_zero(dkv_acc + (size_t)n_pad_kv * hkv * D + kv_row);
@@ -143,24 +144,28 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
   }
 }
 
-// fp32 accumulators -> bf16, four values per thread: dQ, then dK, then dV.
-__global__ void bwd_post_kernel(const float* dq_acc, __nv_bfloat16* dq, int64_t q4, const float* dkv_acc,
-                                __nv_bfloat16* dk, __nv_bfloat16* dv, int64_t kv4, int64_t dv_offset) {
-  int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  const float* src;
-  __nv_bfloat16* dst;
-  if (t < q4) {
-    src = dq_acc + 4 * t, dst = dq + 4 * t;
-  } else if ((t -= q4) < kv4) {
-    src = dkv_acc + 4 * t, dst = dk + 4 * t;
-  } else if ((t -= kv4) < kv4) {
-    src = dkv_acc + dv_offset + 4 * t, dst = dv + 4 * t;
-  } else {
-    return;
-  }
+// fp32 accumulator -> bf16, four values per thread (dQ).
+__global__ void bwd_post_q_kernel(const float* dq_acc, __nv_bfloat16* dq, int64_t q4) {
+  const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= q4) return;
   float v[4];
-  Vec<4>::load(src, v);
-  Vec<4>::store_bf16(dst, v);
+  Vec<4>::load(dq_acc + 4 * t, v);
+  Vec<4>::store_bf16(dq + 4 * t, v);
+}
+
+// fp32 dK (blockIdx.z = 0) / dV (1) accumulators -> bf16 on the 128-row kv tiles listed in
+// acc_tiles (blockIdx.y = list position; the other tiles were stored directly by the backward
+// kernel), four values per thread; tile4 = 4-value groups per tile, values past kv_count skipped.
+__global__ void bwd_post_kv_kernel(const float* dkv_acc, __nv_bfloat16* dk, __nv_bfloat16* dv, int64_t dv_offset,
+                                   const int32_t* acc_tiles, int32_t tile4, int64_t kv_count) {
+  const int32_t t = blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= tile4) return;
+  const int64_t e = (int64_t)acc_tiles[blockIdx.y] * (4 * (int64_t)tile4) + 4 * (int64_t)t;
+  if (e >= kv_count) return;
+  const bool is_v = blockIdx.z != 0;
+  float v[4];
+  Vec<4>::load(dkv_acc + (is_v ? dv_offset : 0) + e, v);
+  Vec<4>::store_bf16((is_v ? dv : dk) + e, v);
 }
 
 // Received fp32 dK/dV partials added into rows of the fp32 accumulators, and those rows
@@ -204,12 +209,14 @@ cudaError_t launch_merge(const int32_t* merges, int64_t n_merges, int32_t hq, in
 template <int D>
 cudaError_t launch_bwd_pre(const __nv_bfloat16* o, const __nv_bfloat16* dout, const float* lse, int64_t n,
                            int64_t n_pad, int64_t n_pad_kv, int32_t hq, int32_t hkv, float* dvec, float* lse2,
-                           float* dq_acc, float* dkv_acc, cudaStream_t stream) {
+                           float* dq_acc, float* dkv_acc, const int32_t* kv_direct, int* work_next,
+                           cudaStream_t stream) {
   const int64_t warps = (n_pad > n_pad_kv ? n_pad : n_pad_kv) * hq;
   if (warps == 0) return cudaSuccess;
   const int64_t blocks = (warps + kWarpsPerBlock - 1) / kWarpsPerBlock;
   bwd_pre_kernel<D><<<(unsigned)blocks, kWarpsPerBlock * 32, 0, stream>>>(o, dout, lse, n, n_pad, n_pad_kv, hq, hkv,
-                                                                          dvec, lse2, dq_acc, dkv_acc);
+                                                                          dvec, lse2, dq_acc, dkv_acc, kv_direct,
+                                                                          work_next);
   return cudaGetLastError();
 }
 
@@ -225,12 +232,23 @@ cudaError_t launch_kv_add(float* dkv_acc, int64_t dv_offset, const float* dk_par
 
 cudaError_t launch_bwd_post(const float* dq_acc, __nv_bfloat16* dq, int64_t count_q, const float* dkv_acc,
                             __nv_bfloat16* dk, __nv_bfloat16* dv, int64_t count_kv, int64_t dv_offset,
-                            cudaStream_t stream) {
-  const int64_t total4 = count_q / 4 + 2 * (count_kv / 4);
-  if (total4 == 0) return cudaSuccess;
-  bwd_post_kernel<<<(unsigned)((total4 + 255) / 256), 256, 0, stream>>>(dq_acc, dq, count_q / 4, dkv_acc, dk, dv,
-                                                                        count_kv / 4, dv_offset);
-  return cudaGetLastError();
+                            const int32_t* acc_tiles, int64_t n_acc_tiles, int64_t row_elems, cudaStream_t stream) {
+  const int64_t q4 = count_q / 4;
+  if (q4 > 0) {
+    bwd_post_q_kernel<<<(unsigned)((q4 + 255) / 256), 256, 0, stream>>>(dq_acc, dq, q4);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  const int32_t tile4 = (int32_t)(128 * row_elems / 4);
+  // grid.y is limited to 65535 tiles per launch: larger lists go in several launches
+  for (int64_t first = 0; first < n_acc_tiles; first += 65535) {
+    const int64_t nt = n_acc_tiles - first < 65535 ? n_acc_tiles - first : 65535;
+    dim3 grid((unsigned)((tile4 + 255) / 256), (unsigned)nt, 2);
+    bwd_post_kv_kernel<<<grid, 256, 0, stream>>>(dkv_acc, dk, dv, dv_offset, acc_tiles + first, tile4, count_kv);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 template cudaError_t launch_merge<64>(const int32_t*, int64_t, int32_t, int64_t, int64_t, const float*,
@@ -238,8 +256,10 @@ template cudaError_t launch_merge<64>(const int32_t*, int64_t, int32_t, int64_t,
 template cudaError_t launch_merge<128>(const int32_t*, int64_t, int32_t, int64_t, int64_t, const float*,
                                        const float*, __nv_bfloat16*, float*, cudaStream_t);
 template cudaError_t launch_bwd_pre<64>(const __nv_bfloat16*, const __nv_bfloat16*, const float*, int64_t, int64_t,
-                                        int64_t, int32_t, int32_t, float*, float*, float*, float*, cudaStream_t);
+                                        int64_t, int32_t, int32_t, float*, float*, float*, float*, const int32_t*,
+                                        int*, cudaStream_t);
 template cudaError_t launch_bwd_pre<128>(const __nv_bfloat16*, const __nv_bfloat16*, const float*, int64_t, int64_t,
-                                         int64_t, int32_t, int32_t, float*, float*, float*, float*, cudaStream_t);
+                                         int64_t, int32_t, int32_t, float*, float*, float*, float*, const int32_t*,
+                                         int*, cudaStream_t);
 
 }  // namespace sap

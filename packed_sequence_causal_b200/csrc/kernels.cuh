@@ -43,6 +43,8 @@ struct BwdParams {
   const float* lse2;          // [hq][n_pad] LSE * log2(e) (+inf past the window)
   const float* dvec;          // [hq][n_pad] D_i = <dO_i, O_i> (0 past the window)
   float* dq_acc;              // [n_pad][hq][D] fp32 dQ accumulator (reduced into through the tdq map)
+  const int32_t* kv_direct;   // per 128-row kv tile of the window: 1 = store dK/dV as bf16 directly
+  int* work_next;             // work items handed out beyond the first gridDim.x (zero at launch)
   int* err;
   uint64_t wait_ns;           // pipeline wait limit of this launch
 };
@@ -53,10 +55,11 @@ template <int D>
 cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
                        int grid, cudaStream_t stream, bool two_cta = false);
 
+// tdkv: the fp32 dK/dV accumulators; tdk, tdv: the bf16 dK, dV outputs (tiles with kv_direct set).
 template <int D>
 cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
-                       const CUtensorMap& tdq, const CUtensorMap& tdkv, const BwdParams& p, int grid,
-                       cudaStream_t stream);
+                       const CUtensorMap& tdq, const CUtensorMap& tdkv, const CUtensorMap& tdk,
+                       const CUtensorMap& tdv, const BwdParams& p, int grid, cudaStream_t stream);
 
 // Merge into O rows [q0, q_end) (O and LSE hold the window's rows; LSE row stride q_end - q0).
 template <int D>
@@ -64,11 +67,14 @@ cudaError_t launch_merge(const int32_t* merges, int64_t n_merges, int32_t hq, in
                          const float* o_part, const float* lse_part, __nv_bfloat16* o, float* lse,
                          cudaStream_t stream);
 
-// n rows of O, dO and LSE (padded to n_pad); n_pad_kv rows of each dK/dV accumulator.
+// n rows of O, dO and LSE (padded to n_pad); n_pad_kv rows of each dK/dV accumulator, except the
+// 128-row tiles t with kv_direct[t] != 0 (their dK/dV are stored directly by the backward kernel);
+// work_next (the backward's work counter) set to zero.
 template <int D>
 cudaError_t launch_bwd_pre(const __nv_bfloat16* o, const __nv_bfloat16* dout, const float* lse, int64_t n,
                            int64_t n_pad, int64_t n_pad_kv, int32_t hq, int32_t hkv, float* dvec, float* lse2,
-                           float* dq_acc, float* dkv_acc, cudaStream_t stream);
+                           float* dq_acc, float* dkv_acc, const int32_t* kv_direct, int* work_next,
+                           cudaStream_t stream);
 
 // dkv_acc rows [row0, row0 + rows) += the fp32 partials dk_part, dv_part ([rows][hkv][D] each), then
 // those rows of dk and dv (same row numbering as the accumulator) are rewritten as bf16.
@@ -76,10 +82,11 @@ cudaError_t launch_kv_add(float* dkv_acc, int64_t dv_offset, const float* dk_par
                           int64_t row0, int64_t rows, int64_t row_elems, __nv_bfloat16* dk, __nv_bfloat16* dv,
                           cudaStream_t stream);
 
-// fp32 accumulators -> bf16: dq (count_q values), dk and dv (count_kv values each; the dV
-// accumulator starts dv_offset values after the dK one).
+// fp32 accumulators -> bf16: dq (count_q values); dk and dv (count_kv values each; the dV
+// accumulator starts dv_offset values after the dK one) on the n_acc_tiles 128-row tiles listed in
+// acc_tiles (row_elems values per row).
 cudaError_t launch_bwd_post(const float* dq_acc, __nv_bfloat16* dq, int64_t count_q, const float* dkv_acc,
                             __nv_bfloat16* dk, __nv_bfloat16* dv, int64_t count_kv, int64_t dv_offset,
-                            cudaStream_t stream);
+                            const int32_t* acc_tiles, int64_t n_acc_tiles, int64_t row_elems, cudaStream_t stream);
 
 }  // namespace sap

@@ -98,12 +98,14 @@ int check_cu(const int32_t* cu, int32_t num_docs, int64_t n) {
   return SAP_OK;
 }
 
-// Backward: items grouped by kv tile, q-tile descending within a kv tile, and each kv tile's
-// list cut into bands of kBwdBandTiles q tiles.  A unit is one (kv tile, band) piece; units are
-// ordered band-major from the top band down, heavy-first within a band.  The persistent CTAs take
-// units in this order, so at any time they all work on Q, dO and dQ rows of about one band (a few
-// tens of MB at 32 heads) and those rows stay in L2; the price is one fp32 dK/dV reduction per unit
-// instead of one bf16 store per kv tile.
+// Backward: items grouped by kv tile, q-tile descending within a kv tile.  A kv tile whose list
+// has at most kBwdBandTiles q tiles is one unit; a longer list is cut into bands of kBwdBandTiles
+// q tiles, one unit per (kv tile, band) piece.  Units are ordered band-major from the top band
+// down (a unit's band is that of its top q tile), heavy-first within a band.  The persistent CTAs
+// take units in this order, so at any time they all work on Q, dO and dQ rows of about one band
+// (a few tens of MB at 32 heads) and those rows stay in L2; the price is one fp32 dK/dV reduction
+// per unit of a cut list instead of one bf16 store per kv tile.  A kv tile with a single unit
+// stores its dK/dV directly (full plans; see kv_direct).
 void build_bwd_schedule(sap_plan_s* p) {
   const int64_t ntk = (p->n + p->block_n - 1) / p->block_n;
   std::vector<int64_t> cnt((size_t)ntk + 1, 0);
@@ -122,15 +124,28 @@ void build_bwd_schedule(sap_plan_s* p) {
     int32_t band, kv_tile, first, count;
   };
   std::vector<Unit> units;
+  std::vector<int32_t> units_of_tile((size_t)ntk, 0);
   for (int64_t t = 0; t < ntk; ++t) {
     int64_t e = cnt[t];
+    const bool whole = cnt[t + 1] - cnt[t] <= kBwdBandTiles;
     while (e < cnt[t + 1]) {
       const int32_t band = p->kv_entries[2 * e] / kBwdBandTiles;
-      int64_t f = e + 1;
+      int64_t f = whole ? cnt[t + 1] : e + 1;
       while (f < cnt[t + 1] && p->kv_entries[2 * f] / kBwdBandTiles == band) ++f;
       units.push_back(Unit{band, (int32_t)t, (int32_t)e, (int32_t)(f - e)});
+      units_of_tile[t]++;
       e = f;
     }
+  }
+  // direct bf16 stores: full plans, kv tiles of a single unit (tile index local to the window)
+  const int64_t kt0 = p->kv_begin / p->block_n;
+  const int64_t ntl = (p->kv_rows() + p->block_n - 1) / p->block_n;
+  p->kv_direct.assign((size_t)ntl, 0);
+  p->kv_acc_tiles.clear();
+  for (int64_t l = 0; l < ntl; ++l) {
+    const int64_t t = kt0 + l;
+    if (p->rank_chunk < 0 && t < ntk && units_of_tile[t] == 1) p->kv_direct[l] = 1;
+    else p->kv_acc_tiles.push_back((int32_t)l);
   }
   std::stable_sort(units.begin(), units.end(), [](const Unit& a, const Unit& b) {
     return a.band != b.band ? a.band > b.band : a.count > b.count;

@@ -8,7 +8,8 @@
 
 #include "sap.h"
 
-// Backward units cover at most this many q tiles of one kv tile's list (one "band").
+// Backward units: a kv tile's list of at most kBwdBandTiles q tiles is one unit; a longer list
+// is cut into the pieces that fall in one band of kBwdBandTiles q tiles each.
 constexpr int32_t kBwdBandTiles = 16;
 
 struct sap_plan_s {
@@ -44,6 +45,11 @@ struct sap_plan_s {
   // backward schedule
   std::vector<int32_t> kv_units;    // [V][3] (kv_tile, first_entry, n_entries): band-major, heavy-first in a band
   std::vector<int32_t> kv_entries;  // [items][2] (q_tile, tag)
+  // Per kv tile of the window (local index = (kv_tile * block_n - kv_begin) / block_n): 1 when the
+  // tile has a single backward unit in a full plan, which then stores the tile's dK/dV as bf16
+  // directly (in a rank plan, dK/dV rows may still receive other devices' partials, so every tile
+  // goes through the fp32 accumulators).  kv_acc_tiles lists the local indices of the other tiles.
+  std::vector<int32_t> kv_direct, kv_acc_tiles;
 
   // per-token document bounds (global token index): first token of the document, last token of the document
   std::vector<int32_t> tok_lo, tok_hi;
@@ -56,7 +62,7 @@ struct sap_plan_s {
   void* dev = nullptr;
   int dev_id = -1;
   size_t off_items = 0, off_units = 0, off_order = 0, off_merges = 0, off_kv_units = 0, off_kv_entries = 0,
-         off_tok_lo = 0, off_tok_hi = 0, dev_words = 0;
+         off_kv_direct = 0, off_kv_acc_tiles = 0, off_tok_lo = 0, off_tok_hi = 0, dev_words = 0;
 
   int64_t q_rows() const { return q_end - q_begin; }
   int64_t kv_rows() const { return q_end - kv_begin; }

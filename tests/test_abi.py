@@ -70,3 +70,17 @@ def test_forward_variant_argument_checked_without_gpu():
     assert lib.sap_set_forward_variant(2) == -1
     assert lib.sap_set_forward_variant(-1) == -1
     assert lib.sap_set_forward_variant(0) == 0
+
+
+def test_kv_add_refuses_a_full_plan_without_gpu():
+    """sap_attn_bwd_kv_add takes rank plans only: a full plan's backward stores the dK/dV of kv
+    tiles with a single unit directly and never writes their accumulator rows.  The refusal comes
+    before any device work (the pointers are never dereferenced)."""
+    lib = sap.load_library()
+    plan = sap.sap_plan([0, 300, 512], 512, 2)
+    assert sap.sap_plan_bwd_direct(plan).tolist() == [1, 1, 1, 1]
+    rank = sap.sap_plan_rank(plan, 1)
+    assert sap.sap_plan_bwd_direct(rank).tolist() == [0, 0, 0, 0]  # window: kv tiles 0..3 (token 256 is in doc 0)
+    fake = ctypes.c_void_p(1 << 20)
+    st = lib.sap_attn_bwd_kv_add(plan.handle, fake, 1 << 30, 2, 1, 64, fake, fake, 0, 128, fake, fake, None)
+    assert st == -1

@@ -178,7 +178,7 @@ def _check_rank_plans(cu, n, bounds, block=128):
         assert sap.sap_plan_chunk_stats(full)["pairs"][c] == pairs
         # schedules of the rank plan satisfy the same invariants as a full plan's
         from test_plan import _check_schedules
-        _check_schedules(r, mine, n, nchunks, block, block)
+        _check_schedules(r, mine, n, nchunks, block, block, is_rank=True)
     assert total_pairs == oracle.unmasked_pairs(cu)
 
 

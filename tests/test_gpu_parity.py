@@ -181,11 +181,15 @@ def test_long_document_elementwise():
 
 @pytest.mark.parametrize("d", [64, 128])
 def test_documents_across_backward_bands(d):
-    """Backward units cover one band of 16 q tiles (2048 tokens) of a kv tile's
-    list, so a kv tile of a long document sums dK/dV over several units.  Here
-    documents start and end inside bands and span up to four of them (N = 10240,
-    GQA 2, P = 5): every element against the full oracle."""
-    _fwd_bwd_full([5000, 1100, 3, 2900, 1237], 4, 2, d, 5, seed=22)
+    """A kv tile's list longer than 16 q tiles is cut into backward units of one band of 16 q
+    tiles (2048 tokens) each, whose fp32 dK/dV partials are summed in the workspace; a shorter
+    list is one unit that stores bf16 dK/dV directly.  Here documents start and end inside
+    bands and span up to four of them (N = 10240, GQA 2, P = 5), so both kinds of kv tile occur:
+    every element against the full oracle."""
+    lens = [5000, 1100, 3, 2900, 1237]
+    direct = sap.sap_plan_bwd_direct(sap.sap_plan(workloads.cu_seqlens_from_lengths(lens), sum(lens), 5))
+    assert 0 < direct.sum() < len(direct)
+    _fwd_bwd_full(lens, 4, 2, d, 5, seed=22)
 
 
 @pytest.mark.parametrize("d", [64, 128])

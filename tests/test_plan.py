@@ -20,7 +20,7 @@ def _plan_and_check(cu, n, nchunks, bm=128, bn=128):
     return plan, items
 
 
-def _check_schedules(plan, items, n, nchunks, bm, bn):
+def _check_schedules(plan, items, n, nchunks, bm, bn, is_rank=False):
     units, order, merges = sap.sap_plan_fwd_schedule(plan)
     # units tile the item list contiguously, one (q-tile, kv-chunk) each
     pos = 0
@@ -68,11 +68,13 @@ def _check_schedules(plan, items, n, nchunks, bm, bn):
         for a, b in zip(part[:-1], part[1:]):
             if units[a, 2] == units[b, 2]:
                 assert (chunk[a], a) < (chunk[b], b)
-    # backward: every item once; each unit is the part of one kv tile's q-descending list that
-    # falls in one band of 16 q tiles; units band-major (top band first), heavy-first within a
-    # band, ties by kv tile
+    # backward: every item once; a kv tile's q-descending list of at most 16 q tiles is one unit,
+    # a longer list is cut into the parts that fall in one band of 16 q tiles; units band-major
+    # (top band first, a unit's band is that of its top q tile), heavy-first within a band, ties by
+    # kv tile
     kv_units, entries = sap.sap_plan_bwd_schedule(plan)
     band = 16
+    list_len = np.bincount(items[:, 1], minlength=int(items[:, 1].max()) + 1 if len(items) else 0)
     seen = set()
     covered = np.zeros(len(entries), dtype=np.int64)
     prev = None
@@ -80,7 +82,10 @@ def _check_schedules(plan, items, n, nchunks, bm, bn):
         assert ne > 0
         grp = entries[e0:e0 + ne]
         assert np.all(np.diff(grp[:, 0]) < 0)
-        assert len(set((grp[:, 0] // band).tolist())) == 1
+        if list_len[kt] <= band:
+            assert ne == list_len[kt]
+        else:
+            assert len(set((grp[:, 0] // band).tolist())) == 1
         covered[e0:e0 + ne] += 1
         for qt, tag in grp:
             seen.add((int(qt), int(kt), int(tag)))
@@ -94,6 +99,16 @@ def _check_schedules(plan, items, n, nchunks, bm, bn):
     # units of one kv tile do not share a band (each band piece is maximal)
     pieces = {(int(kt), int(entries[e0, 0]) // band) for kt, e0, _ in kv_units}
     assert len(pieces) == len(kv_units)
+    # direct dK/dV stores: exactly the kv tiles of a single unit, in full plans only
+    direct = sap.sap_plan_bwd_direct(plan)
+    win = sap.sap_plan_window(plan)
+    n_units_of = np.bincount(kv_units[:, 0], minlength=len(list_len)) if len(kv_units) else np.zeros(0, int)
+    kt0 = win["kv_begin"] // bn
+    expect = np.zeros((win["q_end"] - win["kv_begin"] + bn - 1) // bn, dtype=np.int32)
+    if not is_rank:
+        for l in range(len(expect)):
+            expect[l] = int(kt0 + l < len(n_units_of) and n_units_of[kt0 + l] == 1)
+    np.testing.assert_array_equal(direct, expect)
     assert seen == {(int(a), int(b), int(t)) for a, b, _, _, t in items}
 
 
