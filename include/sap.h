@@ -340,7 +340,10 @@ int sap_set_wait_limit_ns(uint64_t limit_ns);
 
 /* Forward kernel variant for later sap_attn_fwd / sap_attn_fwd_part calls (process-wide; the
  * pages have no counterpart -- a B200 form of the same computation):
- *   0 (default)  one CTA per work item: two query heads of a kv group share each K/V tile load;
+ *   0 (default)  one CTA per work item of two query heads: two heads of a kv group share each
+ *                K/V tile load (even hq / hkv); with an odd group (MHA included) and an even hq,
+ *                two adjacent heads each load their own K/V tiles; an odd hq runs one head per
+ *                work item;
  *   1            two-CTA clusters (tcgen05 cta_group::2) where head_dim = 128 and hq / hkv is a
  *                multiple of 4: a pair of SMs runs every MMA of four query heads of a kv group as
  *                one M = 256 MMA, each SM loading half of every K and V tile; other shapes keep

@@ -361,6 +361,11 @@ __global__ void __launch_bounds__(192, 1)
 // p_half once the first half of P is in TMEM, so the first half of PV runs while
 // the second half of P is being computed.
 //
+// KVS = true (odd GQA group, MHA included): the two heads 2p and 2p+1 may belong to different kv
+// heads, so each tile gets its own K and V tiles: the rings hold K_A(t), K_B(t), ... and
+// V_A(t), V_B(t), ... in order of use, and each stage is released as soon as its one tile has read
+// it.  The kv tile sequence is the same for both tiles (one q tile, one unit).
+//
 // Threads: warp 0 TMA, warp 1 MMA, warps 2..5 softmax of tile 0 (head 2p),
 // warps 6..9 softmax of tile 1 (head 2p+1).
 // TMEM columns: S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [256+D,256+2D).
@@ -396,11 +401,13 @@ struct Fwd2Cfg {
   static constexpr uint32_t COL_O = 256;
 };
 
-template <int D, bool CTA2>
+template <int D, bool CTA2, bool KVS>
 __global__ void __launch_bounds__(320, 1)
     sap_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+  static_assert(!(CTA2 && KVS), "the two-CTA variant shares K/V between the heads of a kv group");
   using C = Fwd2Cfg<D, CTA2>;
+  constexpr int LPS = KVS ? 2 : 1;  // K (and V) tiles loaded per kv step: one per tile with KVS
   extern __shared__ __align__(1024) uint8_t smem[];
   if (smem_u32(smem) & 1023u) {
     if (threadIdx.x == 0) atomicOr(p.err, kErrSmemAlign);
@@ -481,10 +488,44 @@ __global__ void __launch_bounds__(320, 1)
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
-      uint32_t kv_iter = 0, unit_iter = 0;
+      uint32_t kq = 0, vq = 0, unit_iter = 0;  // K / V loads issued (ring positions)
       bool ok = true;
+      // K, V tile of kv tile kt for kv head g into the next ring stage
+      auto load_k = [&](int g, int kt) -> bool {
+        const int s = kq % C::NS;
+        if (!mbar_wait(k_empty + s, ((kq / C::NS) & 1) ^ 1, guard, kErrTimeoutLoad)) return false;
+        if (leader) mbar_arrive_expect_tx(k_full + s, (CTA2 ? 2 : 1) * C::KBYTES);
+        for (int b = 0; b < D / 64; ++b) {
+          if constexpr (CTA2)  // this CTA's 64 kv rows of the tile (the K map has 64-row boxes)
+            tma_load_3d_pair(smem + C::OFF_K + s * C::KBYTES + b * C::KSLAB, &tmK, at_leader(k_full + s), 64 * b,
+                             g, kt * 128 - (int)p.kv0 + 64 * (int)rank);
+          else
+            tma_load_3d(smem + C::OFF_K + s * C::KBYTES + b * C::BOX, &tmK, k_full + s, 64 * b, g,
+                        kt * 128 - (int)p.kv0);
+        }
+        ++kq;
+        return true;
+      };
+      auto load_v = [&](int g, int kt) -> bool {
+        const int s = vq % C::NS;
+        if (!mbar_wait(v_empty + s, ((vq / C::NS) & 1) ^ 1, guard, kErrTimeoutLoad)) return false;
+        // test hook: CTA 0 leaves its first V tile out (nothing is issued), so the MMA wait on it runs out
+        if (!(p.skip_v_load && blockIdx.x == 0 && vq == 0)) {
+          if (leader) mbar_arrive_expect_tx(v_full + s, (CTA2 ? 2 : 1) * C::VBYTES);
+          if constexpr (CTA2)  // this CTA's 64 of the D columns, all 128 kv rows
+            tma_load_3d_pair(smem + C::OFF_V + s * C::VBYTES, &tmV, at_leader(v_full + s), 64 * (int)rank, g,
+                             kt * 128 - (int)p.kv0);
+          else
+            for (int b = 0; b < D / 64; ++b)
+              tma_load_3d(smem + C::OFF_V + s * C::VBYTES + b * C::BOX, &tmV, v_full + s, 64 * b, g,
+                          kt * 128 - (int)p.kv0);
+        }
+        ++vq;
+        return true;
+      };
       for (int w = w0; w < total && ok; w += wstep) {
-        const int u = p.order[w / pairs], h0 = HEADS * (w % pairs) + 2 * (int)rank, g = h0 / p.group;
+        const int u = p.order[w / pairs], h0 = HEADS * (w % pairs) + 2 * (int)rank;
+        const int gA = h0 / p.group, gB = KVS ? (h0 + 1) / p.group : gA;  // kv heads of the two tiles
         const int qt = p.units[4 * u], ib = p.units[4 * u + 1], ic = p.units[4 * u + 2];
         if (!mbar_wait(q_empty, (unit_iter & 1) ^ 1, guard, kErrTimeoutLoad)) break;
         if (leader) mbar_arrive_expect_tx(q_full, (CTA2 ? 4 : 2) * C::QBYTES);
@@ -499,35 +540,15 @@ __global__ void __launch_bounds__(320, 1)
             tma_load_3d(smem + C::OFF_Q1 + b * C::BOX, &tmQ, q_full, 64 * b, h0 + 1, qt * 128 - (int)p.q0);
           }
         }
-        int kt_next = p.items[5 * ib + 1];
+        // Order of the loads = order of their use: K of step 0 (per tile with KVS), then per step t
+        // V(t) and K(t + 1), tile A before tile B.
+        int kt = p.items[5 * ib + 1];
+        if (!load_k(gA, kt) || (KVS && !load_k(gB, kt))) break;
         for (int t = 0; t < ic; ++t) {
-          const int kt = kt_next;
-          if (t + 1 < ic) kt_next = p.items[5 * (ib + t + 1) + 1];
-          const int s = kv_iter % C::NS;
-          const uint32_t ph = (kv_iter / C::NS) & 1;
-          if (!mbar_wait(k_empty + s, ph ^ 1, guard, kErrTimeoutLoad)) { ok = false; break; }
-          if (leader) mbar_arrive_expect_tx(k_full + s, (CTA2 ? 2 : 1) * C::KBYTES);
-          for (int b = 0; b < D / 64; ++b) {
-            if constexpr (CTA2)  // this CTA's 64 kv rows of the tile (the K map has 64-row boxes)
-              tma_load_3d_pair(smem + C::OFF_K + s * C::KBYTES + b * C::KSLAB, &tmK, at_leader(k_full + s), 64 * b,
-                               g, kt * 128 - (int)p.kv0 + 64 * (int)rank);
-            else
-              tma_load_3d(smem + C::OFF_K + s * C::KBYTES + b * C::BOX, &tmK, k_full + s, 64 * b, g,
-                          kt * 128 - (int)p.kv0);
-          }
-          if (!mbar_wait(v_empty + s, ph ^ 1, guard, kErrTimeoutLoad)) { ok = false; break; }
-          // test hook: CTA 0 leaves its first V tile out (nothing is issued), so the MMA wait on it runs out
-          if (!(p.skip_v_load && blockIdx.x == 0 && kv_iter == 0)) {
-            if (leader) mbar_arrive_expect_tx(v_full + s, (CTA2 ? 2 : 1) * C::VBYTES);
-            if constexpr (CTA2)  // this CTA's 64 of the D columns, all 128 kv rows
-              tma_load_3d_pair(smem + C::OFF_V + s * C::VBYTES, &tmV, at_leader(v_full + s), 64 * (int)rank, g,
-                               kt * 128 - (int)p.kv0);
-            else
-              for (int b = 0; b < D / 64; ++b)
-                tma_load_3d(smem + C::OFF_V + s * C::VBYTES + b * C::BOX, &tmV, v_full + s, 64 * b, g,
-                            kt * 128 - (int)p.kv0);
-          }
-          ++kv_iter;
+          const int kt_next = t + 1 < ic ? p.items[5 * (ib + t + 1) + 1] : -1;
+          if (!load_v(gA, kt) || (kt_next >= 0 && !load_k(gA, kt_next))) { ok = false; break; }
+          if (KVS && (!load_v(gB, kt) || (kt_next >= 0 && !load_k(gB, kt_next)))) { ok = false; break; }
+          kt = kt_next;
         }
         ++unit_iter;
       }
@@ -535,10 +556,10 @@ __global__ void __launch_bounds__(320, 1)
       // count both CTAs' copies; the other CTA is held at the final cluster barrier until then.
       if (leader) {
         if (unit_iter > 0) drain_wait(q_full, (unit_iter - 1) & 1, p.wait_ns);
-        for (uint32_t t = (kv_iter > (uint32_t)C::NS ? kv_iter - C::NS : 0); t < kv_iter; ++t) {
+        for (uint32_t t = (kq > (uint32_t)C::NS ? kq - C::NS : 0); t < kq; ++t)
           drain_wait(k_full + t % C::NS, (t / C::NS) & 1, p.wait_ns);
+        for (uint32_t t = (vq > (uint32_t)C::NS ? vq - C::NS : 0); t < vq; ++t)
           drain_wait(v_full + t % C::NS, (t / C::NS) & 1, p.wait_ns);
-        }
       }
     }
   } else if (warp == 1) {
@@ -550,7 +571,7 @@ __global__ void __launch_bounds__(320, 1)
       auto wait_p = [&](uint64_t* bar, uint32_t parity) { return mbar_wait(bar, parity, guard, kErrTimeoutMma); };
       const uint32_t sQ0 = smem_u32(smem + C::OFF_Q0), sQ1 = smem_u32(smem + C::OFF_Q1);
       const uint32_t sK = smem_u32(smem + C::OFF_K), sV = smem_u32(smem + C::OFF_V);
-      uint32_t kv_iter = 0, unit_iter = 0, tile_iter = 0;  // tile_iter counts kv tiles (per tile barrier phases)
+      uint32_t unit_iter = 0, tile_iter = 0;  // tile_iter counts kv tiles (per tile barrier phases)
       bool ok = true;
       auto issue_s = [&](int tile, uint32_t it) {  // S_tile = Q_tile K_it^T
         const uint32_t sQ = tile ? sQ1 : sQ0;
@@ -579,49 +600,61 @@ __global__ void __launch_bounds__(320, 1)
                             (first && kk == 0) ? 0u : 1u);
         }
       };
+      auto wait_k = [&](uint32_t i) { return mbar_wait(k_full + i % C::NS, (i / C::NS) & 1, guard, kErrTimeoutMma); };
+      auto wait_v = [&](uint32_t i) { return mbar_wait(v_full + i % C::NS, (i / C::NS) & 1, guard, kErrTimeoutMma); };
+      uint32_t kc = 0, vc = 0;  // K / V ring positions consumed (LPS per kv step)
       for (int w = w0; w < total && ok; w += wstep) {
         const int u = p.order[w / pairs];
         const int ic = p.units[4 * u + 2];
         if (!mbar_wait(q_full, unit_iter & 1, guard, kErrTimeoutMma)) break;
-        if (!mbar_wait(k_full + kv_iter % C::NS, (kv_iter / C::NS) & 1, guard, kErrTimeoutMma)) break;
+        if (!wait_k(kc)) break;
         tc_fence_after();
-        issue_s(0, kv_iter);
-        issue_s(1, kv_iter);
-        commit(k_empty + kv_iter % C::NS);
-        for (int j = 0; j < ic; ++j, ++tile_iter) {
-          const uint32_t it = kv_iter + j;
-          if (!mbar_wait(v_full + it % C::NS, (it / C::NS) & 1, guard, kErrTimeoutMma)) { ok = false; break; }
+        issue_s(0, kc);
+        if (KVS) {
+          commit(k_empty + kc % C::NS);
+          if (!wait_k(kc + 1)) break;
+          tc_fence_after();
+        }
+        issue_s(1, kc + LPS - 1);
+        commit(k_empty + (kc + LPS - 1) % C::NS);
+        kc += LPS;
+        for (int j = 0; j < ic; ++j, ++tile_iter, vc += LPS) {
+          if (!wait_v(vc)) { ok = false; break; }
           if (!wait_p(p_half + 0, tile_iter & 1)) { ok = false; break; }
           tc_fence_after();
-          issue_pv(0, it, j == 0, 0);
+          issue_pv(0, vc, j == 0, 0);
           if (!wait_p(p_full + 0, tile_iter & 1)) { ok = false; break; }
           tc_fence_after();
-          issue_pv(0, it, j == 0, 1);
+          issue_pv(0, vc, j == 0, 1);
+          if (KVS) commit(v_empty + vc % C::NS);
           const bool more = j + 1 < ic;
           if (more) {
-            if (!mbar_wait(k_full + (it + 1) % C::NS, ((it + 1) / C::NS) & 1, guard, kErrTimeoutMma)) {
-              ok = false;
-              break;
-            }
+            if (!wait_k(kc)) { ok = false; break; }
             tc_fence_after();
-            issue_s(0, it + 1);  // rewrites S0/P0 only after PV0 (issued above) has read P0
+            issue_s(0, kc);  // rewrites S0/P0 only after PV0 (issued above) has read P0
+            if (KVS) commit(k_empty + kc % C::NS);
           }
+          if (KVS && !wait_v(vc + 1)) { ok = false; break; }
           if (!wait_p(p_half + 1, tile_iter & 1)) { ok = false; break; }
           tc_fence_after();
-          issue_pv(1, it, j == 0, 0);
+          issue_pv(1, vc + LPS - 1, j == 0, 0);
           if (!wait_p(p_full + 1, tile_iter & 1)) { ok = false; break; }
           tc_fence_after();
-          issue_pv(1, it, j == 0, 1);
-          commit(v_empty + it % C::NS);
+          issue_pv(1, vc + LPS - 1, j == 0, 1);
+          commit(v_empty + (vc + LPS - 1) % C::NS);
           if (more) {
-            issue_s(1, it + 1);
-            commit(k_empty + (it + 1) % C::NS);
+            if (KVS) {
+              if (!wait_k(kc + 1)) { ok = false; break; }
+              tc_fence_after();
+            }
+            issue_s(1, kc + LPS - 1);
+            commit(k_empty + (kc + LPS - 1) % C::NS);
+            kc += LPS;
           }
         }
         if (!ok) break;
         commit(o_done);
         commit(q_empty);
-        kv_iter += ic;
         ++unit_iter;
       }
       // Wait for every MMA this thread issued before TMEM is released (CTA2: the leader's own barrier).
@@ -797,7 +830,7 @@ cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
   if constexpr (D == 128) {
     if (two_cta) {  // clusters of two CTAs, four heads of a kv group per cluster (group % 4 == 0)
       if (p.group % 4 != 0) return cudaErrorInvalidValue;
-      auto kern = sap_fwd_pair_kernel<128, true>;
+      auto kern = sap_fwd_pair_kernel<128, true, false>;
       using C2 = Fwd2Cfg<128, true>;
       cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C2::SMEM);
       if (e != cudaSuccess) return e;
@@ -828,10 +861,12 @@ cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
       return cudaGetLastError();
     }
   }
-  if (p.group % 2 == 0) {  // two heads of one kv group per CTA
+  // Two query heads per CTA: of one kv group (even group: shared K/V loads), or any two adjacent
+  // heads with their own K/V loads (odd group, even number of query heads).
+  if (p.group % 2 == 0 || p.hq % 2 == 0) {
     const int64_t work = (int64_t)p.n_units * (p.hq / 2);
     const int g2 = (int)(work < grid ? work : grid);
-    auto kern2 = sap_fwd_pair_kernel<D, false>;
+    auto kern2 = p.group % 2 == 0 ? sap_fwd_pair_kernel<D, false, false> : sap_fwd_pair_kernel<D, false, true>;
     cudaError_t e =
         cudaFuncSetAttribute(kern2, cudaFuncAttributeMaxDynamicSharedMemorySize, Fwd2Cfg<D, false>::SMEM);
     if (e != cudaSuccess) return e;

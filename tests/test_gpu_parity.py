@@ -214,6 +214,22 @@ def test_fused_merge_mode(d):
 
 
 @pytest.mark.parametrize("d", [64, 128])
-def test_odd_gqa_group_uses_one_tile_forward(d):
-    """Group size 3 (odd): the one-tile forward kernel with GQA, plus the backward."""
+def test_odd_gqa_group_pairs_heads_with_their_own_kv(d):
+    """Group size 3 (odd), 6 query heads: the two-tile forward pairs heads (0, 1), (2, 3), (4, 5),
+    and the pair (2, 3) straddles two kv heads, so every tile loads its own K/V tiles; plus the
+    backward."""
     _fwd_bwd_full([700, 200, 124], 6, 2, d, 2, seed=42)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_mha_pairs_with_long_kv_lists(d):
+    """MHA (4/4 heads): pairs of heads with their own K/V in the two-tile forward, over units of
+    up to 7 kv tiles (longer than the K/V rings), P = 3 (N = 2688, seven tiles per chunk)."""
+    _fwd_bwd_full([1500, 300, 700, 188], 4, 4, d, 3, seed=43)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_odd_head_count_uses_one_tile_forward(d):
+    """3 query heads on one kv head: an odd number of heads cannot be paired, so the one-tile
+    forward kernel runs; plus the backward."""
+    _fwd_bwd_full([700, 200, 124], 3, 1, d, 2, seed=44)

@@ -4,7 +4,8 @@ sap_test_arm_wait_timeout makes the next forward launch use a 20 ms wait limit a
 first V tile of its first CTA out (no copy is issued, so nothing is in flight).  In that CTA the
 MMA issuer waits for the tile, and the producer waits for the tile's ring stage to be released;
 whichever wait started first runs out at the limit and records its timeout bit in the device
-error word (the two-tile kernel: the MMA issuer's; the one-tile kernel: the producer's), the
+error word (the two-tile kernel, with shared or per-tile K/V: the MMA issuer's; the one-tile
+kernel: the producer's), the
 other roles see the CTA's abort flag, and the CTA winds down (its issued MMAs and copies are
 waited for before tensor memory and shared memory are released); every other CTA finishes
 normally.  The call returns, the host reads SAP_ERR_DEVICE with the bit through
@@ -27,6 +28,7 @@ K_ERR_TIMEOUT_ANY = 0xF  # load, MMA, softmax, epilogue waits
 
 
 @pytest.mark.parametrize("hq,hkv,first", [(4, 2, K_ERR_TIMEOUT_MMA),    # two-tile forward kernel
+                                           (4, 4, K_ERR_TIMEOUT_MMA),    # two-tile, K/V per tile (MHA)
                                            (3, 3, K_ERR_TIMEOUT_LOAD)])  # one-tile forward kernel
 def test_wait_that_runs_out_is_reported_and_the_context_survives(hq, hkv, first):
     b = workloads.custom_batch([700, 324], hq, hkv, 128, seed=61, with_do=False)
