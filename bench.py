@@ -409,8 +409,12 @@ def main():
 
         def e2e_run(steps, start_ev=None, end_ev=None):
             ev = lambda: torch.cuda.Event()  # noqa: E731
-            in_ready, in_free = [ev() for _ in range(steps)], [ev() for _ in range(steps)]
-            out_ready, out_free = [ev() for _ in range(steps)], [ev() for _ in range(steps)]
+            # per step: Q, K, V in (the forward's inputs) and dO in (the backward's) as two events;
+            # O, LSE out as soon as the merge is done and dQ, dK, dV after the backward
+            qkv_ready, do_ready = [ev() for _ in range(steps)], [ev() for _ in range(steps)]
+            in_free = [ev() for _ in range(steps)]
+            fwd_done, bwd_done, out_free = [ev() for _ in range(steps)], [ev() for _ in range(steps)], \
+                [ev() for _ in range(steps)]
             if start_ev is not None:
                 start_ev.record(stream)
             s_in.wait_stream(stream)
@@ -420,27 +424,34 @@ def main():
                 with torch.cuda.stream(s_in):
                     if i >= 2:
                         s_in.wait_event(in_free[i - 2])   # step i-2 no longer reads this set
-                    for dst, src in zip(d_in[i % 2], h_in):
+                    for j, (dst, src) in enumerate(zip(d_in[i % 2], h_in)):
                         dst.copy_(src, non_blocking=True)
-                    in_ready[i].record(s_in)
+                        if j == 2:
+                            qkv_ready[i].record(s_in)
+                    do_ready[i].record(s_in)
 
             copy_in(0)
             for i in range(steps):
                 if i + 1 < steps:
                     copy_in(i + 1)
-                stream.wait_event(in_ready[i])
+                stream.wait_event(qkv_ready[i])
                 if i >= 2:
                     stream.wait_event(out_free[i - 2])    # step i-2's results have left this set
                 qi, ki, vi, doi = d_in[i % 2]
                 oi, lsei, dqi, dki, dvi = d_out[i % 2]
                 sap.sap_attn_fwd(plan, qi, ki, vi, scale, oi, lsei, ws_f, stream)
                 sap.sap_merge(plan, ws_f, hq, d, oi, lsei, stream)
+                fwd_done[i].record(stream)
+                stream.wait_event(do_ready[i])
                 sap.sap_attn_bwd(plan, qi, ki, vi, oi, lsei, doi, scale, dqi, dki, dvi, ws_b, stream)
                 in_free[i].record(stream)
-                out_ready[i].record(stream)
+                bwd_done[i].record(stream)
                 with torch.cuda.stream(s_out):
-                    s_out.wait_event(out_ready[i])
-                    for dst, src in zip(h_out, d_out[i % 2]):
+                    s_out.wait_event(fwd_done[i])
+                    for dst, src in zip(h_out[:2], d_out[i % 2][:2]):  # O, LSE
+                        dst.copy_(src, non_blocking=True)
+                    s_out.wait_event(bwd_done[i])
+                    for dst, src in zip(h_out[2:], d_out[i % 2][2:]):  # dQ, dK, dV
                         dst.copy_(src, non_blocking=True)
                     out_free[i].record(s_out)
             stream.wait_stream(s_in)
@@ -466,7 +477,8 @@ def main():
                "ms_per_step": round(e2e_ms / args.steps, 3),
                "tokens_per_s": round(world * n * args.steps / (e2e_ms / 1e3), 1),
                "overlap": "double-buffered: step s+1's inputs in and step s's results out on two copy "
-                          "streams while step s+1 computes"}
+                          "streams while step s+1 computes; dO in while the forward runs, O and LSE out "
+                          "while the backward runs"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
