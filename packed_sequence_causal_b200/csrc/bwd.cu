@@ -137,15 +137,15 @@ __global__ void __launch_bounds__(448, 1)
     }
     mbar_init(s_full, 1);
     mbar_init(dp_full, 1);
-    mbar_init(p_ready, 256);
-    mbar_init(ds_ready, 256);
+    mbar_init(p_ready, 8);    // one arrival per softmax warp
+    mbar_init(ds_ready, 8);
     mbar_init(ds_free, 1);
     mbar_init(dq_full, 1);
-    mbar_init(dq_free, 128);
+    mbar_init(dq_free, 4);    // one arrival per drain warp
     mbar_init(dkdv_full, 1);
-    mbar_init(dkdv_free, 128);
+    mbar_init(dkdv_free, 4);
     mbar_init(mma_drain, 1);
-    mbar_init(stg_ready, 128);
+    mbar_init(stg_ready, 4);
     mbar_init(stg_free, 1);
     mbar_init(dv_done, 1);
     for (int s = 0; s < C::NW; ++s) {
@@ -393,7 +393,7 @@ __global__ void __launch_bounds__(448, 1)
             tmem_st32_u(R1, pk);  // P^T over this half's first 32 S^T columns (already read)
           }
           tc_fence_before();
-          mbar_arrive(p_ready);
+          mbar_arrive_warp(p_ready);
           if (!mbar_wait_warp(dp_full, it & 1, guard, kErrTimeoutSoftmax)) { ok = false; break; }
           // d = 64: dS^T has its own buffer, free once dK/dQ of the previous iteration completed.
           // d = 128: dS^T goes over dO_j once dV_j (its last reader) has completed.
@@ -427,7 +427,7 @@ __global__ void __launch_bounds__(448, 1)
           }
           fence_async_smem();
           tc_fence_before();
-          mbar_arrive(ds_ready);
+          mbar_arrive_warp(ds_ready);
         }
       }
     }
@@ -469,12 +469,12 @@ __global__ void __launch_bounds__(448, 1)
               for (int e2 = 0; e2 < 32; ++e2) stg[(32 * c + e2) * 128 + t] = v[e2] * p.scale;
             }
             fence_async_smem();
-            mbar_arrive(stg_ready);
+            mbar_arrive_warp(stg_ready);
             float v2[32], v3[32];
             tmem_ld32(lane_base + C::COL_DQ + 64, v2);
             tmem_ld32(lane_base + C::COL_DQ + 96, v3);
             tc_fence_before();
-            mbar_arrive(dq_free);  // all of dQ^T is in registers or staged: R2 may take the next dP^T
+            mbar_arrive_warp(dq_free);  // all of dQ^T is in registers or staged: R2 may take the next dP^T
             if (!mbar_wait_warp(stg_ready, hs & 1, guard, kErrTimeoutEpilogue)) { ok = false; break; }
             if (t == 0) {
               tma_reduce_add_3d(&tmDQ, stg, 0, h, qt * 128 - (int)p.q0);
@@ -490,7 +490,7 @@ __global__ void __launch_bounds__(448, 1)
               stg[(32 + e2) * 128 + t] = v3[e2] * p.scale;
             }
             fence_async_smem();
-            mbar_arrive(stg_ready);
+            mbar_arrive_warp(stg_ready);
             if (!mbar_wait_warp(stg_ready, hs & 1, guard, kErrTimeoutEpilogue)) { ok = false; break; }
             if (t == 0) {
               tma_reduce_add_3d(&tmDQ, stg, 0, h, qt * 128 - (int)p.q0 + 64);
@@ -510,7 +510,7 @@ __global__ void __launch_bounds__(448, 1)
             tmem_ld32(lane_base + C::COL_DQ, v0);
             tmem_ld32(lane_base + C::COL_DQ + 32, v1);
             tc_fence_before();
-            mbar_arrive(dq_free);  // all of dQ is in registers: the next dQ may overwrite its columns
+            mbar_arrive_warp(dq_free);  // all of dQ is in registers: the next dQ may overwrite its columns
 #pragma unroll
             for (int c16 = 0; c16 < 8; ++c16) {
               const uint32_t off = sw128_offset(t, c16);
@@ -522,7 +522,7 @@ __global__ void __launch_bounds__(448, 1)
                            __float_as_uint(v1[4 * c16 + 3] * p.scale));
             }
             fence_async_smem();
-            mbar_arrive(stg_ready);
+            mbar_arrive_warp(stg_ready);
             if (!mbar_wait_warp(stg_ready, hs & 1, guard, kErrTimeoutEpilogue)) { ok = false; break; }
             if (t == 0) {
               tma_reduce_add_3d(&tmDQ, epi, 0, h, qt * 128 - (int)p.q0);
@@ -558,7 +558,7 @@ __global__ void __launch_bounds__(448, 1)
         tmem_ld32(lane_base + col + 32, v1);
         if (m == NCH - 1) {  // all of dK/dV has been read: the next unit may accumulate over it
           tc_fence_before();
-          mbar_arrive(dkdv_free);
+          mbar_arrive_warp(dkdv_free);
         }
         if (direct) {
 #pragma unroll
@@ -580,7 +580,7 @@ __global__ void __launch_bounds__(448, 1)
           }
         }
         fence_async_smem();
-        mbar_arrive(stg_ready);
+        mbar_arrive_warp(stg_ready);
         if (!mbar_wait_warp(stg_ready, hs & 1, guard, kErrTimeoutEpilogue)) { ok = false; break; }
         if (t == 0) {
           const int row = kt * 128 - (int)p.kv0;  // first row of the kv tile in the key/value-side buffers
