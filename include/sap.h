@@ -196,7 +196,8 @@ int sap_plan_bwd_direct(sap_plan_t plan, const int32_t** flags, int64_t* n_tiles
  * explainer page, FAQ on equivalence with one device -- allows): the forward schedule gets one unit per
  * q-tile spanning all of its kv chunks, so sap_attn_fwd carries the online
  * softmax across chunk boundaries and writes O and LSE directly -- no fp32
- * partials, no forward workspace, and sap_merge has nothing to do.  The result
+ * partials (the forward workspace holds only the work counter and may be NULL),
+ * and sap_merge has nothing to do.  The result
  * is the merged result of the chunked path (the merge is exact), computed in
  * one pass; the per-(q-chunk, kv-chunk) partials are not produced.  enable = 0
  * restores the chunked schedule.  Host-side only: the device copy of the plan
@@ -215,9 +216,10 @@ void sap_plan_destroy(sap_plan_t plan);
 /* Workspace bytes (plumbing; no counterpart in the pages) for a call with these head counts
  * (which = SAP_WS_FWD for
  * sap_attn_fwd + sap_merge, SAP_WS_BWD for sap_attn_bwd).  The forward
- * workspace holds the fp32 partial outputs and LSEs of the partial slots; the
- * backward one holds the fp32 dQ, dK and dV accumulators and the per-row D and
- * LSE*log2(e). */
+ * workspace holds the fp32 partial outputs and LSEs of the partial slots and
+ * the forward's work counter; the backward one holds the fp32 dQ, dK and dV
+ * accumulators, the per-row D and LSE*log2(e) and the backward's work counter.
+ * Calls that share a workspace must not run at the same time. */
 int sap_workspace_size(sap_plan_t plan, int32_t hq, int32_t hkv, int32_t head_dim, int32_t which, size_t* bytes);
 
 /* Forward (HSAP page, abstract: the partial attention computation of each part of the sequence
@@ -227,7 +229,10 @@ int sap_workspace_size(sap_plan_t plan, int32_t hq, int32_t hkv, int32_t head_di
  * with online softmax in fp32 on tcgen05 tensor cores.  A q-tile with one unit
  * writes bf16 O and fp32 LSE directly; the others leave fp32 partials (O, LSE)
  * in the workspace for sap_merge.  Rows of a partial that see no key have
- * LSE = -inf and O = 0. */
+ * LSE = -inf and O = 0.  The workspace may be NULL when the plan has no partial slots; with a
+ * workspace of the full size the persistent CTAs take their work items in schedule order from a
+ * counter in it (reset on `stream` first), without one in a fixed round-robin order (same
+ * results: every work item is computed the same way whichever CTA takes it). */
 int sap_attn_fwd(sap_plan_t plan, const void* q, const void* k, const void* v, int32_t hq, int32_t hkv,
                  int32_t head_dim, float softmax_scale, void* o, float* lse, void* workspace, size_t ws_bytes,
                  void* stream);

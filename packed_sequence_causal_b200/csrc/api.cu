@@ -133,14 +133,15 @@ int check_kernel_plan(const sap_plan_s* p) {
 
 // Workspace layouts (256-byte aligned pieces).
 struct FwdWs {
-  size_t o_part = 0, lse_part = 0, total = 0;
+  size_t o_part = 0, lse_part = 0, work_next = 0, total = 0;
 };
 FwdWs fwd_ws(const sap_plan_s* p, int32_t hq, int32_t hd) {
   FwdWs w;
   const size_t slots = (size_t)p->n_slots;
-  w.o_part = 0;
-  w.lse_part = round_up((int64_t)(slots * hq * 128 * hd * 4), 256);
-  w.total = w.lse_part + round_up((int64_t)(slots * hq * 128 * 4), 256);
+  w.o_part = 0;                                                           // [slots][hq][128][hd] fp32
+  w.lse_part = round_up((int64_t)(slots * hq * 128 * hd * 4), 256);      // [slots][hq][128] fp32
+  w.work_next = w.lse_part + round_up((int64_t)(slots * hq * 128 * 4), 256);  // int: work counter
+  w.total = w.work_next + 256;
   return w;
 }
 struct BwdWs {
@@ -535,6 +536,13 @@ int sap_attn_fwd_part(sap_plan_t p, int32_t part, int32_t max_ctas, const void* 
   const int64_t work = (int64_t)fp.n_units * hq;
   if (work == 0) return SAP_OK;
   if (work > INT32_MAX) return SAP_ERR_INVALID_ARG;
+  // A full workspace carries the work counter of the dynamic work order (reset on this stream
+  // before the launch); without one (allowed when there are no partial slots) the order is static.
+  if (workspace && ws_bytes >= ws.total && aligned16(workspace)) {
+    fp.work_next = reinterpret_cast<int*>(wsb + ws.work_next);
+    const cudaError_t ez = cudaMemsetAsync(fp.work_next, 0, sizeof(int), static_cast<cudaStream_t>(stream));
+    if (ez != cudaSuccess) return cuda_fail(ez);
+  }
   const int sms = max_ctas > 0 && max_ctas < di->sms ? max_ctas : di->sms;
   const int grid = (int)(work < sms ? work : sms);
   cudaError_t e = head_dim == 64

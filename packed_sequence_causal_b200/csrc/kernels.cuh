@@ -27,6 +27,8 @@ struct FwdParams {
   int* err;               // device error word
   uint64_t wait_ns;       // pipeline wait limit of this launch
   int32_t skip_v_load;    // test hook: CTA 0 leaves its first V load out, so a wait runs out
+  int* work_next;         // two-tile kernel, one-CTA form: work items handed out beyond the first
+                          // gridDim.x (zero at launch); nullptr: static round-robin order
 };
 
 struct BwdParams {

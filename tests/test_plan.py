@@ -223,7 +223,7 @@ def test_fused_merge_schedule(name):
         pos += c
     assert pos == len(items)
     assert sorted(order.tolist()) == list(range(len(units)))
-    assert sap.sap_workspace_size(plan, w.hq, w.hkv, w.d, sap.SAP_WS_FWD) == 0
+    assert sap.sap_workspace_size(plan, w.hq, w.hkv, w.d, sap.SAP_WS_FWD) == 256  # the work counter only
     sap.sap_plan_set_fused_merge(plan, False)
     for a, b in zip(chunked, sap.sap_plan_fwd_schedule(plan)):
         np.testing.assert_array_equal(a, b)
