@@ -244,17 +244,21 @@ __global__ void __launch_bounds__(448, 1)
       const uint32_t sDS = smem_u32(smem + C::OFF_DS);
       const uint32_t sST = smem_u32(smem + C::OFF_ST);
       const uint32_t R1 = tmem + C::COL_R1, R2 = tmem + C::COL_R2;
+      // Shared-memory descriptors, computed once per operand base; per k-slice only an offset is
+      // added (K-major: 16-byte leading offset; MN-major: one box apart).
+      const uint64_t dK_k = sdesc_sw128(sK, 16, 1024), dV_k = sdesc_sw128(sV, 16, 1024);
+      const uint64_t dK_mn = sdesc_sw128(sK, C::BOX, 1024);
       uint32_t unit_iter = 0, it = 0;  // it: global iteration counter (all barriers below count per iteration)
       bool ok = true;
       auto stage_q = [&](uint32_t i) { return sST + (i % C::NSQ) * C::STAGE; };
       auto issue_s = [&](uint32_t i) -> bool {  // S^T_i = K Q_i^T -> R1
         if (!mbar_wait(q_full + i % C::NSQ, (i / C::NSQ) & 1, guard, kErrTimeoutMma)) return false;
         tc_fence_after();
-        const uint32_t sQ = stage_q(i);
+        const uint64_t dQ_k = sdesc_sw128(stage_q(i), 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t ko = (kk / 4) * C::BOX + (kk % 4) * 32;
-          mma_bf16(R1, sdesc_sw128(sK + ko, 16, 1024), sdesc_sw128(sQ + ko, 16, 1024), id_sq, kk > 0);
+          mma_bf16(R1, sdesc_off(dK_k, ko), sdesc_off(dQ_k, ko), id_sq, kk > 0);
         }
         tc_commit(s_full);
         return true;
@@ -272,6 +276,8 @@ __global__ void __launch_bounds__(448, 1)
         if (!issue_s(it)) break;
         for (int j = 0; j < n_it; ++j, ++it) {
           const uint32_t sQ = stage_q(it), sDO = sQ + C::TILE;
+          const uint64_t dQ_mn = sdesc_sw128(sQ, C::BOX, 1024);
+          const uint64_t dDO_k = sdesc_sw128(sDO, 16, 1024), dDO_mn = sdesc_sw128(sDO, C::BOX, 1024);
           // dV += P^T_j dO_j first (P^T in TMEM, packed bf16 over the S^T columns of each half):
           // P^T_j is usually ready well before the previous dQ has been drained.
           if (!mbar_wait(p_ready, it & 1, guard, kErrTimeoutMma)) { ok = false; break; }
@@ -283,7 +289,7 @@ __global__ void __launch_bounds__(448, 1)
 #pragma unroll
           for (int kk = 0; kk < 128 / 16; ++kk)
             mma_bf16_tmem_a(tmem + C::COL_DV, R1 + (kk / 4) * 64 + (kk % 4) * 8,
-                            sdesc_sw128(sDO + kk * 2048, C::BOX, 1024), id_kv, (j > 0 || kk > 0) ? 1u : 0u);
+                            sdesc_off(dDO_mn, kk * 2048), id_kv, (j > 0 || kk > 0) ? 1u : 0u);
           if (C::DQ_T) tc_commit(dv_done);
           // dP^T_j -> R2 once the previous dQ (D = 128: same columns) has been drained
           if (C::DQ_T && it > 0 && !mbar_wait(dq_free, (it - 1) & 1, guard, kErrTimeoutMma)) { ok = false; break; }
@@ -291,10 +297,11 @@ __global__ void __launch_bounds__(448, 1)
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t ko = (kk / 4) * C::BOX + (kk % 4) * 32;
-            mma_bf16(R2, sdesc_sw128(sV + ko, 16, 1024), sdesc_sw128(sDO + ko, 16, 1024), id_sq, kk > 0);
+            mma_bf16(R2, sdesc_off(dV_k, ko), sdesc_off(dDO_k, ko), id_sq, kk > 0);
           }
           tc_commit(dp_full);
           const uint32_t sDSj = C::DQ_T ? sDO : sDS;  // d = 128: dS^T_j over dO_j
+          const uint64_t dDS_k = sdesc_sw128(sDSj, 16, 1024), dDS_mn = sdesc_sw128(sDSj, C::BOX, 1024);
           // S^T_{j+1}: R1 is rewritten only after dV_j (issued above) has read P^T_j
           if (j + 1 < n_it && !issue_s(it + 1)) { ok = false; break; }
           // dQ_j and dK += dS^T_j Q_j
@@ -306,15 +313,15 @@ __global__ void __launch_bounds__(448, 1)
           for (int kk = 0; kk < 128 / 16; ++kk) {
             // D=128: dQ^T[d][q] = sum_kv K[kv][d] dS^T[kv][q]  (A = K, B = dS^T, both MN-major)
             // D=64 : dQ[q][d]   = sum_kv dS^T[kv][q] K[kv][d]  (A = dS^T, B = K, both MN-major)
-            const uint64_t kd = sdesc_sw128(sK + kk * 2048, C::BOX, 1024);
-            const uint64_t sd = sdesc_sw128(sDSj + kk * 2048, C::BOX, 1024);
+            const uint64_t kd = sdesc_off(dK_mn, kk * 2048);
+            const uint64_t sd = sdesc_off(dDS_mn, kk * 2048);
             mma_bf16(tmem + C::COL_DQ, C::DQ_T ? kd : sd, C::DQ_T ? sd : kd, id_dq, kk > 0);
           }
           tc_commit(dq_full);
 #pragma unroll
           for (int kk = 0; kk < 128 / 16; ++kk) {
-            const uint64_t a = sdesc_sw128(sDSj + (kk / 4) * C::BOX + (kk % 4) * 32, 16, 1024);
-            mma_bf16(tmem + C::COL_DK, a, sdesc_sw128(sQ + kk * 2048, C::BOX, 1024), id_kv,
+            const uint64_t a = sdesc_off(dDS_k, (kk / 4) * C::BOX + (kk % 4) * 32);
+            mma_bf16(tmem + C::COL_DK, a, sdesc_off(dQ_mn, kk * 2048), id_kv,
                      (j > 0 || kk > 0) ? 1u : 0u);
           }
           if (!C::DQ_T) tc_commit(ds_free);

@@ -375,6 +375,10 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
   d |= (uint64_t)2 << 61;
   return d;
 }
+// The descriptor of an address `bytes` (a multiple of 16) past the one `d` describes: the start
+// address field holds bits 4..17 of a shared-memory address, which cannot carry out for
+// addresses below 256 KB.
+__device__ __forceinline__ uint64_t sdesc_off(uint64_t d, uint32_t bytes) { return d + (uint64_t)(bytes >> 4); }
 
 // Instruction descriptor, kind::f16 with bf16 A/B and fp32 D:
 // D format F32 = 1 at [4,6), A format BF16 = 1 at [7,10), B format BF16 = 1 at
