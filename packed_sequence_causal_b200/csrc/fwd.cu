@@ -632,13 +632,16 @@ __global__ void __launch_bounds__(320, 1)
       const uint32_t sK = smem_u32(smem + C::OFF_K), sV = smem_u32(smem + C::OFF_V);
       uint32_t unit_iter = 0, tile_iter = 0;  // tile_iter counts kv tiles (per tile barrier phases)
       bool ok = true;
+      // descriptors computed once per operand base; per k-slice only an offset is added
+      const uint64_t dQ0 = sdesc_sw128(sQ0, 16, 1024), dQ1 = sdesc_sw128(sQ1, 16, 1024);
+      const uint64_t dK = sdesc_sw128(sK, 16, 1024), dV = sdesc_sw128(sV, C::BOX, 1024);
       auto issue_s = [&](int tile, uint32_t it) {  // S_tile = Q_tile K_it^T
-        const uint32_t sQ = tile ? sQ1 : sQ0;
-        const int s = it % C::NS;
+        const uint64_t dQ = tile ? dQ1 : dQ0;
+        const uint64_t dKs = sdesc_off(dK, (it % C::NS) * C::KBYTES);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t a = sdesc_sw128(sQ + (kk / 4) * C::BOX + (kk % 4) * 32, 16, 1024);
-          const uint64_t bd = sdesc_sw128(sK + s * C::KBYTES + (kk / 4) * C::KSLAB + (kk % 4) * 32, 16, 1024);
+          const uint64_t a = sdesc_off(dQ, (kk / 4) * C::BOX + (kk % 4) * 32);
+          const uint64_t bd = sdesc_off(dKs, (kk / 4) * C::KSLAB + (kk % 4) * 32);
           if constexpr (CTA2)
             mma_bf16_pair(tmem + 128 * tile, a, bd, idesc_qk, kk > 0);
           else
@@ -647,10 +650,10 @@ __global__ void __launch_bounds__(320, 1)
         commit(s_full + tile);
       };
       auto issue_pv = [&](int tile, uint32_t it, bool first, int part) {  // O_tile += P_tile V_it (half), P from TMEM
-        const int s = it % C::NS;
+        const uint64_t dVs = sdesc_off(dV, (it % C::NS) * C::VBYTES);
 #pragma unroll
         for (int kk = 4 * part; kk < 4 * part + 4; ++kk) {
-          const uint64_t bd = sdesc_sw128(sV + s * C::VBYTES + kk * 2048, C::BOX, 1024);
+          const uint64_t bd = sdesc_off(dVs, kk * 2048);
           if constexpr (CTA2)
             mma_bf16_tmem_a_pair(tmem + C::COL_O + D * tile, tmem + 128 * tile + kk * 8, bd, idesc_pv,
                                  (first && kk == 0) ? 0u : 1u);
