@@ -164,6 +164,9 @@ __global__ void __launch_bounds__(192, 1)
       constexpr uint32_t idesc_pv = idesc_bf16(128, D, false, true);
       const uint32_t sQ = smem_u32(smem + C::OFF_Q), sK = smem_u32(smem + C::OFF_K),
                      sV = smem_u32(smem + C::OFF_V), sP = smem_u32(smem + C::OFF_P);
+      // descriptors computed once per operand base; per k-slice and stage only an offset is added
+      const uint64_t dQ = sdesc_sw128(sQ, 16, 1024), dK = sdesc_sw128(sK, 16, 1024);
+      const uint64_t dV = sdesc_sw128(sV, C::BOX, 1024), dP = sdesc_sw128(sP, 16, 1024);
       uint32_t kv_iter = 0, unit_iter = 0, s_iter = 0, pv_iter = 0;
       bool ok = true;
       for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
@@ -180,8 +183,8 @@ __global__ void __launch_bounds__(192, 1)
           const bool first = (it == kv_iter);  // first tile of this unit
 #pragma unroll
           for (int kk = 0; kk < 128 / 16; ++kk) {
-            const uint64_t a = sdesc_sw128(sP + (kk / 4) * C::BOX + (kk % 4) * 32, 16, 1024);
-            const uint64_t b = sdesc_sw128(sV + s * C::KVBYTES + kk * 2048, C::BOX, 1024);
+            const uint64_t a = sdesc_off(dP, (kk / 4) * C::BOX + (kk % 4) * 32);
+            const uint64_t b = sdesc_off(dV, s * C::KVBYTES + kk * 2048);
             mma_bf16(tmem + C::COL_O, a, b, idesc_pv, (first && kk == 0) ? 0u : 1u);
           }
           tc_commit(pv_done);
@@ -199,8 +202,8 @@ __global__ void __launch_bounds__(192, 1)
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t a = sdesc_sw128(sQ + (kk / 4) * C::BOX + (kk % 4) * 32, 16, 1024);
-            const uint64_t bd = sdesc_sw128(sK + s * C::KVBYTES + (kk / 4) * C::BOX + (kk % 4) * 32, 16, 1024);
+            const uint64_t a = sdesc_off(dQ, (kk / 4) * C::BOX + (kk % 4) * 32);
+            const uint64_t bd = sdesc_off(dK, s * C::KVBYTES + (kk / 4) * C::BOX + (kk % 4) * 32);
             mma_bf16(tmem + 128 * b, a, bd, idesc_qk, kk > 0 ? 1u : 0u);
           }
           tc_commit(s_full + b);
