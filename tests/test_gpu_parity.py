@@ -163,6 +163,35 @@ def test_repeat_calls_are_identical_forward():
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
 
 
+@pytest.mark.parametrize("d", [64, 128])
+def test_forward_work_order_does_not_change_the_result(d):
+    """The forward takes its work items dynamically (a counter in the workspace) or round-robin (no
+    workspace, allowed without partial slots), on any grid: every item is computed the same way
+    whichever CTA takes it, so all orders give the same bytes.  Fused-merge plan (no slots), GQA 2
+    (shared K/V) and MHA (K/V per tile)."""
+    for hq, hkv in ((4, 2), (4, 4)):
+        b = workloads.custom_batch([900, 40, 1300, 257, 575], hq, hkv, d, seed=45, with_do=False)
+        n = b.q.shape[0]  # 3072: three chunks of eight tiles
+        q, k, v = (t.to("cuda").contiguous() for t in (b.q, b.k, b.v))
+        plan = sap.sap_plan(b.cu_seqlens, n, 3)
+        sap.sap_plan_set_fused_merge(plan, True)
+        assert sap.sap_plan_stats(plan)["n_partial_slots"] == 0
+        ws = sap.alloc_workspace(plan, hq, hkv, d, sap.SAP_WS_FWD, "cuda")
+        scale = 1.0 / math.sqrt(d)
+        outs = []
+        for workspace, max_ctas in ((ws, 0), (ws, 3), (None, 0), (None, 5)):
+            o = torch.empty_like(q)
+            lse = torch.empty((hq, n), dtype=torch.float32, device="cuda")
+            sap.sap_attn_fwd_part(plan, 0, q, k, v, scale, o, lse, workspace, max_ctas=max_ctas)
+            outs.append((o, lse))
+        assert sap.sap_device_status() == 0
+        for o, lse in outs[1:]:
+            assert torch.equal(o, outs[0][0]) and torch.equal(lse, outs[0][1])
+        ro, rl = oracle.attn_fwd(b.q, b.k, b.v, b.cu_seqlens, scale)
+        assert_close(outs[0][0], ro, "O (work orders)")
+        assert_lse(outs[0][1], rl, "LSE (work orders)")
+
+
 def test_workspace_too_small_is_rejected():
     b = workloads.custom_batch([700, 324], 2, 1, 64, seed=13, with_do=True)
     r = Run(b, 8)
