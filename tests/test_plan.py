@@ -227,3 +227,26 @@ def test_fused_merge_schedule(name):
     sap.sap_plan_set_fused_merge(plan, False)
     for a, b in zip(chunked, sap.sap_plan_fwd_schedule(plan)):
         np.testing.assert_array_equal(a, b)
+
+
+@pytest.mark.parametrize("tiles", [15, 16, 17, 33])
+def test_backward_units_at_the_band_limit(tiles):
+    """One document of `tiles` q tiles: kv tile 0's list has `tiles` entries.  Up to 16 entries it
+    is one backward unit (and, in a full plan, its dK/dV are stored directly); 17 or more are cut at
+    the 16-tile band boundaries into one unit per band, accumulated in fp32."""
+    n = 128 * tiles
+    plan = sap.sap_plan([0, n], n, 1)
+    kv_units, entries = sap.sap_plan_bwd_schedule(plan)
+    direct = sap.sap_plan_bwd_direct(plan)
+    for kt in range(tiles):
+        mine = kv_units[kv_units[:, 0] == kt]
+        list_len = tiles - kt  # q tiles kt .. tiles - 1
+        assert mine[:, 2].sum() == list_len
+        if list_len <= 16:
+            assert len(mine) == 1 and direct[kt] == 1
+        else:
+            bands = {int(q) // 16 for q in range(kt, tiles)}
+            assert len(mine) == len(bands) and direct[kt] == 0
+            for _, e0, ne in mine:
+                qs = entries[e0:e0 + ne, 0]
+                assert len({int(q) // 16 for q in qs}) == 1
