@@ -74,9 +74,9 @@ struct BwdCfg {
   static constexpr int OFF_EPI = (D == 128) ? OFF_DS : OFF_ST + NSQ * STAGE;
   static constexpr int OFF_BAR = (D == 128) ? OFF_ST + NSQ * STAGE : OFF_EPI + EPI_BYTES;
   static constexpr int NW = 4;  // work-index ring depth
-  static constexpr int NBAR = 2 + 2 * NSQ + 13 + 2 * NW;
+  static constexpr int NBAR = 2 + 2 * NSQ + 11 + 2 * NW;
   // The dynamic shared window starts 1024-byte aligned (checked at run time),
-  // so no alignment slack is reserved: the D = 128 layout needs 231,672 bytes.
+  // so no alignment slack is reserved: the D = 128 layout needs 231,656 bytes.
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 4 * NW;
   static_assert(SMEM <= 232448, "shared memory per block");
   static_assert(OFF_EPI % 1024 == 0 && OFF_ST % 1024 == 0 && STAGE % 1024 == 0, "128-byte swizzle alignment");
@@ -110,16 +110,14 @@ __global__ void __launch_bounds__(448, 1)
   uint64_t* dp_full = s_full + 1;
   uint64_t* p_ready = dp_full + 1;
   uint64_t* ds_ready = p_ready + 1;
-  uint64_t* ds_free = ds_ready + 1;
-  uint64_t* dq_full = ds_free + 1;
+  uint64_t* dq_full = ds_ready + 1;
   uint64_t* dq_free = dq_full + 1;
   uint64_t* dkdv_full = dq_free + 1;
   uint64_t* dkdv_free = dkdv_full + 1;
   uint64_t* mma_drain = dkdv_free + 1;
   uint64_t* stg_ready = mma_drain + 1;  // the staging buffer holds a dQ or dK/dV piece
   uint64_t* stg_free = stg_ready + 1;   // its reduction has read the staging buffer
-  uint64_t* dv_done = stg_free + 1;     // dV has read dO: dS^T may go over it (d = 128)
-  uint64_t* sched_full = dv_done + 1;   // [NW] the producer wrote the next work index
+  uint64_t* sched_full = stg_free + 1;  // [NW] the producer wrote the next work index
   uint64_t* sched_empty = sched_full + C::NW;  // [NW] every other role has read it
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBAR);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -139,7 +137,6 @@ __global__ void __launch_bounds__(448, 1)
     mbar_init(dp_full, 1);
     mbar_init(p_ready, 8);    // one arrival per softmax warp
     mbar_init(ds_ready, 8);
-    mbar_init(ds_free, 1);
     mbar_init(dq_full, 1);
     mbar_init(dq_free, 4);    // one arrival per drain warp
     mbar_init(dkdv_full, 1);
@@ -147,7 +144,6 @@ __global__ void __launch_bounds__(448, 1)
     mbar_init(mma_drain, 1);
     mbar_init(stg_ready, 4);
     mbar_init(stg_free, 1);
-    mbar_init(dv_done, 1);
     for (int s = 0; s < C::NW; ++s) {
       mbar_init(sched_full + s, 1);
       mbar_init(sched_empty + s, 1 + 8 + 4);  // the MMA thread, the 8 softmax and 4 drain warps
@@ -290,7 +286,6 @@ __global__ void __launch_bounds__(448, 1)
           for (int kk = 0; kk < 128 / 16; ++kk)
             mma_bf16_tmem_a(tmem + C::COL_DV, R1 + (kk / 4) * 64 + (kk % 4) * 8,
                             sdesc_off(dDO_mn, kk * 2048), id_kv, (j > 0 || kk > 0) ? 1u : 0u);
-          if (C::DQ_T) tc_commit(dv_done);
           // dP^T_j -> R2 once the previous dQ (D = 128: same columns) has been drained
           if (C::DQ_T && it > 0 && !mbar_wait(dq_free, (it - 1) & 1, guard, kErrTimeoutMma)) { ok = false; break; }
           tc_fence_after();
@@ -324,7 +319,6 @@ __global__ void __launch_bounds__(448, 1)
             mma_bf16(tmem + C::COL_DK, a, sdesc_off(dQ_mn, kk * 2048), id_kv,
                      (j > 0 || kk > 0) ? 1u : 0u);
           }
-          if (!C::DQ_T) tc_commit(ds_free);
           tc_commit(q_empty + it % C::NSQ);
         }
         if (!ok) break;
@@ -366,7 +360,8 @@ __global__ void __launch_bounds__(448, 1)
               reinterpret_cast<const float*>(smem + C::OFF_ST + (it % C::NSQ) * C::STAGE + 2 * C::TILE) + 64 * half;
           const float* dvec = lse2 + 128;
           const int c_lo = j_lo - qt * 128 - 64 * half, c_hi = j_hi - qt * 128 - 64 * half;
-          if (!mbar_wait_warp(q_full + it % C::NSQ, (it / C::NSQ) & 1, guard, kErrTimeoutSoftmax)) { ok = false; break; }
+          // S^T_j is issued only after the MMA thread has seen the stage's loads (Q, dO, LSE, D) land,
+          // so its completion also means that this stage's vectors are in shared memory.
           if (!mbar_wait_warp(s_full, it & 1, guard, kErrTimeoutSoftmax)) { ok = false; break; }
           tc_fence_after();
           float pr[64];
@@ -401,14 +396,10 @@ __global__ void __launch_bounds__(448, 1)
           }
           tc_fence_before();
           mbar_arrive_warp(p_ready);
+          // dp_full tracks every MMA the MMA thread issued before dP^T_j: dV_j (d = 128: dS^T_j goes
+          // over dO_j, which dV_j was the last to read) and the previous iteration's dQ and dK (d = 64:
+          // the dS^T buffer they read is free again).
           if (!mbar_wait_warp(dp_full, it & 1, guard, kErrTimeoutSoftmax)) { ok = false; break; }
-          // d = 64: dS^T has its own buffer, free once dK/dQ of the previous iteration completed.
-          // d = 128: dS^T goes over dO_j once dV_j (its last reader) has completed.
-          if (C::DQ_T ? !mbar_wait_warp(dv_done, it & 1, guard, kErrTimeoutSoftmax)
-                      : (it > 0 && !mbar_wait_warp(ds_free, (it - 1) & 1, guard, kErrTimeoutSoftmax))) {
-            ok = false;
-            break;
-          }
           tc_fence_after();
           uint8_t* sDSt = (C::DQ_T ? smem + C::OFF_ST + (it % C::NSQ) * C::STAGE + C::TILE : smem + C::OFF_DS) +
                           half * C::BOX;
