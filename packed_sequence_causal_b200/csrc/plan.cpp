@@ -226,6 +226,13 @@ int sap_plan_build(const int32_t* cu, int32_t num_docs, int64_t n, int32_t num_c
   // items, canonical order
   p->items.clear();
   const int64_t ntq = (n + block_m - 1) / block_m;
+  const int64_t ntk = (n + block_n - 1) / block_n;
+  std::vector<int32_t> kv_chunk((size_t)ntk);  // chunk of each kv tile's first key (bounds ascend)
+  for (int64_t kt = 0; kt < ntk; ++kt) kv_chunk[(size_t)kt] = chunk_of(kt * block_n);
+  int64_t n_items = 0;
+  for (int64_t qt = 0; qt < ntq; ++qt)
+    n_items += (std::min<int64_t>(qt * block_m + block_m, n) - 1) / block_n - p->tok_lo[qt * block_m] / block_n + 1;
+  p->items.reserve((size_t)n_items);
   for (int64_t qt = 0; qt < ntq; ++qt) {
     const int64_t i0 = qt * block_m;
     const int64_t ilast = std::min<int64_t>(i0 + block_m, n) - 1;  // last real row
@@ -243,7 +250,7 @@ int sap_plan_build(const int32_t* cu, int32_t num_docs, int64_t n, int32_t num_c
         tag = SAP_TAG_CAUSAL;
       else
         tag = SAP_TAG_MASKED;
-      p->items.push_back(sap_item_t{(int32_t)qt, (int32_t)kt, qc, chunk_of(j0), tag});
+      p->items.push_back(sap_item_t{(int32_t)qt, (int32_t)kt, qc, kv_chunk[(size_t)kt], tag});
     }
   }
   count_chunk_pairs(p);
