@@ -58,7 +58,7 @@ struct Vec<4> {
 // Merge of the partials of one q-tile: warp = (merge entry, head, row).  O and LSE hold the
 // query rows [q0, q_end) (global token indices); LSE's row stride is q_end - q0.
 template <int D>
-__global__ void __launch_bounds__(kWarpsPerBlock * 32)
+__global__ void __launch_bounds__(kWarpsPerBlock * 32, 8)  // 8 resident blocks: more rows' loads in flight
     merge_kernel(const int32_t* merges, int64_t n_merges, int32_t hq, int64_t q0, int64_t q_end,
                  const float* o_part, const float* lse_part, __nv_bfloat16* o, float* lse) {
   constexpr int E = D / 32;
@@ -81,12 +81,12 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
     float sum = 0.f;
     for (int b = 0; b < ns; ++b) sum += __expf(lse_part[((size_t)(s0 + b) * hq + h) * 128 + r] - mx);
     lse_all = mx + __logf(sum);
-    // up to four partials' rows are loaded before they are accumulated (in order), so that
+    // up to two partials' rows are loaded before they are accumulated (in order), so that
     // several 4*D-byte loads per warp are in flight
-    for (int b0 = 0; b0 < ns; b0 += 4) {
-      float v[4][E], wgt[4];
+    for (int b0 = 0; b0 < ns; b0 += 2) {
+      float v[2][E], wgt[2];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < 2; ++u) {
         if (b0 + u < ns) {
           const size_t row = ((size_t)(s0 + b0 + u) * hq + h) * 128 + r;
           wgt[u] = lse_part[row];
@@ -94,7 +94,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
         }
       }
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < 2; ++u) {
         if (b0 + u < ns) {
           const float w = __expf(wgt[u] - lse_all);
 #pragma unroll
