@@ -81,8 +81,8 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, 8)  // 8 resident blocks:
     float sum = 0.f;
     for (int b = 0; b < ns; ++b) sum += __expf(lse_part[((size_t)(s0 + b) * hq + h) * 128 + r] - mx);
     lse_all = mx + __logf(sum);
-    // up to two partials' rows are loaded before they are accumulated (in order), so that
-    // several 4*D-byte loads per warp are in flight
+    // two partials' rows are loaded before they are accumulated (in order): with eight resident
+    // blocks (32 registers) more warps' loads are in flight than four rows per round would allow
     for (int b0 = 0; b0 < ns; b0 += 2) {
       float v[2][E], wgt[2];
 #pragma unroll
