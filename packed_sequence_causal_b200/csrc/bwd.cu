@@ -54,6 +54,12 @@
 
 namespace sap {
 
+// Each unit walks its q tiles starting at entry kt mod (entries), wrapping around, so that the units
+// of one band that run at the same time reduce into different q tiles' dQ rows rather than all into
+// the band's first tile.
+__device__ __forceinline__ int entry_rotation(int kt, int ne) { return ne > 1 ? kt % ne : 0; }
+__device__ __forceinline__ int rotated(int e, int rot, int ne) { return e + rot >= ne ? e + rot - ne : e + rot; }
+
 template <int D>
 struct BwdCfg {
   static constexpr int NSQ = (D == 64) ? 3 : 2;  // Q/dO ring depth
@@ -202,11 +208,12 @@ __global__ void __launch_bounds__(448, 1)
           tma_load_3d(smem + C::OFF_V + b * C::BOX, &tmV, kv_full, 64 * b, g, kt * 128 - (int)p.kv0);
         }
         // entries are walked q-tile outer, head inner; the next q tile is fetched one entry ahead
-        int qt_next = p.entries[2 * e0];
+        const int rot = entry_rotation(kt, ne);
+        int qt_next = p.entries[2 * (e0 + rot)];
         for (int e = 0; e < ne && ok; ++e) {
           const int qt = qt_next;
           const int qrow = qt * 128 - (int)p.q0;  // first row of the q tile in the query-side buffers
-          if (e + 1 < ne) qt_next = p.entries[2 * (e0 + e + 1)];
+          if (e + 1 < ne) qt_next = p.entries[2 * (e0 + rotated(e + 1, rot, ne))];
           for (int hh = 0; hh < G; ++hh) {
             const int h = g * G + hh;
             const int s = q_iter % C::NSQ;
@@ -274,8 +281,20 @@ __global__ void __launch_bounds__(448, 1)
           const uint32_t sQ = stage_q(it), sDO = sQ + C::TILE;
           const uint64_t dQ_mn = sdesc_sw128(sQ, C::BOX, 1024);
           const uint64_t dDO_k = sdesc_sw128(sDO, 16, 1024), dDO_mn = sdesc_sw128(sDO, C::BOX, 1024);
-          // dV += P^T_j dO_j first (P^T in TMEM, packed bf16 over the S^T columns of each half):
-          // P^T_j is usually ready well before the previous dQ has been drained.
+          auto issue_dp = [&]() {  // dP^T_j = V dO_j^T -> R2
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t ko = (kk / 4) * C::BOX + (kk % 4) * 32;
+              mma_bf16(R2, sdesc_off(dV_k, ko), sdesc_off(dDO_k, ko), id_sq, kk > 0);
+            }
+            tc_commit(dp_full);
+          };
+          // D = 64: dP^T_j needs only V and dO_j, and R2 is free once the softmax has read dP^T_{j-1}
+          // (before it signalled dS^T_{j-1}), so it is issued before P^T_j is waited for and is ready
+          // when the softmax has written P^T_j.
+          if (!C::DQ_T) issue_dp();
+          // dV += P^T_j dO_j (P^T in TMEM, packed bf16 over the S^T columns of each half); at D = 128
+          // it goes first because P^T_j is usually ready well before the previous dQ has been drained.
           if (!mbar_wait(p_ready, it & 1, guard, kErrTimeoutMma)) { ok = false; break; }
           if (j == 0 && unit_iter > 0 && !mbar_wait(dkdv_free, (unit_iter - 1) & 1, guard, kErrTimeoutMma)) {
             ok = false;
@@ -286,15 +305,12 @@ __global__ void __launch_bounds__(448, 1)
           for (int kk = 0; kk < 128 / 16; ++kk)
             mma_bf16_tmem_a(tmem + C::COL_DV, R1 + (kk / 4) * 64 + (kk % 4) * 8,
                             sdesc_off(dDO_mn, kk * 2048), id_kv, (j > 0 || kk > 0) ? 1u : 0u);
-          // dP^T_j -> R2 once the previous dQ (D = 128: same columns) has been drained
-          if (C::DQ_T && it > 0 && !mbar_wait(dq_free, (it - 1) & 1, guard, kErrTimeoutMma)) { ok = false; break; }
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t ko = (kk / 4) * C::BOX + (kk % 4) * 32;
-            mma_bf16(R2, sdesc_off(dV_k, ko), sdesc_off(dDO_k, ko), id_sq, kk > 0);
+          // D = 128: dP^T_j -> R2 once the previous dQ^T (same columns) has been drained
+          if (C::DQ_T) {
+            if (it > 0 && !mbar_wait(dq_free, (it - 1) & 1, guard, kErrTimeoutMma)) { ok = false; break; }
+            tc_fence_after();
+            issue_dp();
           }
-          tc_commit(dp_full);
           const uint32_t sDSj = C::DQ_T ? sDO : sDS;  // d = 128: dS^T_j over dO_j
           const uint64_t dDS_k = sdesc_sw128(sDSj, 16, 1024), dDS_mn = sdesc_sw128(sDSj, C::BOX, 1024);
           // S^T_{j+1}: R1 is rewritten only after dV_j (issued above) has read P^T_j
@@ -351,10 +367,14 @@ __global__ void __launch_bounds__(448, 1)
       const bool real_row = jrow < p.q_end;
       const int j_lo = real_row ? (int)jrow : 1;  // queries i with j <= i <= last token of the document
       const int j_hi = real_row ? p.tok_hi[jrow] : 0;
-      int qt_next = p.entries[2 * e0], tag_next = p.entries[2 * e0 + 1];
+      const int rot = entry_rotation(kt, ne);
+      int qt_next = p.entries[2 * (e0 + rot)], tag_next = p.entries[2 * (e0 + rot) + 1];
       for (int e = 0; e < ne && ok; ++e) {
         const int qt = qt_next, tag = tag_next;
-        if (e + 1 < ne) qt_next = p.entries[2 * (e0 + e + 1)], tag_next = p.entries[2 * (e0 + e + 1) + 1];
+        if (e + 1 < ne) {
+          const int en = e0 + rotated(e + 1, rot, ne);
+          qt_next = p.entries[2 * en], tag_next = p.entries[2 * en + 1];
+        }
         for (int hh = 0; hh < G; ++hh, ++it) {
           const float* lse2 =
               reinterpret_cast<const float*>(smem + C::OFF_ST + (it % C::NSQ) * C::STAGE + 2 * C::TILE) + 64 * half;
@@ -444,10 +464,11 @@ __global__ void __launch_bounds__(448, 1)
       }
       const int u = w / p.hkv, g = w % p.hkv;
       const int kt = p.kv_units[3 * u], e0 = p.kv_units[3 * u + 1], ne = p.kv_units[3 * u + 2];
-      int qt_next = p.entries[2 * e0];
+      const int rot = entry_rotation(kt, ne);
+      int qt_next = p.entries[2 * (e0 + rot)];
       for (int e = 0; e < ne && ok; ++e) {
         const int qt = qt_next;
-        if (e + 1 < ne) qt_next = p.entries[2 * (e0 + e + 1)];
+        if (e + 1 < ne) qt_next = p.entries[2 * (e0 + rotated(e + 1, rot, ne))];
         for (int hh = 0; hh < G; ++hh, ++it) {
           const int h = g * G + hh;
           if (!mbar_wait_warp(dq_full, it & 1, guard, kErrTimeoutEpilogue)) { ok = false; break; }
