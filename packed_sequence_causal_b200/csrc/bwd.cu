@@ -21,10 +21,12 @@
 //                  S^T_{j+1}          (R1 is free once dV_j has read P^T_j)
 //                  dQ_j               (D=128: dQ^T = K^T dS^T -> R2; D=64: dQ = dS K -> DQ)
 //                  dK    += dS^T_j Q_j  (A = dS^T from shared memory) -> dK
-//                dV goes first because P^T_j is ready long before the previous dQ^T
-//                has left R2 (which dP^T_j needs at D = 128), and dQ before dK so
-//                that its drain overlaps dK; the Q/dO ring slot is released once dK_j
-//                and dQ_j have read it.
+//                At D = 128 dV goes first because P^T_j is ready long before the
+//                previous dQ^T has left R2 (which dP^T_j needs); at D = 64 dP^T_j has
+//                R2 to itself and is issued first, right after dK_{j-1}, so that it is
+//                ready when the softmax has written P^T_j.  dQ goes before dK so that
+//                its drain overlaps dK; the Q/dO ring slot is released once dK_j and
+//                dQ_j have read it.
 //   warps 2..9   two warpgroups, one per half of the 128 q columns; thread t
 //                owns kv row j = kt*128 + t.  P^T = exp2(S^T c - LSE2_i) on the
 //                pairs of its document with i >= j (all pairs for FULL tiles),
