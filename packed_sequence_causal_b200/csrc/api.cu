@@ -87,12 +87,12 @@ int make_map(CUtensorMap* map, const void* base, int64_t rows, int32_t heads, in
   return SAP_OK;
 }
 
-// fp32 dQ accumulator [rows][heads][hd] -> 3-D map whose box is one q tile of one head
-// (128 rows x hd features, no swizzle): the target of the backward's bulk reductions.
+// fp32 dQ accumulator [rows][heads][hd] -> 3-D map whose box is a quarter q tile of one head
+// (32 rows x hd features, no swizzle): the target of the backward's bulk reductions.
 int make_map_f32_tile(CUtensorMap* map, void* base, int64_t rows, int32_t heads, int32_t hd) {
   cuuint64_t dims[3] = {(cuuint64_t)hd, (cuuint64_t)heads, (cuuint64_t)rows};
   cuuint64_t strides[2] = {(cuuint64_t)hd * 4, (cuuint64_t)heads * hd * 4};
-  cuuint32_t box[3] = {(cuuint32_t)hd, 1, 64};  // half a q tile: the kernel stages and reduces 64 rows at a time
+  cuuint32_t box[3] = {(cuuint32_t)hd, 1, 32};  // a quarter of a q tile: the kernel stages and reduces 32 rows at a time
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,

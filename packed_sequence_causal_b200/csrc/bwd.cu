@@ -37,12 +37,13 @@
 //                operand by dQ): for D = 128 over the ring slot's dO tile once dV_j
 //                has read it, for D = 64 into a buffer of its own.
 //   warps 10..13 drain dQ from TMEM into the fp32 accumulator by TMA bulk
-//                reductions (D = 128: dQ^T staged 64 q rows at a time in a dedicated
-//                buffer; D = 64: dQ staged as two 128-byte-swizzled boxes of 32
-//                features), and at the end of a work item add its dK and dV into
-//                fp32 accumulators the same way (the conversion to bf16 is a
-//                separate elementwise kernel), or, when the kv tile has no other
-//                unit, store them as bf16 directly.
+//                reductions (D = 128: dQ^T staged 32 q rows at a time; D = 64: dQ
+//                staged as two 128-byte-swizzled boxes of 32 features) through a
+//                staging buffer of two 16 KB slots, so that two reductions are in
+//                flight, and at the end of a work item add its dK and dV into fp32
+//                accumulators the same way (the conversion to bf16 is a separate
+//                elementwise kernel), or, when the kv tile has no other unit, store
+//                them as bf16 directly.
 //
 // TMEM columns: dK [0,D), dV [D,2D), R1 = S^T/P^T [2D, 2D+128),
 // R2 = dP^T [2D+128, 2D+256); dQ shares R2 for D = 128 (dP^T is consumed
@@ -72,19 +73,23 @@ struct BwdCfg {
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + TILE;
   // d = 64: dS^T (128 x 128 bf16).  d = 128: dS^T lives in the dO half of its iteration's stage and this
-  // region stages half a dQ tile (64 q rows x 128 fp32) for the TMA reduction.
+  // region is the staging buffer (two slots of 32 q rows x 128 fp32 of dQ, or of one dK/dV box).
   static constexpr int OFF_DS = OFF_V + TILE;
   static constexpr int OFF_ST = OFF_DS + 128 * 128 * 2;  // stages: Q, dO, lse2, dvec
   // dK/dV epilogue staging (128 rows x 64 fp32 as two 128-byte-swizzled boxes of 32 features):
   // d = 128 shares the dQ staging buffer; d = 64 has its own, which also stages dQ (d = 64 dQ is
   // [q][d] in TMEM, the same row-per-lane shape).  Same warps and barriers in both cases.
   static constexpr int EPI_BYTES = 128 * 64 * 4;
+  // The staging buffer is used as two 16 KB slots at d = 128 (two TMA operations in flight) and as
+  // one 32 KB slot at d = 64, where a dQ tile is two 16 KB boxes that leave together.
+  static constexpr int NSLOT = (D == 128) ? 2 : 1;
+  static constexpr int SLOT = EPI_BYTES / NSLOT;
   static constexpr int OFF_EPI = (D == 128) ? OFF_DS : OFF_ST + NSQ * STAGE;
   static constexpr int OFF_BAR = (D == 128) ? OFF_ST + NSQ * STAGE : OFF_EPI + EPI_BYTES;
   static constexpr int NW = 4;  // work-index ring depth
-  static constexpr int NBAR = 2 + 2 * NSQ + 11 + 2 * NW;
+  static constexpr int NBAR = 2 + 2 * NSQ + 13 + 2 * NW;
   // The dynamic shared window starts 1024-byte aligned (checked at run time),
-  // so no alignment slack is reserved: the D = 128 layout needs 231,656 bytes.
+  // so no alignment slack is reserved: the D = 128 layout needs 231,672 bytes.
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 4 * NW;
   static_assert(SMEM <= 232448, "shared memory per block");
   static_assert(OFF_EPI % 1024 == 0 && OFF_ST % 1024 == 0 && STAGE % 1024 == 0, "128-byte swizzle alignment");
@@ -123,9 +128,9 @@ __global__ void __launch_bounds__(448, 1)
   uint64_t* dkdv_full = dq_free + 1;
   uint64_t* dkdv_free = dkdv_full + 1;
   uint64_t* mma_drain = dkdv_free + 1;
-  uint64_t* stg_ready = mma_drain + 1;  // the staging buffer holds a dQ or dK/dV piece
-  uint64_t* stg_free = stg_ready + 1;   // its reduction has read the staging buffer
-  uint64_t* sched_full = stg_free + 1;  // [NW] the producer wrote the next work index
+  uint64_t* stg_ready = mma_drain + 1;  // [2] a staging slot holds a dQ or dK/dV box
+  uint64_t* stg_free = stg_ready + 2;   // [2] the slot's TMA operation has read it
+  uint64_t* sched_full = stg_free + 2;  // [NW] the producer wrote the next work index
   uint64_t* sched_empty = sched_full + C::NW;  // [NW] every other role has read it
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBAR);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -150,8 +155,10 @@ __global__ void __launch_bounds__(448, 1)
     mbar_init(dkdv_full, 1);
     mbar_init(dkdv_free, 4);
     mbar_init(mma_drain, 1);
-    mbar_init(stg_ready, 4);
-    mbar_init(stg_free, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(stg_ready + s, 4);  // one arrival per drain warp
+      mbar_init(stg_free + s, 1);
+    }
     for (int s = 0; s < C::NW; ++s) {
       mbar_init(sched_full + s, 1);
       mbar_init(sched_empty + s, 1 + 8 + 4);  // the MMA thread, the 8 softmax and 4 drain warps
@@ -456,7 +463,41 @@ __global__ void __launch_bounds__(448, 1)
     const int quad = warp & 3;
     const int t = quad * 32 + lane;
     const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
-    uint32_t it = 0, unit_iter = 0, hs = 0;  // hs: uses of the staging buffer (dQ halves, dK/dV pieces)
+    // Staging: each use of a slot stages one piece and thread 0 issues its TMA operations.  With two
+    // 16 KB slots (d = 128: a quarter of a dQ^T tile, one [128 rows][32 fp32] box of dK/dV, or one
+    // bf16 [128 rows][64] box of a directly stored dK/dV) the slots are used in turn and two
+    // operations are in flight: after issuing use n, thread 0 waits only until use n - 1 has read
+    // its slot and then frees that slot.  With one 32 KB slot (d = 64: a dQ tile or 64 dK/dV features
+    // as two [128 rows][32 fp32] boxes) thread 0 waits until the use has read the slot.  stg_ready[s]
+    // needs all four drain warps and stg_free[s] completes only after the use (two slots: the next
+    // use) has been issued, so neither parity wait can skip a phase.
+    uint32_t it = 0, unit_iter = 0, n_stg = 0;  // n_stg: uses of the staging slots
+    uint8_t* const stg_base = smem + (C::DQ_T ? C::OFF_DS : C::OFF_EPI);
+    auto stg_acquire = [&]() -> uint8_t* {  // warp-wide: the slot of use n_stg, once it is free
+      const uint32_t s = C::NSLOT == 2 ? n_stg & 1 : 0;
+      const uint32_t k = C::NSLOT == 2 ? n_stg >> 1 : n_stg;  // earlier uses of this slot
+      if (k >= 1 && !mbar_wait_warp(stg_free + s, (k - 1) & 1, guard, kErrTimeoutEpilogue)) return nullptr;
+      return stg_base + s * C::SLOT;
+    };
+    auto stg_ready_sync = [&]() -> bool {  // warp-wide, after this warp has written its rows
+      const uint32_t s = C::NSLOT == 2 ? n_stg & 1 : 0;
+      fence_async_smem();
+      mbar_arrive_warp(stg_ready + s);
+      return mbar_wait_warp(stg_ready + s, (C::NSLOT == 2 ? n_stg >> 1 : n_stg) & 1, guard, kErrTimeoutEpilogue);
+    };
+    auto stg_done = [&]() {  // after thread 0 has issued the use's TMA operations
+      if (t == 0) {
+        bulk_commit_group();
+        if (C::NSLOT == 1) {
+          bulk_wait_group_read0();
+          mbar_arrive(stg_free);
+        } else if (n_stg >= 1) {
+          bulk_wait_group_read1();
+          mbar_arrive(stg_free + ((n_stg & 1) ^ 1));
+        }
+      }
+      ++n_stg;
+    };
     bool ok = true;
     for (uint32_t wi = 0; ok; ++wi) {
       const int w = take_work(wi, kErrTimeoutEpilogue);
@@ -471,62 +512,55 @@ __global__ void __launch_bounds__(448, 1)
       for (int e = 0; e < ne && ok; ++e) {
         const int qt = qt_next;
         if (e + 1 < ne) qt_next = p.entries[2 * (e0 + rotated(e + 1, rot, ne))];
+        const int qrow = qt * 128 - (int)p.q0;  // first row of the q tile in the query-side buffers
         for (int hh = 0; hh < G; ++hh, ++it) {
           const int h = g * G + hh;
           if (!mbar_wait_warp(dq_full, it & 1, guard, kErrTimeoutEpilogue)) { ok = false; break; }
           tc_fence_after();
           if (C::DQ_T) {
-            // Lane t holds feature t of dQ^T (one column per q row).  Each half of the tile (64 q rows)
-            // is staged row-major [q][d] in the dedicated buffer and added to the accumulator by one TMA
-            // bulk reduction; thread 0 releases the buffer once the reduction has read it.  stg_ready
-            // needs every drain thread and stg_free follows it, so neither parity wait can skip a phase.
-            float* stg = reinterpret_cast<float*>(smem + C::OFF_DS);
-            if (hs > 0 && !mbar_wait_warp(stg_free, (hs - 1) & 1, guard, kErrTimeoutEpilogue)) { ok = false; break; }
+            // Lane t holds feature t of dQ^T (one column per q row).  Each quarter of the tile (32 q
+            // rows) is staged row-major [q][d] in one slot and added to the accumulator by one TMA
+            // bulk reduction.  The first two quarters go through the slots, the last two are held in
+            // registers, so R2 is released once the first two are staged.
 #pragma unroll 1
-            for (int c = 0; c < 2; ++c) {
+            for (int c = 0; c < 2 && ok; ++c) {
               float v[32];
               tmem_ld32(lane_base + C::COL_DQ + 32 * c, v);
+              float* stg = reinterpret_cast<float*>(stg_acquire());
+              if (!stg) { ok = false; break; }
 #pragma unroll
-              for (int e2 = 0; e2 < 32; ++e2) stg[(32 * c + e2) * 128 + t] = v[e2] * p.scale;
+              for (int e2 = 0; e2 < 32; ++e2) stg[e2 * 128 + t] = v[e2] * p.scale;
+              if (!stg_ready_sync()) { ok = false; break; }
+              if (t == 0) tma_reduce_add_3d(&tmDQ, stg, 0, h, qrow + 32 * c);
+              stg_done();
             }
-            fence_async_smem();
-            mbar_arrive_warp(stg_ready);
+            if (!ok) break;
             float v2[32], v3[32];
             tmem_ld32(lane_base + C::COL_DQ + 64, v2);
             tmem_ld32(lane_base + C::COL_DQ + 96, v3);
             tc_fence_before();
             mbar_arrive_warp(dq_free);  // all of dQ^T is in registers or staged: R2 may take the next dP^T
-            if (!mbar_wait_warp(stg_ready, hs & 1, guard, kErrTimeoutEpilogue)) { ok = false; break; }
-            if (t == 0) {
-              tma_reduce_add_3d(&tmDQ, stg, 0, h, qt * 128 - (int)p.q0);
-              bulk_commit_group();
-              bulk_wait_group_read0();
-              mbar_arrive(stg_free);
-            }
-            ++hs;
-            if (!mbar_wait_warp(stg_free, (hs - 1) & 1, guard, kErrTimeoutEpilogue)) { ok = false; break; }
+            float* stg = reinterpret_cast<float*>(stg_acquire());
+            if (!stg) { ok = false; break; }
 #pragma unroll
-            for (int e2 = 0; e2 < 32; ++e2) {
-              stg[e2 * 128 + t] = v2[e2] * p.scale;
-              stg[(32 + e2) * 128 + t] = v3[e2] * p.scale;
-            }
-            fence_async_smem();
-            mbar_arrive_warp(stg_ready);
-            if (!mbar_wait_warp(stg_ready, hs & 1, guard, kErrTimeoutEpilogue)) { ok = false; break; }
-            if (t == 0) {
-              tma_reduce_add_3d(&tmDQ, stg, 0, h, qt * 128 - (int)p.q0 + 64);
-              bulk_commit_group();
-              bulk_wait_group_read0();
-              mbar_arrive(stg_free);
-            }
-            ++hs;
-            continue;
+            for (int e2 = 0; e2 < 32; ++e2) stg[e2 * 128 + t] = v2[e2] * p.scale;
+            if (!stg_ready_sync()) { ok = false; break; }
+            if (t == 0) tma_reduce_add_3d(&tmDQ, stg, 0, h, qrow + 64);
+            stg_done();
+            stg = reinterpret_cast<float*>(stg_acquire());
+            if (!stg) { ok = false; break; }
+#pragma unroll
+            for (int e2 = 0; e2 < 32; ++e2) stg[e2 * 128 + t] = v3[e2] * p.scale;
+            if (!stg_ready_sync()) { ok = false; break; }
+            if (t == 0) tma_reduce_add_3d(&tmDQ, stg, 0, h, qrow + 96);
+            stg_done();
           } else {
             // Lane t holds q row t of dQ (D = 64 features).  The tile is staged, times the softmax
-            // scale, as two 128-byte-swizzled boxes [128 rows][32 fp32] in the epilogue buffer (the
-            // same layout and barriers as the dK/dV epilogue) and added by two TMA bulk reductions.
-            uint8_t* epi = smem + C::OFF_EPI;
-            if (hs > 0 && !mbar_wait_warp(stg_free, (hs - 1) & 1, guard, kErrTimeoutEpilogue)) { ok = false; break; }
+            // scale, as two 128-byte-swizzled boxes [128 rows][32 fp32] (the same layout as the
+            // dK/dV epilogue) in the one slot and added by two TMA bulk reductions.
+            static_assert(C::DQ_T || C::NSLOT == 1, "d = 64 stages a dQ tile in one 32 KB slot");
+            uint8_t* b = stg_acquire();
+            if (!b) { ok = false; break; }
             float v0[32], v1[32];
             tmem_ld32(lane_base + C::COL_DQ, v0);
             tmem_ld32(lane_base + C::COL_DQ + 32, v1);
@@ -535,24 +569,19 @@ __global__ void __launch_bounds__(448, 1)
 #pragma unroll
             for (int c16 = 0; c16 < 8; ++c16) {
               const uint32_t off = sw128_offset(t, c16);
-              st_shared_v4(smem_u32(epi + off), __float_as_uint(v0[4 * c16] * p.scale),
+              st_shared_v4(smem_u32(b + off), __float_as_uint(v0[4 * c16] * p.scale),
                            __float_as_uint(v0[4 * c16 + 1] * p.scale), __float_as_uint(v0[4 * c16 + 2] * p.scale),
                            __float_as_uint(v0[4 * c16 + 3] * p.scale));
-              st_shared_v4(smem_u32(epi + C::EPI_BYTES / 2 + off), __float_as_uint(v1[4 * c16] * p.scale),
+              st_shared_v4(smem_u32(b + C::EPI_BYTES / 2 + off), __float_as_uint(v1[4 * c16] * p.scale),
                            __float_as_uint(v1[4 * c16 + 1] * p.scale), __float_as_uint(v1[4 * c16 + 2] * p.scale),
                            __float_as_uint(v1[4 * c16 + 3] * p.scale));
             }
-            fence_async_smem();
-            mbar_arrive_warp(stg_ready);
-            if (!mbar_wait_warp(stg_ready, hs & 1, guard, kErrTimeoutEpilogue)) { ok = false; break; }
+            if (!stg_ready_sync()) { ok = false; break; }
             if (t == 0) {
-              tma_reduce_add_3d(&tmDQ, epi, 0, h, qt * 128 - (int)p.q0);
-              tma_reduce_add_3d(&tmDQ, epi + C::EPI_BYTES / 2, 32, h, qt * 128 - (int)p.q0);
-              bulk_commit_group();
-              bulk_wait_group_read0();
-              mbar_arrive(stg_free);
+              tma_reduce_add_3d(&tmDQ, b, 0, h, qrow);
+              tma_reduce_add_3d(&tmDQ, b + C::EPI_BYTES / 2, 32, h, qrow);
             }
-            ++hs;
+            stg_done();
           }
         }
       }
@@ -560,20 +589,19 @@ __global__ void __launch_bounds__(448, 1)
       if (!mbar_wait_warp(dkdv_full, unit_iter & 1, guard, kErrTimeoutEpilogue)) break;
       tc_fence_after();
       // This unit's dK (times the softmax scale left out of dS) and dV leave TMEM 64 features at a
-      // time: lane t holds row t and stages it into the epilogue buffer, and thread 0 issues the TMA.
-      // A kv tile with other units adds its partial to the fp32 accumulators: two 128-byte-swizzled
-      // boxes [128 rows][32 fp32] reduced into them (rows past N hold zeros: their keys and values
-      // were loaded as zeros and all their pairs are masked).  A kv tile with no other unit (direct)
-      // is final: one 128-byte-swizzled box [128 rows][64 bf16] stored to the bf16 output.
+      // time: lane t holds row t and stages it, and thread 0 issues the TMA.  A kv tile with other
+      // units adds its partial to the fp32 accumulators: two 128-byte-swizzled boxes [128 rows][32
+      // fp32] reduced into them (rows past N hold zeros: their keys and values were loaded as zeros
+      // and all their pairs are masked).  A kv tile with no other unit (direct) is final: one
+      // 128-byte-swizzled box [128 rows][64 bf16] stored to the bf16 output.
       const bool direct = p.kv_direct[(kt * 128 - (int)p.kv0) >> 7] != 0;
-      uint8_t* epi = smem + C::OFF_EPI;
+      const int row = kt * 128 - (int)p.kv0;  // first row of the kv tile in the key/value-side buffers
       constexpr int NCH = 2 * (D / 64);
 #pragma unroll 1
-      for (int m = 0; m < NCH; ++m) {
+      for (int m = 0; m < NCH && ok; ++m) {
         const int which = m / (D / 64), cb = m % (D / 64);
         const uint32_t col = (which == 0 ? C::COL_DK : C::COL_DV) + 64 * cb;
         const float f = which == 0 ? p.scale : 1.f;
-        if (hs > 0 && !mbar_wait_warp(stg_free, (hs - 1) & 1, guard, kErrTimeoutEpilogue)) { ok = false; break; }
         float v0[32], v1[32];
         tmem_ld32(lane_base + col, v0);
         tmem_ld32(lane_base + col + 32, v1);
@@ -582,41 +610,42 @@ __global__ void __launch_bounds__(448, 1)
           mbar_arrive_warp(dkdv_free);
         }
         if (direct) {
+          uint8_t* b = stg_acquire();
+          if (!b) { ok = false; break; }
 #pragma unroll
           for (int c16 = 0; c16 < 8; ++c16) {
             const float* v = c16 < 4 ? v0 + 8 * c16 : v1 + 8 * (c16 - 4);
-            st_shared_v4(smem_u32(epi + sw128_offset(t, c16)), pack_bf16x2(v[0] * f, v[1] * f),
+            st_shared_v4(smem_u32(b + sw128_offset(t, c16)), pack_bf16x2(v[0] * f, v[1] * f),
                          pack_bf16x2(v[2] * f, v[3] * f), pack_bf16x2(v[4] * f, v[5] * f),
                          pack_bf16x2(v[6] * f, v[7] * f));
           }
+          if (!stg_ready_sync()) { ok = false; break; }
+          if (t == 0) tma_store_3d(which == 0 ? &tmDK : &tmDV, b, 64 * cb, g, row);
+          stg_done();
         } else {
+          const int row0 = (which == 0 ? 0 : (int)p.n_pad_kv) + row;
+          // two slots: one box per use; one slot: both boxes in one use
+          constexpr int PER_USE = C::NSLOT == 2 ? 1 : 2;
+#pragma unroll 1
+          for (int c = 0; c < 2 && ok; c += PER_USE) {
+            uint8_t* b = stg_acquire();
+            if (!b) { ok = false; break; }
 #pragma unroll
-          for (int c16 = 0; c16 < 8; ++c16) {
-            const uint32_t off = sw128_offset(t, c16);
-            st_shared_v4(smem_u32(epi + off), __float_as_uint(v0[4 * c16] * f), __float_as_uint(v0[4 * c16 + 1] * f),
-                         __float_as_uint(v0[4 * c16 + 2] * f), __float_as_uint(v0[4 * c16 + 3] * f));
-            st_shared_v4(smem_u32(epi + C::EPI_BYTES / 2 + off), __float_as_uint(v1[4 * c16] * f),
-                         __float_as_uint(v1[4 * c16 + 1] * f), __float_as_uint(v1[4 * c16 + 2] * f),
-                         __float_as_uint(v1[4 * c16 + 3] * f));
+            for (int k = 0; k < PER_USE; ++k) {
+              const float* v = c + k == 0 ? v0 : v1;
+#pragma unroll
+              for (int c16 = 0; c16 < 8; ++c16)
+                st_shared_v4(smem_u32(b + k * (C::EPI_BYTES / 2) + sw128_offset(t, c16)),
+                             __float_as_uint(v[4 * c16] * f), __float_as_uint(v[4 * c16 + 1] * f),
+                             __float_as_uint(v[4 * c16 + 2] * f), __float_as_uint(v[4 * c16 + 3] * f));
+            }
+            if (!stg_ready_sync()) { ok = false; break; }
+            if (t == 0)
+              for (int k = 0; k < PER_USE; ++k)
+                tma_reduce_add_3d(&tmDKV, b + k * (C::EPI_BYTES / 2), 64 * cb + 32 * (c + k), g, row0);
+            stg_done();
           }
         }
-        fence_async_smem();
-        mbar_arrive_warp(stg_ready);
-        if (!mbar_wait_warp(stg_ready, hs & 1, guard, kErrTimeoutEpilogue)) { ok = false; break; }
-        if (t == 0) {
-          const int row = kt * 128 - (int)p.kv0;  // first row of the kv tile in the key/value-side buffers
-          if (direct) {
-            tma_store_3d(which == 0 ? &tmDK : &tmDV, epi, 64 * cb, g, row);
-          } else {
-            const int row0 = (which == 0 ? 0 : (int)p.n_pad_kv) + row;
-            tma_reduce_add_3d(&tmDKV, epi, 64 * cb, g, row0);
-            tma_reduce_add_3d(&tmDKV, epi + C::EPI_BYTES / 2, 64 * cb + 32, g, row0);
-          }
-          bulk_commit_group();
-          bulk_wait_group_read0();
-          mbar_arrive(stg_free);
-        }
-        ++hs;
       }
       if (!ok) break;
       ++unit_iter;
