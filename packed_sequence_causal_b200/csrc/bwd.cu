@@ -485,7 +485,7 @@ __global__ void __launch_bounds__(448, 1)
       mbar_arrive_warp(stg_ready + s);
       return mbar_wait_warp(stg_ready + s, (C::NSLOT == 2 ? n_stg >> 1 : n_stg) & 1, guard, kErrTimeoutEpilogue);
     };
-    auto stg_done = [&]() {  // after thread 0 has issued the use's TMA operations
+    auto stg_done = [&]() {  // warp-wide, after thread 0 has issued the use's TMA operations
       if (t == 0) {
         bulk_commit_group();
         if (C::NSLOT == 1) {
@@ -496,6 +496,7 @@ __global__ void __launch_bounds__(448, 1)
           mbar_arrive(stg_free + ((n_stg & 1) ^ 1));
         }
       }
+      __syncwarp();  // the warp is converged again before its next warp-collective TMEM load
       ++n_stg;
     };
     bool ok = true;
