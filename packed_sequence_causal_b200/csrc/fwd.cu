@@ -408,7 +408,7 @@ struct Fwd2Cfg {
   static constexpr int OFF_V = OFF_K + NS * KBYTES;
   static constexpr int OFF_BAR = OFF_V + NS * VBYTES;
   static constexpr int NW = 4;  // work-index ring depth (dynamic order)
-  static constexpr int NBAR = 2 + 4 * NS + 2 + 2 + 2 + 2 + 2 * NW;
+  static constexpr int NBAR = 2 + 4 * NS + 2 + 2 + 2 + 2 + 2 * NW + 4;
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 4 * NW;
   static constexpr int THREADS = 320;
   static constexpr uint32_t COL_O = 256;
@@ -440,6 +440,8 @@ __global__ void __launch_bounds__(320, 1)
   uint64_t* mma_drain = o_done + 1;
   uint64_t* sched_full = mma_drain + 1;        // [NW] the producer wrote the next work index
   uint64_t* sched_empty = sched_full + C::NW;  // [NW] the MMA thread and the 8 softmax warps read it
+  uint64_t* s_loaded = sched_empty + C::NW;    // [2] d = 64: the softmax has read all of S
+  uint64_t* pv_done = s_loaded + 2;            // [2] d = 64: the tile's PV has completed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBAR);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* sched_w = reinterpret_cast<volatile int*>(smem + C::OFF_BAR + C::NBAR * 8 + 16);  // [NW]
@@ -449,6 +451,12 @@ __global__ void __launch_bounds__(320, 1)
   // Softmax-to-MMA handoffs: one arrival per warp at d = 64, one per thread at d = 128 (measured:
   // per-warp arrivals made the d = 64 forward 1.3% faster and the d = 128 forward 0.8% slower).
   constexpr bool kPWarp = D == 64;
+  // Early S (d = 64): TMEM has 128 columns beyond S0, S1, O0 and O1, so each tile's P (packed bf16,
+  // 64 columns) gets a region of its own, [384 + 64 * tile, +64), instead of going over S.  The next S
+  // then needs neither P's columns nor the PV: it is issued as soon as the softmax has read all of S,
+  // and the softmax finds it ready instead of waiting for the PV and the next S to run.  The softmax
+  // writes the next P once the PV that read the previous one has completed.
+  constexpr bool kEarlyS = D == 64 && !CTA2;
   auto softmax_arrive = [](uint64_t* bar) {
     if constexpr (kPWarp)
       mbar_arrive_warp(bar);
@@ -480,6 +488,8 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(s_full + b, 1);
       mbar_init(p_full + b, CTA2 ? 256 : kPWarp ? 4 : 128);  // per softmax warp (d = 64) or thread
       mbar_init(p_half + b, CTA2 ? 256 : kPWarp ? 4 : 128);
+      mbar_init(s_loaded + b, kPWarp ? 4 : 128);
+      mbar_init(pv_done + b, 1);
     }
     mbar_init(o_done, 1);
     mbar_init(mma_drain, 1);
@@ -654,14 +664,15 @@ __global__ void __launch_bounds__(320, 1)
       };
       auto issue_pv = [&](int tile, uint32_t it, bool first, int part) {  // O_tile += P_tile V_it (half), P from TMEM
         const uint64_t dVs = sdesc_off(dV, (it % C::NS) * C::VBYTES);
+        const uint32_t colP = kEarlyS ? 384u + 64u * tile : 128u * tile;
 #pragma unroll
         for (int kk = 4 * part; kk < 4 * part + 4; ++kk) {
           const uint64_t bd = sdesc_off(dVs, kk * 2048);
           if constexpr (CTA2)
-            mma_bf16_tmem_a_pair(tmem + C::COL_O + D * tile, tmem + 128 * tile + kk * 8, bd, idesc_pv,
+            mma_bf16_tmem_a_pair(tmem + C::COL_O + D * tile, tmem + colP + kk * 8, bd, idesc_pv,
                                  (first && kk == 0) ? 0u : 1u);
           else
-            mma_bf16_tmem_a(tmem + C::COL_O + D * tile, tmem + 128 * tile + kk * 8, bd, idesc_pv,
+            mma_bf16_tmem_a(tmem + C::COL_O + D * tile, tmem + colP + kk * 8, bd, idesc_pv,
                             (first && kk == 0) ? 0u : 1u);
         }
       };
@@ -686,6 +697,43 @@ __global__ void __launch_bounds__(320, 1)
         commit(k_empty + (kc + LPS - 1) % C::NS);
         kc += LPS;
         for (int j = 0; j < ic; ++j, ++tile_iter, vc += LPS) {
+          if constexpr (kEarlyS) {
+            // Per tile: the first PV half, the next S once the softmax has read all of S (it signals
+            // p_half, then s_loaded, then p_full), the second PV half.
+            const bool more = j + 1 < ic;
+            const uint32_t g = tile_iter;
+            if (!wait_v(vc) || !wait_p(p_half + 0, g & 1)) { ok = false; break; }
+            tc_fence_after();
+            issue_pv(0, vc, j == 0, 0);
+            if (more) {
+              if (!mbar_wait(s_loaded + 0, g & 1, guard, kErrTimeoutMma) || !wait_k(kc)) { ok = false; break; }
+              tc_fence_after();
+              issue_s(0, kc);
+              if (KVS) commit(k_empty + kc % C::NS);
+            }
+            if (!wait_p(p_full + 0, g & 1)) { ok = false; break; }
+            tc_fence_after();
+            issue_pv(0, vc, j == 0, 1);
+            commit(pv_done + 0);
+            if (KVS) commit(v_empty + vc % C::NS);
+            if ((KVS && !wait_v(vc + 1)) || !wait_p(p_half + 1, g & 1)) { ok = false; break; }
+            tc_fence_after();
+            issue_pv(1, vc + LPS - 1, j == 0, 0);
+            if (more) {
+              if (!mbar_wait(s_loaded + 1, g & 1, guard, kErrTimeoutMma)) { ok = false; break; }
+              if (KVS && !wait_k(kc + 1)) { ok = false; break; }
+              tc_fence_after();
+              issue_s(1, kc + LPS - 1);
+              commit(k_empty + (kc + LPS - 1) % C::NS);
+              kc += LPS;
+            }
+            if (!wait_p(p_full + 1, g & 1)) { ok = false; break; }
+            tc_fence_after();
+            issue_pv(1, vc + LPS - 1, j == 0, 1);
+            commit(pv_done + 1);
+            commit(v_empty + (vc + LPS - 1) % C::NS);
+            continue;
+          }
           if (!wait_v(vc)) { ok = false; break; }
           if (!wait_p(p_half + 0, tile_iter & 1)) { ok = false; break; }
           tc_fence_after();
@@ -738,6 +786,7 @@ __global__ void __launch_bounds__(320, 1)
     const int r = quad * 32 + lane;
     const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
     const uint32_t colS = 128 * tile, colO = C::COL_O + D * tile;
+    const uint32_t colP = kEarlyS ? 384u + 64u * tile : colS;  // P: own region (early S) or over S
     uint32_t tile_iter = 0, unit_iter = 0;
     const float sl2 = p.scale_log2;
     bool ok = true;
@@ -773,7 +822,17 @@ __global__ void __launch_bounds__(320, 1)
         for (int e = 0; e < 4; ++e) mx8[e] = fmaxf(mx8[e], mx8[e + 4]);
         const float mx = fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3]));
         const float m_tile = mx * sl2;
-        // s_full of this tile also means the previous PV into O has completed.
+        // s_full of this tile also means the previous PV into O has completed -- except with early S,
+        // where S_g is issued before the second half of PV_{g-1}: there the previous PV is waited for
+        // here, before O is rescaled or P_g written over P_{g-1} (S_g was issued after PV_{g-2}, so
+        // the parity wait cannot be a phase behind).
+        if (kEarlyS && j > 0) {
+          if (!mbar_wait_warp(pv_done + tile, (tile_iter - 1) & 1, guard, kErrTimeoutSoftmax)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+        }
         const bool grow = m_tile > m + 8.0f;
         const float alpha = grow ? ex2(m - m_tile) : 1.f;
         if (j > 0 && __any_sync(0xffffffffu, grow && l > 0.f)) {
@@ -800,6 +859,10 @@ __global__ void __launch_bounds__(320, 1)
           float sh[64];
           tmem_ld32(lane_base + colS + 64 * half, sh);
           tmem_ld32(lane_base + colS + 64 * half + 32, sh + 32);
+          if (kEarlyS && half == 1) {  // all of S has been read: the next S may be written
+            tc_fence_before();
+            softmax_arrive(s_loaded + tile);
+          }
           if (tag != 0) {
             const int c_lo = row_lo - kt * 128 - 64 * half, c_hi = row_hi - kt * 128 - 64 * half;
 #pragma unroll
@@ -813,7 +876,7 @@ __global__ void __launch_bounds__(320, 1)
             rs4[e & 3] += p0 + p1;
             pk[e] = pack_bf16x2(p0, p1);
           }
-          tmem_st32_u(lane_base + colS + 32 * half, pk);  // P over the S columns already read
+          tmem_st32_u(lane_base + colP + 32 * half, pk);  // P: over the S columns already read, or its own region
           if (half == 0) {  // PV over kv rows 0..63 may start while the second half is computed
             tc_fence_before();
             if constexpr (CTA2)
