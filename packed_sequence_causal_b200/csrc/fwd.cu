@@ -380,7 +380,8 @@ __global__ void __launch_bounds__(192, 1)
 //
 // Threads: warp 0 TMA, warp 1 MMA, warps 2..5 softmax of tile 0 (head 2p),
 // warps 6..9 softmax of tile 1 (head 2p+1).
-// TMEM columns: S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [256+D,256+2D).
+// TMEM columns: S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [256+D,256+2D); at D = 64 also
+// P0 [384,448) and P1 [448,512) (P has columns of its own there; at D = 128 it goes over S).
 //
 // CTA2 = true (D = 128, GQA group a multiple of 4): a cluster of two CTAs takes one q tile of
 // four query heads of a kv group, two per CTA, and runs every MMA as one two-CTA tcgen05.mma
