@@ -142,6 +142,24 @@ def test_large_scores(lens, hq, hkv, nchunks, seed, scale):
     assert_close(dv, rdv, "dV (large scores)")
 
 
+@pytest.mark.parametrize("d", [64, 128])
+def test_running_max_grows_along_the_kv_walk(d):
+    """Keys of the long document scaled per kv tile by factors from 1 to 4 in a scrambled order, with
+    logits about 3x the usual spread: a q tile's running max keeps jumping by more than 2^8 between
+    kv steps of one unit, so the forward's lazy O rescale runs at later kv steps -- where, at d = 64,
+    the next S has already been issued and the rescale first waits for the previous PV."""
+    b = workloads.custom_batch([1500, 300], 4, 2, d, seed=71, with_do=False)
+    tile = torch.arange(b.k.shape[0]) // 128
+    factor = 1.0 + 3.0 * ((tile * 5) % 11).float() / 10.0
+    factor[1500:] = 1.0
+    b.k = (b.k.float() * factor[:, None, None]).to(torch.bfloat16)
+    r = Run(b, 1, 0.35)
+    o, lse = r.fwd()
+    ro, rl = oracle.attn_fwd(b.q, b.k, b.v, b.cu_seqlens, r.scale)
+    assert_close(o, ro, "O (growing running max)")
+    assert_lse(lse, rl, "LSE (growing running max)")
+
+
 def test_empty_batch_is_a_no_op():
     plan = sap.sap_plan([0], 0, 1)
     z = torch.zeros((0, 2, 64), dtype=torch.bfloat16, device="cuda")
